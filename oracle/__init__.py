@@ -1,0 +1,407 @@
+"""CPU oracle for the diffusion-LM noising-plus-loss path.
+
+TEST INFRASTRUCTURE ONLY.  Only the test suite, the package entry point's
+``smoke()`` check and the CPU-baseline leg of ``bench.py`` may import this
+module.  The product path never does, and this module imports nothing from
+the product package: the two share no code.  The only module both sides use
+is ``dlm_inputs`` (seeded synthetic inputs; none of the method's arithmetic).
+
+Scalar loops (hash, corruption, per-row CE in double) are in
+``dlm_oracle.c``; this file orchestrates them and holds the row plan, the
+weights and the reductions, written in numpy float64.
+
+Sources (page title, section):
+  [LLaDA]   "LLaDA-8B-MDLM-LoRA", Training table, row "Objective".
+  [Axolotl] "Native diffusion language-model training": model table
+            (noise, alignment, objective per model); "Packed training";
+            "Adapters, merging and inference" (Cut Cross Entropy: full-vocab
+            CE from hidden states, aligned targets, plain linear head).
+  [Gemma]   "diffusiongemma-26B-A4B-it-ALWAYS-THINK", Finetuning notes.
+
+Readings where the pages are silent (each listed in the design notes):
+  * loss normaliser for absorbing noise = number of non-pad tokens N;
+  * shifted rows: row i scores token i+1 of the same unit; each unit's last
+    row is unscored; position 0 may be corrupted but no row scores it;
+  * uniform canvas: every non-pad canvas target is scored, mean over them;
+  * encoder AR: row i scores token i+1 of the same unit, mean over pairs;
+  * the softmax runs over the whole vocabulary, mask-id column included.
+
+Pins: every function here is checked, in ``tests/test_oracle_*.py``, against
+something other than itself (published SplitMix64 vectors, a sequential
+re-derivation, closed forms, finite differences, a textbook log-softmax,
+binomial/chi-square statistics).  The end-to-end loss value has no worked
+example on the pages: parity unpinned for the whole-pipeline number itself
+(its parts are pinned).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+ABSORBING, UNIFORM = 0, 1
+ALIGNED, SHIFTED = 0, 1
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        u64, i64, i32, f32 = ctypes.c_uint64, ctypes.c_int64, ctypes.c_int32, ctypes.c_float
+        vp = ctypes.c_void_p
+        L.dlmo_splitmix64_at.restype = u64
+        L.dlmo_splitmix64_at.argtypes = [u64, u64]
+        L.dlmo_counter.restype = u64
+        L.dlmo_counter.argtypes = [ctypes.c_uint32, ctypes.c_uint32, ctypes.c_uint32]
+        L.dlmo_sample_t.restype = None
+        L.dlmo_sample_t.argtypes = [u64, i32, i32, f32, vp, vp]
+        L.dlmo_corrupt.restype = ctypes.c_int
+        L.dlmo_corrupt.argtypes = [i32, i32, vp, vp, i64, vp, vp, i32, i32, i32, u64, vp, vp]
+        for name in ("dlmo_ce_rows_bf16", "dlmo_ce_rows_f64"):
+            f = getattr(L, name)
+            f.restype = None
+            f.argtypes = [vp, i64, i32, i64, vp, vp, vp, vp]
+        for name in ("dlmo_grad_rows_bf16", "dlmo_grad_rows_f64"):
+            f = getattr(L, name)
+            f.restype = None
+            f.argtypes = [vp, i64, i32, i64, vp, vp, vp, vp, vp]
+        L.dlmo_bf16_to_f64.restype = None
+        L.dlmo_bf16_to_f64.argtypes = [vp, i64, vp]
+        _lib = L
+    return _lib
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --------------------------------------------------------------------------
+# Layout of tokens into units (sequences or packed documents)
+# --------------------------------------------------------------------------
+@dataclass
+class Layout:
+    """n_units sequences of seq_len tokens (cu_seqlens None), or n_units
+    packed documents delimited by cu_seqlens [n_units+1]; pad_mask [n_tokens]
+    with 1 = pad, or None."""
+    n_units: int
+    seq_len: int
+    cu_seqlens: Optional[np.ndarray]
+    pad_mask: Optional[np.ndarray]
+
+    @property
+    def n_tokens(self) -> int:
+        if self.cu_seqlens is None:
+            return self.n_units * self.seq_len
+        return int(self.cu_seqlens[-1])
+
+    def unit_of_token(self) -> np.ndarray:
+        n = self.n_tokens
+        if self.cu_seqlens is None:
+            return np.arange(n, dtype=np.int64) // self.seq_len
+        unit = np.empty(n, dtype=np.int64)
+        cu = self.cu_seqlens
+        for u in range(self.n_units):
+            unit[cu[u]:cu[u + 1]] = u
+        return unit
+
+    def nonpad(self) -> np.ndarray:
+        if self.pad_mask is None:
+            return np.ones(self.n_tokens, dtype=bool)
+        return self.pad_mask == 0
+
+
+# --------------------------------------------------------------------------
+# Hash, time draw, corruption  (C loops)
+# --------------------------------------------------------------------------
+def splitmix64_at(seed: int, counter: int) -> int:
+    return int(lib().dlmo_splitmix64_at(seed, counter))
+
+
+def counter(stream: int, unit: int, pos: int) -> int:
+    return int(lib().dlmo_counter(stream, unit, pos))
+
+
+def sample_t(seed: int, n_units: int, mode: int, eps: float):
+    """[LLaDA] absorbing: t ~ U(0,1), p = (1-eps) t + eps.
+    [Gemma] uniform: t ~ U(eps,1), p = t.  Returns float32 (t, p)."""
+    t = np.zeros(n_units, np.float32)
+    p = np.zeros(n_units, np.float32)
+    lib().dlmo_sample_t(seed, n_units, mode, ctypes.c_float(eps), _p(t), _p(p))
+    return t, p
+
+
+def corrupt(layout: Layout, clean: np.ndarray, p: np.ndarray, mode: int,
+            mask_id: int, vocab: int, seed: int):
+    """[LLaDA]/[Gemma] seeded corruption; returns (noisy int32, corrupted uint8)."""
+    clean = np.ascontiguousarray(clean, np.int32)
+    p = np.ascontiguousarray(p, np.float32)
+    n = layout.n_tokens
+    noisy = np.zeros(n, np.int32)
+    corr = np.zeros(n, np.uint8)
+    cu = None if layout.cu_seqlens is None else np.ascontiguousarray(layout.cu_seqlens, np.int32)
+    pm = None if layout.pad_mask is None else np.ascontiguousarray(layout.pad_mask, np.uint8)
+    rc = lib().dlmo_corrupt(layout.n_units, layout.seq_len, _p(cu), _p(pm), n, _p(clean),
+                            _p(p), mode, mask_id, vocab, seed, _p(noisy), _p(corr))
+    if rc != 0:
+        raise ValueError("inconsistent layout")
+    return noisy, corr
+
+
+# --------------------------------------------------------------------------
+# Row plan: which logits row is scored, against which target, with what weight
+# --------------------------------------------------------------------------
+@dataclass
+class RowPlan:
+    target: np.ndarray   # int64 [rows], -1 = unscored
+    unit: np.ndarray     # int64 [rows]
+    weight: np.ndarray   # float64 [rows], 0 on unscored rows
+
+
+def plan_diffusion(layout: Layout, clean: np.ndarray, corrupted: Optional[np.ndarray],
+                   p: Optional[np.ndarray], mode: int, align: int) -> RowPlan:
+    """Diffusion term.  Row i scores token j = i (aligned) or j = i+1 of the
+    same unit (shifted; [Axolotl] model table: Dream's logit i predicts token
+    i+1).  The target must be a non-pad token; absorbing noise additionally
+    requires it to be corrupted ([LLaDA]: CE on masked tokens).
+      absorbing: weight = 1 / (p_unit * N), N = non-pad tokens in the call.
+      uniform:   weight = 1 / (number of scored canvas rows)  (mean, [Gemma]).
+    """
+    n = layout.n_tokens
+    unit = layout.unit_of_token()
+    nonpad = layout.nonpad()
+    target = np.full(n, -1, np.int64)
+    weight = np.zeros(n, np.float64)
+    if align == ALIGNED:
+        j = np.arange(n)
+        ok = nonpad.copy()
+    else:
+        j = np.arange(n) + 1
+        ok = np.zeros(n, bool)
+        ok[:-1] = (unit[1:] == unit[:-1]) & nonpad[1:]
+        j = np.minimum(j, n - 1)
+    if mode == ABSORBING:
+        ok &= corrupted[j].astype(bool)
+    target[ok] = clean[j[ok]]
+    if mode == ABSORBING:
+        N = int(nonpad.sum())
+        if N > 0:
+            weight[ok] = 1.0 / (p[unit[ok]].astype(np.float64) * N)
+    else:
+        cnt = int(ok.sum())
+        if cnt > 0:
+            weight[ok] = 1.0 / cnt
+    return RowPlan(target, unit, weight)
+
+
+def plan_encoder(layout: Layout, clean: np.ndarray, lam: float) -> RowPlan:
+    """[Gemma] encoder AR term: plain causal next-token CE over the clean full
+    sequence.  Row i scores token i+1 of the same unit (non-pad); weight =
+    lam / (number of such pairs)."""
+    n = layout.n_tokens
+    unit = layout.unit_of_token()
+    nonpad = layout.nonpad()
+    ok = np.zeros(n, bool)
+    ok[:-1] = (unit[1:] == unit[:-1]) & nonpad[1:]
+    target = np.full(n, -1, np.int64)
+    target[:-1][ok[:-1]] = clean[1:][ok[:-1]]
+    weight = np.zeros(n, np.float64)
+    cnt = int(ok.sum())
+    if cnt > 0:
+        weight[ok] = lam / cnt
+    return RowPlan(target, unit, weight)
+
+
+# --------------------------------------------------------------------------
+# Per-row CE and gradient over a logits matrix (C loops, double)
+# --------------------------------------------------------------------------
+def ce_rows(logits: np.ndarray, vocab: int, rows: np.ndarray, targets: np.ndarray):
+    """(lse, ce) in double for the listed rows.  `logits` is a 2-D uint16
+    array of bf16 bit patterns [rows_total, ld] or a 2-D float64 array."""
+    rows = np.ascontiguousarray(rows, np.int64)
+    targets = np.ascontiguousarray(targets, np.int32)
+    n = rows.shape[0]
+    lse = np.zeros(n, np.float64)
+    ce = np.zeros(n, np.float64)
+    if n == 0:
+        return lse, ce
+    assert logits.flags.c_contiguous
+    ld = logits.shape[1]
+    if logits.dtype == np.uint16:
+        lib().dlmo_ce_rows_bf16(_p(logits), ld, vocab, n, _p(rows), _p(targets), _p(lse), _p(ce))
+    elif logits.dtype == np.float64:
+        lib().dlmo_ce_rows_f64(_p(logits), ld, vocab, n, _p(rows), _p(targets), _p(lse), _p(ce))
+    else:
+        raise TypeError(logits.dtype)
+    return lse, ce
+
+
+def grad_rows(logits: np.ndarray, vocab: int, rows: np.ndarray, targets: np.ndarray,
+              coef: np.ndarray, lse: np.ndarray) -> np.ndarray:
+    """coef_k * (softmax(row_k) - onehot(target_k)) in double, [n, vocab]."""
+    rows = np.ascontiguousarray(rows, np.int64)
+    targets = np.ascontiguousarray(targets, np.int32)
+    coef = np.ascontiguousarray(coef, np.float64)
+    lse = np.ascontiguousarray(lse, np.float64)
+    n = rows.shape[0]
+    out = np.zeros((n, vocab), np.float64)
+    if n == 0:
+        return out
+    ld = logits.shape[1]
+    if logits.dtype == np.uint16:
+        lib().dlmo_grad_rows_bf16(_p(logits), ld, vocab, n, _p(rows), _p(targets), _p(coef),
+                                  _p(lse), _p(out))
+    else:
+        lib().dlmo_grad_rows_f64(_p(logits), ld, vocab, n, _p(rows), _p(targets), _p(coef),
+                                 _p(lse), _p(out))
+    return out
+
+
+def bf16_to_f64(a: np.ndarray) -> np.ndarray:
+    a = np.ascontiguousarray(a, np.uint16)
+    out = np.empty(a.shape, np.float64)
+    lib().dlmo_bf16_to_f64(_p(a), a.size, _p(out))
+    return out
+
+
+# --------------------------------------------------------------------------
+# The loss over one logits tensor, and the two-term uniform loss
+# --------------------------------------------------------------------------
+@dataclass
+class TermResult:
+    plan: RowPlan
+    rows: np.ndarray      # scored row indices
+    lse: np.ndarray       # per scored row
+    ce: np.ndarray        # per scored row
+    row_loss: np.ndarray  # [rows_total] weight * ce, 0 on unscored rows
+
+
+def term(logits: np.ndarray, vocab: int, plan: RowPlan) -> TermResult:
+    rows = np.nonzero(plan.target >= 0)[0]
+    lse, ce = ce_rows(logits, vocab, rows, plan.target[rows])
+    row_loss = np.zeros(plan.target.shape[0], np.float64)
+    row_loss[rows] = plan.weight[rows] * ce
+    return TermResult(plan, rows, lse, ce, row_loss)
+
+
+def reduce_units(n_units: int, *terms: TermResult):
+    """Per-unit sums of weight*ce (per-example reduction, [Axolotl]
+    "Objective and recurrence options") and the total loss."""
+    unit_loss = np.zeros(n_units, np.float64)
+    for tr in terms:
+        np.add.at(unit_loss, tr.plan.unit, tr.row_loss)
+    return float(unit_loss.sum()), unit_loss
+
+
+def term_grad(logits: np.ndarray, vocab: int, tr: TermResult, rows: np.ndarray,
+              grad_scale: float) -> np.ndarray:
+    """dlogits for the listed rows (scored or not), double [len(rows), vocab]:
+    grad_scale * weight * (softmax - onehot) on scored rows, exact zeros else."""
+    rows = np.asarray(rows, np.int64)
+    out = np.zeros((rows.shape[0], vocab), np.float64)
+    scored = tr.plan.target[rows] >= 0
+    if scored.any():
+        sel = rows[scored]
+        # lse of the selected rows, looked up from the scored list
+        pos = np.searchsorted(tr.rows, sel)
+        lse = tr.lse[pos]
+        coef = grad_scale * tr.plan.weight[sel]
+        out[scored] = grad_rows(logits, vocab, sel, tr.plan.target[sel], coef, lse)
+    return out
+
+
+def loss_absorbing(layout: Layout, logits: np.ndarray, vocab: int, clean: np.ndarray,
+                   corrupted: np.ndarray, p: np.ndarray, align: int):
+    plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, align)
+    tr = term(logits, vocab, plan)
+    loss, unit_loss = reduce_units(layout.n_units, tr)
+    return loss, unit_loss, tr
+
+
+def loss_uniform(canvas: Layout, logits: np.ndarray, canvas_clean: np.ndarray,
+                 encoder: Layout, enc_logits: np.ndarray, enc_clean: np.ndarray,
+                 vocab: int, lam: float, align: int = ALIGNED):
+    """[Gemma] total = canvas CE (mean) + lam * encoder AR CE (mean)."""
+    pc = plan_diffusion(canvas, canvas_clean, None, None, UNIFORM, align)
+    pe = plan_encoder(encoder, enc_clean, lam)
+    tc = term(logits, vocab, pc)
+    te = term(enc_logits, vocab, pe)
+    loss, unit_loss = reduce_units(canvas.n_units, tc, te)
+    return loss, unit_loss, tc, te
+
+
+# --------------------------------------------------------------------------
+# Fused lm_head (Cut Cross Entropy style): logits = H W^T never rounded
+# --------------------------------------------------------------------------
+def linear_logits(H_rows: np.ndarray, W: np.ndarray, chunk: int = 16384) -> np.ndarray:
+    """Z = H_rows W^T in double from bf16 inputs (library matmul as one step).
+    H_rows: uint16 [n, D] (bf16 bits); W: uint16 [V, D]."""
+    Hd = bf16_to_f64(H_rows)
+    V = W.shape[0]
+    Z = np.empty((Hd.shape[0], V), np.float64)
+    for v0 in range(0, V, chunk):
+        Wd = bf16_to_f64(W[v0:v0 + chunk])
+        Z[:, v0:v0 + chunk] = Hd @ Wd.T
+    return Z
+
+
+def linear_loss(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
+                corrupted: np.ndarray, p: np.ndarray, grad_scale: float = 1.0,
+                want_grads: bool = True):
+    """[Axolotl] CCE path, aligned absorbing only.  Rows of H at masked
+    positions form Z = H_M W^T in double; CE and weights as for the unfused
+    loss; dZ = grad_scale * w * (softmax - onehot); dH_M = dZ W, dW = dZ^T H_M,
+    other rows of dH exactly zero."""
+    plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, ALIGNED)
+    rows = np.nonzero(plan.target >= 0)[0]
+    V, D = W.shape
+    Z = linear_logits(H[rows], W)
+    local = np.arange(rows.shape[0], dtype=np.int64)
+    lse, ce = ce_rows(Z, V, local, plan.target[rows])
+    row_loss = np.zeros(plan.target.shape[0], np.float64)
+    row_loss[rows] = plan.weight[rows] * ce
+    unit_loss = np.zeros(layout.n_units, np.float64)
+    np.add.at(unit_loss, plan.unit, row_loss)
+    out = dict(loss=float(unit_loss.sum()), unit_loss=unit_loss, rows=rows, lse=lse, ce=ce,
+               plan=plan)
+    if want_grads:
+        dZ = grad_rows(Z, V, local, plan.target[rows], grad_scale * plan.weight[rows], lse)
+        del Z
+        Hd = bf16_to_f64(H[rows])
+        dH = np.zeros((H.shape[0], D), np.float64)
+        dW = np.zeros((V, D), np.float64)
+        chunk = 16384
+        for v0 in range(0, V, chunk):
+            Wd = bf16_to_f64(W[v0:v0 + chunk])
+            dH[rows] += dZ[:, v0:v0 + chunk] @ Wd
+            dW[v0:v0 + chunk] = dZ[:, v0:v0 + chunk].T @ Hd
+        out.update(dH=dH, dW=dW)
+    return out
+
+
+def linear_rows(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
+                corrupted: np.ndarray, p: np.ndarray, sample_rows: np.ndarray,
+                grad_scale: float = 1.0):
+    """Full-size spot check: for a few scored rows only, their CE, weight*ce
+    and their row of dH (which needs only that row's own softmax)."""
+    plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, ALIGNED)
+    sample_rows = np.asarray(sample_rows, np.int64)
+    assert (plan.target[sample_rows] >= 0).all()
+    V, D = W.shape
+    Z = linear_logits(H[sample_rows], W)
+    local = np.arange(sample_rows.shape[0], dtype=np.int64)
+    tgt = plan.target[sample_rows]
+    lse, ce = ce_rows(Z, V, local, tgt)
+    coef = grad_scale * plan.weight[sample_rows]
+    dZ = grad_rows(Z, V, local, tgt, coef, lse)
+    dH = np.zeros((sample_rows.shape[0], D), np.float64)
+    for v0 in range(0, V, 16384):
+        dH += dZ[:, v0:v0 + 16384] @ bf16_to_f64(W[v0:v0 + 16384])
+    return dict(ce=ce, lse=lse, weighted=plan.weight[sample_rows] * ce, dH=dH, plan=plan)
