@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Benchmark of the diffusion-LM noising-plus-loss hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+dlm_sample_t -> dlm_corrupt -> dlm_loss_fwd_bwd (fused forward + backward,
+bf16 dlogits for every row), all through the C ABI of libdlm.so.
+
+Default workload: the LLaDA-like absorbing-mask loss, B=1 L=4096 V=126464,
+aligned logits, clean-token logit +4, logits N(0, 3) bf16 (1.04 GB, larger
+than L2, so no flush between steps is needed).  Each timed step draws a new t
+(seed = 1000 + step), so the scored rows vary like in training.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Multi-GPU: replicas only (the path has no data exchange); every rank runs the
+same workload on its own GPU, timing is the max over ranks, value = scored
+tokens of all ranks / that time ("scaling": "weak").
+
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "diffusion-loss fwd+bwd scored tokens/s; achieved HBM GB/s vs B200 peak"
+UNIT = "scored tokens/s"
+DEFAULT_WORKLOAD = "abs_b1_l4096_v126464"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+CE_SOURCE = os.path.join(ROOT, "diffusion_lm_loss_b200", "csrc", "dlm_ce.cu")
+CE_PROFILE = os.path.join(ROOT, "profiles", "ce_cluster_abs_b1_l4096_v126464.md")
+
+
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def ce_traffic_ratio():
+    """DRAM bytes / algorithmic bytes of the CE kernel from the committed ncu
+    summary, or None when the kernel source changed since the capture."""
+    try:
+        txt = open(CE_PROFILE).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    m_r = re.search(r"traffic_over_algorithmic:\s*([0-9.]+)", txt)
+    if not (m_sha and m_r):
+        return None
+    sha = hashlib.sha256(open(CE_SOURCE, "rb").read()).hexdigest()
+    return float(m_r.group(1)) if sha == m_sha.group(1) else None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu=timestamp,{self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def mark_begin(self):
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t1 = datetime.datetime.now()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+            except ValueError:
+                continue
+            rows.append((ts, f))
+        inside = [r for r in rows if self.t0 and self.t1 and self.t0 <= r[0] <= self.t1]
+        use = inside or rows[len(rows) // 2:len(rows) // 2 + 1]
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1][2]) for r in use if r[1][2].replace(".", "").isdigit()]
+        smax = [float(r[1][3]) for r in use if r[1][3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, f in use:
+            for n, v in zip(names, f[6:10]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(use),
+                "samples_in_timed_region": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def algorithmic_ce_bytes(rows: int, scored: int, vocab: int) -> int:
+    """Bytes the weighted-CE fwd+bwd must move per launch: each scored row is
+    read once (2V) and every row's bf16 gradient written once (2V); plus the
+    row list (16 B) read and the per-row loss (4 B) written."""
+    return 2 * vocab * scored + 2 * vocab * rows + 20 * rows
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import dlm_inputs as di
+    import diffusion_lm_loss_b200 as dlm
+
+    rank, local_rank, world = env_rank()
+    if args.gpus != world:
+        if world == 1 and args.gpus > 1:
+            raise SystemExit("--gpus N>1 must be launched with torch.distributed.run (one rank per GPU)")
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    spec = di.WORKLOADS[args.workload]
+    if spec.kind != "loss":
+        raise SystemExit("the bench times the materialised-logits loss workloads")
+    case = di.make_case(spec, dev, seed=spec.data_seed + rank)
+    V = spec.vocab
+    mode, align = spec.mode, spec.align
+    B = spec.n_units
+    uniform = mode == di.UNIFORM
+    lay = dlm.make_layout(B, spec.seq_len)
+    enc_lay = dlm.make_layout(B, spec.prefix + spec.seq_len) if uniform else None
+    out = None
+
+    def step(seed, logits, clean, enc_logits=None, enc_clean=None, ev=None):
+        nonlocal out
+        t, p = dlm.sample_t(seed, B, mode, spec.eps)
+        _, corr = dlm.corrupt(lay, clean, p, mode, spec.mask_id, V, seed)
+        if ev is not None:
+            ev[0].record()
+        out = dlm.loss_fwd_bwd(lay, logits, V, clean, corr, p, mode, align,
+                               enc_layout=enc_lay, enc_logits=enc_logits, enc_ids=enc_clean,
+                               enc_ar_weight=spec.enc_ar_weight, out=out)
+        if ev is not None:
+            ev[1].record()
+        return corr
+
+    K, W = args.steps, args.warmup
+    for i in range(W):
+        step(10 + i, case.logits, case.clean, case.enc_logits, case.enc_clean)
+    torch.cuda.synchronize()
+
+    vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    loss_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark_begin()
+    t_start.record()
+    for i in range(K):
+        step(1000 + i, case.logits, case.clean, case.enc_logits, case.enc_clean, ev=loss_ev[i])
+    t_end.record()
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    loss_ms = sum(a.elapsed_time(b) for a, b in loss_ev) / K
+    clk = clocks.stop() if rank == 0 else None
+
+    # scored rows of the timed steps (recomputed outside the timed region)
+    scored = 0
+    rows = case.n_tokens + (B * (spec.prefix + spec.seq_len) if uniform else 0)
+    if uniform:
+        enc_pairs = B * (spec.prefix + spec.seq_len - 1)
+        scored = K * (case.n_tokens + enc_pairs) if align == di.ALIGNED else None
+    if not uniform or scored is None:
+        tot = torch.zeros((), dtype=torch.int64, device=dev)
+        for i in range(K):
+            t, p = dlm.sample_t(1000 + i, B, mode, spec.eps)
+            _, corr = dlm.corrupt(lay, case.clean, p, mode, spec.mask_id, V, 1000 + i)
+            if align == di.SHIFTED:
+                c = corr.view(B, spec.seq_len)[:, 1:]
+                tot += c.sum()
+            else:
+                tot += corr.sum(dtype=torch.int64)
+        scored = int(tot.item())
+
+    t_all = torch.tensor([ms, loss_ms], dtype=torch.float64, device=dev)
+    n_all = torch.tensor([scored], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_all, op=dist.ReduceOp.MAX)
+        dist.all_reduce(n_all, op=dist.ReduceOp.SUM)
+    ms, loss_ms = float(t_all[0]), float(t_all[1])
+    scored_all = float(n_all[0])
+    value = scored_all / (ms / 1e3)
+
+    # e2e: inputs from pinned host memory, H2D + step + D2H of the loss
+    e2e = None
+    if not args.no_e2e:
+        Ke = max(1, min(K, args.e2e_steps))
+        h_logits = case.logits.cpu().pin_memory()
+        h_clean = case.clean.cpu().pin_memory()
+        h_enc_logits = case.enc_logits.cpu().pin_memory() if uniform else None
+        h_enc_clean = case.enc_clean.cpu().pin_memory() if uniform else None
+        d_logits = torch.empty_like(case.logits)
+        d_clean = torch.empty_like(case.clean)
+        d_enc_logits = torch.empty_like(case.enc_logits) if uniform else None
+        d_enc_clean = torch.empty_like(case.enc_clean) if uniform else None
+        h_loss = torch.empty(Ke, dtype=torch.float32).pin_memory()
+        h2d = h_logits.numel() * 2 + h_clean.numel() * 4
+        if uniform:
+            h2d += h_enc_logits.numel() * 2 + h_enc_clean.numel() * 4
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+
+        def e2e_step(i):
+            d_logits.copy_(h_logits, non_blocking=True)
+            d_clean.copy_(h_clean, non_blocking=True)
+            if uniform:
+                d_enc_logits.copy_(h_enc_logits, non_blocking=True)
+                d_enc_clean.copy_(h_enc_clean, non_blocking=True)
+            step(1000 + i, d_logits, d_clean, d_enc_logits, d_enc_clean)
+            h_loss[i:i + 1].copy_(out.loss, non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s0.record()
+        for i in range(Ke):
+            e2e_step(i)
+        s1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e_ms = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        # the same seeds as the first Ke timed steps: scored rows in proportion
+        e2e_val = scored_all * (Ke / K) / (float(e_ms[0]) / 1e3)
+        e2e = {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": 4,
+               "steps": Ke, "ms_per_step": float(e_ms[0]) / Ke}
+        del d_logits, h_logits
+
+    hbm, _, peak_kind = peaks()
+    alg_bytes = algorithmic_ce_bytes(rows, scored / K if world == 1 else scored_all / world / K, V)
+    achieved = alg_bytes / (loss_ms / 1e3) / 1e9
+    ratio = ce_traffic_ratio()
+    roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": (ratio * alg_bytes) if ratio else None,
+            "kernel": "k_ce_cluster (timed as the whole dlm_loss_fwd_bwd call: plan + CE + reduce)",
+            "algorithmic_bytes_per_launch": alg_bytes, "launch_ms": loss_ms,
+            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
+            "frac_of_8TBps": achieved / 8000.0}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(spec)
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": spec.key, "description": spec.description, "global_batch": B * world,
+                   "seq_len": spec.seq_len, "vocab": V, "parallelism": f"replicas{world}",
+                   "l2": "inputs larger than L2 (logits %.2f GB per replica)" % (case.logits.numel() * 2 / 1e9),
+                   "scored_tokens": scored_all, "seeds": "t/corruption seed 1000+step"},
+        "roofline": roof, "cpu_baseline": cpu, "clocks": clk, "e2e": e2e,
+        "gpu_launches": 5 * K,
+    }
+    print(json.dumps(res), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_step(spec, case_cpu, seed, rows_sample):
+    """The oracle as it stands on the first `rows_sample` rows of each unit's
+    sequence: time draw, corruption, CE of the scored rows, gradient of all
+    rows.  Returns the number of scored rows."""
+    import numpy as np
+
+    import dlm_inputs as di
+    import oracle
+
+    B = spec.n_units
+    L = min(spec.seq_len, rows_sample)
+    lay = oracle.Layout(B, L, None, None)
+    clean = case_cpu.clean.view(B, spec.seq_len)[:, :L].reshape(-1).numpy()
+    x = di.bf16_bits(case_cpu.logits.view(B, spec.seq_len, -1)[:, :L].reshape(B * L, -1))
+    _, p = oracle.sample_t(seed, B, spec.mode, spec.eps)
+    if spec.mode == oracle.ABSORBING:
+        _, corr = oracle.corrupt(lay, clean, p, spec.mode, spec.mask_id, spec.vocab, seed)
+        loss, unit, tr = oracle.loss_absorbing(lay, x, spec.vocab, clean, corr, p, spec.align)
+        oracle.term_grad(x, spec.vocab, tr, np.arange(B * L), 1.0)
+        return int(tr.rows.shape[0])
+    raise SystemExit("reference arm: uniform workloads not wired")
+
+
+def _calibrated_rows(spec, per_step_s, cap=1024):
+    """Rows per sequence such that one oracle step takes about per_step_s."""
+    import dlm_inputs as di
+
+    probe = spec.scaled(seq_len=min(spec.seq_len, 16))
+    case = di.make_case(probe, "cpu")
+    oracle_step(probe, case, 0, probe.seq_len)          # first call builds / loads the oracle
+    t0 = time.perf_counter()
+    oracle_step(probe, case, 1, probe.seq_len)
+    per_row = (time.perf_counter() - t0) / (probe.seq_len * probe.n_units)
+    rows = int(per_step_s / max(per_row, 1e-9) / probe.n_units)
+    return max(4, min(spec.seq_len, cap, rows))
+
+
+def _oracle_threads():
+    return int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+
+
+def cpu_baseline(spec, budget_s=15.0, steps=3):
+    import dlm_inputs as di
+
+    rows = _calibrated_rows(spec, budget_s / steps)
+    sub = spec.scaled(seq_len=rows)
+    case = di.make_case(sub, "cpu")
+    t0 = time.perf_counter()
+    scored = 0
+    for i in range(steps):
+        scored += oracle_step(sub, case, 1000 + i, rows)
+    dt = time.perf_counter() - t0
+    return {"value": scored / dt, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"{steps} steps of the same workload cut to its first {rows} rows per "
+                      f"sequence ({spec.vocab}-wide rows; time draw, corruption, CE of the scored "
+                      f"rows, double-precision gradient of every row): {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on the machine's host
+    cores, each step a bounded sample of the workload sized so that the
+    whole run ends in about two minutes."""
+    rank, _, world = env_rank()
+    if rank != 0:
+        return
+    import dlm_inputs as di
+
+    spec = di.WORKLOADS[args.workload]
+    rows = _calibrated_rows(spec, 100.0 / (args.steps + args.warmup))
+    sub = spec.scaled(seq_len=rows)
+    case = di.make_case(sub, "cpu")
+    for i in range(args.warmup):
+        oracle_step(sub, case, 10 + i, rows)
+    t0 = time.perf_counter()
+    scored = 0
+    for i in range(args.steps):
+        scored += oracle_step(sub, case, 1000 + i, rows)
+    dt = time.perf_counter() - t0
+    val = scored / dt
+    sample = (f"each step: the workload cut to its first {rows} rows per sequence (V={spec.vocab}); "
+              f"the oracle's whole path (time draw, corruption, CE, double-precision gradient)")
+    res = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic",
+           "config": {"workload": spec.key, "description": spec.description,
+                      "global_batch": spec.n_units, "seq_len": rows, "vocab": spec.vocab,
+                      "parallelism": "cpu"},
+           "cpu_baseline": {"value": val, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,269 @@
+"""Python binding of the B200 diffusion-LM noising-plus-loss library.
+
+Argument marshalling only: every step runs in the CUDA kernels of
+``libdlm.so`` (built from ``csrc/`` for sm_100a); torch provides device
+memory and streams.  There is no CPU fallback -- importing this module
+without the built library, or calling it on a non-sm_100 device, raises.
+
+Two layers:
+  * ``lib()``: the raw C ABI through ctypes, functions named as in
+    ``include/dlm.h`` (``dlm_sample_t``, ``dlm_corrupt``,
+    ``dlm_loss_fwd_bwd``, ``dlm_linear_loss_fwd_bwd``, ...);
+  * tensor helpers with the same names minus the prefix (``sample_t``,
+    ``corrupt``, ``loss_fwd_bwd``, ``linear_loss_fwd_bwd``) that allocate
+    outputs and workspace with torch on the current device and call the ABI
+    on the current torch stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libdlm.so")
+
+ABSORBING, UNIFORM = 0, 1
+ALIGNED, SHIFTED = 0, 1
+
+DEV_BAD_TOKEN_ID = 0x1
+DEV_BAD_LAYOUT = 0x2
+DEV_WAIT_TIMEOUT = 0x4
+
+STATUS = {0: "DLM_OK", 1: "DLM_ERR_INVALID_ARGUMENT", 2: "DLM_ERR_UNSUPPORTED",
+          3: "DLM_ERR_WORKSPACE_TOO_SMALL", 4: "DLM_ERR_CUDA"}
+
+# every symbol include/dlm.h declares
+EXPORTS = ("dlm_status_string", "dlm_version", "dlm_sample_t", "dlm_corrupt",
+           "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_linear_loss_workspace_size",
+           "dlm_linear_loss_fwd_bwd", "dlm_get_device_status")
+
+
+class DlmError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Layout(ctypes.Structure):
+    """dlm_layout_t: n_units sequences of seq_len tokens (cu_seqlens NULL) or
+    n_units packed documents (cu_seqlens [n_units+1] int32 on the device);
+    pad_mask [n_tokens] uint8 on the device (1 = pad) or NULL."""
+    _fields_ = [("n_units", ctypes.c_int32), ("seq_len", ctypes.c_int32),
+                ("n_tokens", ctypes.c_int64), ("cu_seqlens", ctypes.c_void_p),
+                ("pad_mask", ctypes.c_void_p)]
+
+
+def make_layout(n_units: int, seq_len: int = 0, cu_seqlens: Optional[torch.Tensor] = None,
+                pad_mask: Optional[torch.Tensor] = None, n_tokens: Optional[int] = None) -> Layout:
+    if cu_seqlens is not None:
+        _check(cu_seqlens, torch.int32, "cu_seqlens")
+        if n_tokens is None:
+            raise ValueError("packed layouts need n_tokens (cu_seqlens lives on the device)")
+        cu = cu_seqlens.data_ptr()
+    else:
+        cu = None
+        n_tokens = n_units * seq_len if n_tokens is None else n_tokens
+    pm = None
+    if pad_mask is not None:
+        _check(pad_mask, torch.uint8, "pad_mask")
+        pm = pad_mask.data_ptr()
+    return Layout(n_units, seq_len, n_tokens, cu, pm)
+
+
+_lib = None
+
+
+def lib():
+    """The loaded C ABI (ctypes), with argument and return types declared."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built: run python -m diffusion_lm_loss_b200.build "
+                          "(there is no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, u64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64,
+                                  ctypes.c_float, ctypes.c_size_t)
+    lp = ctypes.POINTER(Layout)
+    L.dlm_status_string.restype = ctypes.c_char_p
+    L.dlm_status_string.argtypes = [ctypes.c_int]
+    L.dlm_version.restype = ctypes.c_int
+    L.dlm_version.argtypes = []
+    L.dlm_sample_t.restype = ctypes.c_int
+    L.dlm_sample_t.argtypes = [u64, i32, i32, f32, vp, vp, vp]
+    L.dlm_corrupt.restype = ctypes.c_int
+    L.dlm_corrupt.argtypes = [lp, vp, vp, i32, i32, i32, u64, vp, vp, vp, vp]
+    L.dlm_loss_workspace_size.restype = sz
+    L.dlm_loss_workspace_size.argtypes = [lp, lp]
+    L.dlm_loss_fwd_bwd.restype = ctypes.c_int
+    L.dlm_loss_fwd_bwd.argtypes = [lp, vp, i64, i32, vp, vp, vp, i32, i32, lp, vp, i64, vp, f32,
+                                   f32, vp, vp, vp, vp, vp, sz, vp]
+    L.dlm_linear_loss_workspace_size.restype = sz
+    L.dlm_linear_loss_workspace_size.argtypes = [lp, i32, i32]
+    L.dlm_linear_loss_fwd_bwd.restype = ctypes.c_int
+    L.dlm_linear_loss_fwd_bwd.argtypes = [lp, vp, vp, i32, i32, vp, vp, vp, f32, vp, vp, vp, vp,
+                                          vp, sz, vp]
+    L.dlm_get_device_status.restype = ctypes.c_int
+    L.dlm_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
+    _lib = L
+    return L
+
+
+def _check(t: torch.Tensor, dtype, name: str):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor (there is no CPU path)")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ok(code: int, where: str):
+    if code != 0:
+        raise DlmError(code, where)
+
+
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t
+
+
+# --------------------------------------------------------------------------
+# tensor helpers
+# --------------------------------------------------------------------------
+def sample_t(seed: int, n_units: int, mode: int = ABSORBING, eps: float = 1e-3,
+             device=None):
+    """(t, p): float32 [n_units] on the current (or given) CUDA device."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    t = torch.empty(n_units, dtype=torch.float32, device=dev)
+    p = torch.empty(n_units, dtype=torch.float32, device=dev)
+    _ok(lib().dlm_sample_t(seed, n_units, mode, eps, _ptr(t), _ptr(p), _stream()), "dlm_sample_t")
+    return t, p
+
+
+def corrupt(layout: Layout, clean_ids: torch.Tensor, p: torch.Tensor, mode: int = ABSORBING,
+            mask_id: int = 0, vocab: int = 0, seed: int = 0,
+            dev_status: Optional[torch.Tensor] = None):
+    """(noisy int32, corrupted uint8), same length as clean_ids."""
+    _check(clean_ids, torch.int32, "clean_ids")
+    _check(p, torch.float32, "p")
+    noisy = torch.empty_like(clean_ids)
+    corr = torch.empty(clean_ids.shape, dtype=torch.uint8, device=clean_ids.device)
+    _ok(lib().dlm_corrupt(ctypes.byref(layout), _ptr(clean_ids), _ptr(p), mode, mask_id, vocab, seed,
+                          _ptr(noisy), _ptr(corr), _ptr(dev_status), _stream()), "dlm_corrupt")
+    return noisy, corr
+
+
+@dataclass
+class LossOut:
+    loss: torch.Tensor            # float32 [1]
+    unit_loss: torch.Tensor       # float32 [n_units]
+    dlogits: torch.Tensor         # bf16, logits' shape
+    enc_dlogits: Optional[torch.Tensor]
+    workspace: torch.Tensor       # uint8; holds the device status word
+
+    def device_status(self) -> int:
+        return device_status(self.workspace)
+
+
+def loss_workspace_size(layout: Layout, enc_layout: Optional[Layout] = None) -> int:
+    return int(lib().dlm_loss_workspace_size(ctypes.byref(layout),
+                                             ctypes.byref(enc_layout) if enc_layout else None))
+
+
+def loss_fwd_bwd(layout: Layout, logits: torch.Tensor, vocab: int, clean_ids: torch.Tensor,
+                 corrupted: Optional[torch.Tensor], p: Optional[torch.Tensor],
+                 mode: int = ABSORBING, align: int = ALIGNED,
+                 enc_layout: Optional[Layout] = None, enc_logits: Optional[torch.Tensor] = None,
+                 enc_ids: Optional[torch.Tensor] = None, enc_ar_weight: float = 1.0,
+                 grad_scale: float = 1.0, out: Optional[LossOut] = None) -> LossOut:
+    """Weighted CE forward + backward (see dlm_loss_fwd_bwd).  logits: bf16
+    [rows, ld] (2-D, row stride ld >= vocab).  Reuses the buffers of `out`
+    when given (no allocation)."""
+    _check(logits, torch.bfloat16, "logits")
+    _check(clean_ids, torch.int32, "clean_ids")
+    if logits.dim() != 2 or logits.stride(1) != 1:
+        raise ValueError("logits must be 2-D with unit column stride")
+    ld = logits.stride(0)
+    enc_ld = 0
+    if enc_logits is not None:
+        _check(enc_logits, torch.bfloat16, "enc_logits")
+        _check(enc_ids, torch.int32, "enc_ids")
+        if enc_logits.dim() != 2 or enc_logits.stride(1) != 1:
+            raise ValueError("enc_logits must be 2-D with unit column stride")
+        enc_ld = enc_logits.stride(0)
+    dev = logits.device
+    if out is None:
+        ws = torch.empty(loss_workspace_size(layout, enc_layout), dtype=torch.uint8, device=dev)
+        out = LossOut(torch.empty(1, dtype=torch.float32, device=dev),
+                      torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
+                      torch.empty_like(logits),
+                      torch.empty_like(enc_logits) if enc_logits is not None else None, ws)
+    _ok(lib().dlm_loss_fwd_bwd(
+        ctypes.byref(layout), _ptr(logits), ld, vocab, _ptr(clean_ids), _ptr(corrupted), _ptr(p),
+        mode, align, ctypes.byref(enc_layout) if enc_layout is not None else None,
+        _ptr(enc_logits), enc_ld, _ptr(enc_ids), enc_ar_weight, grad_scale, _ptr(out.loss),
+        _ptr(out.unit_loss), _ptr(out.dlogits), _ptr(out.enc_dlogits), _ptr(out.workspace),
+        out.workspace.numel(), _stream()), "dlm_loss_fwd_bwd")
+    return out
+
+
+@dataclass
+class LinearOut:
+    loss: torch.Tensor
+    unit_loss: torch.Tensor
+    d_hidden: torch.Tensor
+    d_weight: Optional[torch.Tensor]
+    workspace: torch.Tensor
+
+    def device_status(self) -> int:
+        return device_status(self.workspace)
+
+
+def linear_loss_workspace_size(layout: Layout, d_model: int, vocab: int) -> int:
+    return int(lib().dlm_linear_loss_workspace_size(ctypes.byref(layout), d_model, vocab))
+
+
+def linear_loss_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: torch.Tensor,
+                        clean_ids: torch.Tensor, corrupted: torch.Tensor, p: torch.Tensor,
+                        grad_scale: float = 1.0, want_d_weight: bool = True,
+                        out: Optional[LinearOut] = None) -> LinearOut:
+    """Fused lm_head + absorbing aligned loss (see dlm_linear_loss_fwd_bwd)."""
+    _check(hidden, torch.bfloat16, "hidden")
+    _check(weight, torch.bfloat16, "weight")
+    if not (hidden.is_contiguous() and weight.is_contiguous()):
+        raise ValueError("hidden and weight must be contiguous")
+    T, D = hidden.shape
+    V, D2 = weight.shape
+    if D != D2:
+        raise ValueError("hidden / weight d_model mismatch")
+    dev = hidden.device
+    if out is None:
+        ws = torch.empty(linear_loss_workspace_size(layout, D, V), dtype=torch.uint8, device=dev)
+        out = LinearOut(torch.empty(1, dtype=torch.float32, device=dev),
+                        torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
+                        torch.empty_like(hidden),
+                        torch.empty_like(weight) if want_d_weight else None, ws)
+    _ok(lib().dlm_linear_loss_fwd_bwd(
+        ctypes.byref(layout), _ptr(hidden), _ptr(weight), D, V, _ptr(clean_ids), _ptr(corrupted),
+        _ptr(p), grad_scale, _ptr(out.loss), _ptr(out.unit_loss), _ptr(out.d_hidden),
+        _ptr(out.d_weight), _ptr(out.workspace), out.workspace.numel(), _stream()),
+        "dlm_linear_loss_fwd_bwd")
+    return out
+
+
+def device_status(workspace: torch.Tensor) -> int:
+    """Device status word of a loss workspace (synchronises the stream)."""
+    v = ctypes.c_uint32(0)
+    _ok(lib().dlm_get_device_status(_ptr(workspace), ctypes.byref(v), _stream()),
+        "dlm_get_device_status")
+    return int(v.value)

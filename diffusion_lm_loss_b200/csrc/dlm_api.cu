@@ -1,0 +1,54 @@
+// dlm_api.cu -- status strings, version, the device check and the
+// device-status read-back of the C ABI.
+#include <mutex>
+
+#include "dlm_host.h"
+
+namespace dlm {
+
+dlm_status_t check_device() {
+    // compute capability 10.0 (B200) only; cached per device ordinal
+    static std::mutex mu;
+    static int known[64];   // 0 = unknown, 1 = ok, 2 = unsupported
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return DLM_ERR_CUDA; }
+    if (dev < 0 || dev >= 64) return DLM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> g(mu);
+    if (known[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return DLM_ERR_CUDA;
+        }
+        known[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    return known[dev] == 1 ? DLM_OK : DLM_ERR_UNSUPPORTED;
+}
+
+}  // namespace dlm
+
+extern "C" const char* dlm_status_string(dlm_status_t status) {
+    switch (status) {
+        case DLM_OK: return "DLM_OK";
+        case DLM_ERR_INVALID_ARGUMENT: return "DLM_ERR_INVALID_ARGUMENT";
+        case DLM_ERR_UNSUPPORTED: return "DLM_ERR_UNSUPPORTED";
+        case DLM_ERR_WORKSPACE_TOO_SMALL: return "DLM_ERR_WORKSPACE_TOO_SMALL";
+        case DLM_ERR_CUDA: return "DLM_ERR_CUDA";
+        default: return "DLM_ERR_UNKNOWN";
+    }
+}
+
+extern "C" int dlm_version(void) { return 100; }   // 0.1.0
+
+extern "C" dlm_status_t dlm_get_device_status(const void* workspace, uint32_t* host_status,
+                                              dlm_stream_t stream) {
+    if (!workspace || !host_status) return DLM_ERR_INVALID_ARGUMENT;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(host_status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+        cudaGetLastError();
+        return DLM_ERR_CUDA;
+    }
+    return DLM_OK;
+}

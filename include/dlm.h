@@ -1,0 +1,230 @@
+/*
+ * dlm.h -- C ABI of the B200 (sm_100a) diffusion-LM noising-plus-loss library.
+ *
+ * One training step of a native diffusion language model, between the clean
+ * token ids of a batch and the gradient of the loss with respect to the
+ * model's logits (or its hidden states and output head):
+ *
+ *   dlm_sample_t             per-sequence (or per-document) time t and mask
+ *                            probability p
+ *   dlm_corrupt              seeded corruption of the clean ids
+ *   dlm_loss_fwd_bwd         inverse-time weighted CE over the vocabulary at
+ *                            the corrupted positions, forward + backward, from
+ *                            materialised bf16 logits
+ *   dlm_linear_loss_fwd_bwd  the same loss from hidden states and a linear
+ *                            output head, logits never materialised
+ *
+ * The method (page title, section):
+ *   "LLaDA-8B-MDLM-LoRA", Training table, row "Objective": t ~ U(0,1) per
+ *       sequence, mask probability p = (1 - 1e-3) t + 1e-3, cross-entropy on
+ *       masked tokens divided by p.
+ *   "Native diffusion language-model training", model table: absorbing mask
+ *       with aligned logits (Nemotron) or shifted logits (Dream); uniform token
+ *       noise with a causal encoder (DiffusionGemma).  "Packed training":
+ *       documents stay isolated; positions restart at document boundaries.
+ *       "Adapters, merging and inference": Cut Cross Entropy computes the
+ *       full-vocabulary CE from hidden states without materialising logits,
+ *       aligned targets, plain linear head.
+ *   "diffusiongemma-26B-A4B-it-ALWAYS-THINK", Finetuning notes: total =
+ *       diffusion CE + encoder_loss_weight * encoder AR CE; canvas positions
+ *       replaced by uniform-random vocabulary ids at rate t ~ U(eps, 1).
+ *
+ * Conventions for every call
+ *   - All array arguments are DEVICE pointers owned by the caller, except the
+ *     dlm_layout_t structs themselves (host memory, read during the call).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronise, except dlm_get_device_status.
+ *   - The library allocates no device memory.  Scratch comes from a caller
+ *     workspace of at least dlm_*_workspace_size() bytes, 256-byte aligned.
+ *     A workspace may be reused by calls ordered on one stream; calls that
+ *     overlap on the GPU need separate workspaces.
+ *   - Host-checkable errors return before anything is enqueued.  Errors that
+ *     depend on device data (an id outside [0, vocab), a non-monotone
+ *     cu_seqlens, a bounded wait that ran out) set bits in a device status
+ *     word; the affected rows are treated as unscored and the call still
+ *     completes.  Read the word with dlm_get_device_status.
+ *   - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16).
+ *   - Requires compute capability 10.0 (B200); other devices get
+ *     DLM_ERR_UNSUPPORTED.
+ */
+#ifndef DLM_H_
+#define DLM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Symbols of this ABI are the only ones the shared library exports. */
+#if defined(__GNUC__)
+#define DLM_API __attribute__((visibility("default")))
+#else
+#define DLM_API
+#endif
+
+typedef enum dlm_status {
+    DLM_OK = 0,
+    DLM_ERR_INVALID_ARGUMENT = 1,
+    DLM_ERR_UNSUPPORTED = 2,
+    DLM_ERR_WORKSPACE_TOO_SMALL = 3,
+    DLM_ERR_CUDA = 4
+} dlm_status_t;
+
+/* noise process */
+enum { DLM_ABSORBING = 0, DLM_UNIFORM = 1 };
+/* logit alignment: row i scores token i, or token i+1 of the same unit */
+enum { DLM_ALIGNED = 0, DLM_SHIFTED = 1 };
+
+/* bits of the device status word */
+#define DLM_DEV_BAD_TOKEN_ID   0x1u  /* a scored target id outside [0, vocab)      */
+#define DLM_DEV_BAD_LAYOUT     0x2u  /* cu_seqlens not 0..n_tokens non-decreasing  */
+#define DLM_DEV_WAIT_TIMEOUT   0x4u  /* a bounded on-chip wait gave up             */
+
+/* Opaque CUDA stream (ABI-compatible with cudaStream_t / CUstream). */
+typedef struct CUstream_st *dlm_stream_t;
+
+/* How tokens are grouped into units (the thing t is drawn for).
+ *   Dense:  cu_seqlens == NULL; n_units sequences of seq_len tokens each,
+ *           token i of the flattened [n_units, seq_len] array is position
+ *           i % seq_len of unit i / seq_len.  n_tokens = n_units * seq_len.
+ *   Packed: cu_seqlens = [n_units + 1] int32 document offsets (device),
+ *           cu_seqlens[0] = 0, non-decreasing, cu_seqlens[n_units] = n_tokens;
+ *           seq_len is ignored.  Positions restart at each document start.
+ *   pad_mask: [n_tokens] uint8 (device), 1 = padding, or NULL.  Pads are
+ *           never corrupted, never scored, and not counted in N.
+ * Limits: n_units < 2^24, positions < 2^31, n_tokens < 2^31. */
+typedef struct dlm_layout {
+    int32_t n_units;
+    int32_t seq_len;
+    int64_t n_tokens;
+    const int32_t *cu_seqlens;
+    const uint8_t *pad_mask;
+} dlm_layout_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+DLM_API const char *dlm_status_string(dlm_status_t status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+DLM_API int dlm_version(void);
+
+/* ------------------------------------------------------------------------
+ * dlm_sample_t -- time and mask probability per unit.
+ *   "LLaDA-8B-MDLM-LoRA", Training table, row "Objective" (absorbing):
+ *       t = u,                 p = (1 - eps) t + eps
+ *   "diffusiongemma-26B-A4B-it-ALWAYS-THINK", Finetuning notes (uniform):
+ *       t = (1 - eps) u + eps, p = t
+ * u = k / 2^24 where k = top 24 bits of SplitMix64 output number
+ * (counter + 1) from state `seed`, counter = unit << 32 (stream 0);
+ * fp32 arithmetic with one rounding per operation (c1 = 1 - eps first).
+ * t, p: [n_units] float (device, written).  mode: DLM_ABSORBING|DLM_UNIFORM.
+ * eps in [0, 1).  n_units = 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+DLM_API dlm_status_t dlm_sample_t(uint64_t seed, int32_t n_units, int32_t mode, float eps,
+                          float *t, float *p, dlm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * dlm_corrupt -- seeded corruption of clean ids ("LLaDA-8B-MDLM-LoRA",
+ * Training table, row "Objective"; "diffusiongemma-26B-A4B-it-ALWAYS-THINK",
+ * Finetuning notes; "Native diffusion language-model training", Packed
+ * training).  Per non-pad token at position `pos` of unit `u`:
+ *   corrupted = (float)(h1 >> 40) < p[u] * 2^24       (strict, exact fp32)
+ *   h1 = SplitMix64(seed, counter = 1 << 56 | u << 32 | pos)
+ *   absorbing: noisy = mask_id
+ *   uniform:   noisy = ((h2 >> 32) * vocab) >> 32,  h2 with stream 2 in place
+ *              of 1 -- a uniform id in [0, vocab), may equal the clean id.
+ * Pads keep their id and are never corrupted.  Uncorrupted tokens keep their
+ * clean id.  For uniform noise pass the canvas tokens only.
+ *   clean_ids [n_tokens] int32, p [n_units] float (from dlm_sample_t),
+ *   noisy_ids [n_tokens] int32 (written), corrupted [n_tokens] uint8 (written,
+ *   0/1), dev_status: a device uint32 that gets DLM_DEV_BAD_LAYOUT or'ed in
+ *   if cu_seqlens is inconsistent (may be NULL).
+ * mask_id is only read for absorbing noise; vocab only for uniform noise.
+ * ---------------------------------------------------------------------- */
+DLM_API dlm_status_t dlm_corrupt(const dlm_layout_t *layout, const int32_t *clean_ids,
+                         const float *p, int32_t mode, int32_t mask_id, int32_t vocab,
+                         uint64_t seed, int32_t *noisy_ids, uint8_t *corrupted,
+                         uint32_t *dev_status, dlm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * dlm_loss_fwd_bwd -- weighted CE over the vocabulary, forward + backward,
+ * from materialised bf16 logits.
+ *
+ * Rows and targets (diffusion term, one logits row per token of `layout`):
+ *   row i scores token j = i (DLM_ALIGNED) or j = i + 1 of the same unit
+ *   (DLM_SHIFTED; a unit's last row is unscored); j must be non-pad.
+ *   absorbing: only corrupted j are scored, weight w = 1 / (p[unit] * N),
+ *              N = number of non-pad tokens of `layout`.
+ *   uniform:   every such j is scored, w = 1 / (number of scored rows).
+ * Encoder AR term (uniform only, enc_logits != NULL): one row per token of
+ *   `enc_layout`; row i scores enc_ids[i+1] of the same unit (non-pad),
+ *   w = enc_ar_weight / (number of such rows).  enc_layout.n_units must equal
+ *   layout.n_units (unit u of the canvas is unit u of the encoder sequence).
+ * Per scored row r with target y:  ce_r = logsumexp(x_r) - x_r[y] over the
+ *   full vocabulary (mask-id column included).
+ * Outputs:
+ *   loss[0]          = sum_r w_r ce_r                               (float)
+ *   unit_loss[u]     = the same sum over unit u's rows (may be NULL)
+ *   dlogits[r, v]    = grad_scale * w_r * (softmax(x_r)_v - [v == y_r]) on
+ *                      scored rows, exactly 0 on every other row; bf16, same
+ *                      layout as logits; every element of [rows, vocab] is
+ *                      written (columns vocab..ld-1 are not touched).
+ *   enc_dlogits      = the same for the encoder rows.
+ * logits: [layout.n_tokens rows, ld] bf16, row stride ld >= vocab elements.
+ * enc_logits: [enc_layout.n_tokens, enc_ld] bf16.  clean_ids / enc_ids:
+ * int32 clean ids.  corrupted: from dlm_corrupt (absorbing; ignored for
+ * uniform).  p: [n_units] from dlm_sample_t (absorbing; ignored for uniform).
+ * Reductions run in a fixed order: results are bitwise reproducible.
+ * Fast path when vocab, ld, enc_ld are multiples of 8 and the logits /
+ * dlogits pointers are 16-byte aligned; any other shape takes a slower
+ * general kernel with the same results.
+ * ---------------------------------------------------------------------- */
+DLM_API size_t dlm_loss_workspace_size(const dlm_layout_t *layout, const dlm_layout_t *enc_layout);
+
+DLM_API dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t *layout, const uint16_t *logits, int64_t ld,
+                              int32_t vocab, const int32_t *clean_ids, const uint8_t *corrupted,
+                              const float *p, int32_t mode, int32_t align,
+                              const dlm_layout_t *enc_layout, const uint16_t *enc_logits,
+                              int64_t enc_ld, const int32_t *enc_ids, float enc_ar_weight,
+                              float grad_scale, float *loss, float *unit_loss,
+                              uint16_t *dlogits, uint16_t *enc_dlogits,
+                              void *workspace, size_t workspace_bytes, dlm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * dlm_linear_loss_fwd_bwd -- the absorbing, aligned loss above with
+ * logits = hidden @ weight^T formed tile by tile on the tensor cores and never
+ * written to memory ("Native diffusion language-model training", Adapters,
+ * merging and inference: Cut Cross Entropy, plain linear head, aligned).
+ *   hidden [n_tokens, d_model] bf16 row-major; weight [vocab, d_model] bf16
+ *   row-major.  Logits are formed in fp32 from the bf16 inputs.
+ *   d_hidden [n_tokens, d_model] bf16 (written; rows of unscored tokens = 0).
+ *   d_weight [vocab, d_model] bf16 (written), or NULL to skip it.
+ *   loss / unit_loss as for dlm_loss_fwd_bwd (unit_loss may be NULL).
+ * Requires d_model % 64 == 0 and vocab % 8 == 0, 16-byte aligned pointers.
+ * ---------------------------------------------------------------------- */
+DLM_API size_t dlm_linear_loss_workspace_size(const dlm_layout_t *layout, int32_t d_model,
+                                      int32_t vocab);
+
+DLM_API dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t *layout, const uint16_t *hidden,
+                                     const uint16_t *weight, int32_t d_model, int32_t vocab,
+                                     const int32_t *clean_ids, const uint8_t *corrupted,
+                                     const float *p, float grad_scale, float *loss,
+                                     float *unit_loss, uint16_t *d_hidden, uint16_t *d_weight,
+                                     void *workspace, size_t workspace_bytes,
+                                     dlm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * dlm_get_device_status -- copy the device status word of a loss workspace
+ * (first 4 bytes) to *host_status after the work queued on `stream`;
+ * synchronises `stream`.  Each dlm_loss_fwd_bwd / dlm_linear_loss_fwd_bwd
+ * call clears the word first, so it reports that call.
+ * ---------------------------------------------------------------------- */
+DLM_API dlm_status_t dlm_get_device_status(const void *workspace, uint32_t *host_status,
+                                   dlm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DLM_H_ */

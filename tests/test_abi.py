@@ -1,0 +1,106 @@
+"""The C-ABI library loads and exports every symbol include/dlm.h declares;
+host-side argument checks reject bad calls before anything touches a GPU
+(no compute calls here: these run without a device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+import diffusion_lm_loss_b200 as dlm
+from diffusion_lm_loss_b200 import build as dlm_build
+
+
+@pytest.fixture(scope="module")
+def L():
+    dlm_build.build()
+    return dlm.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "dlm.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dlm_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_four_path_calls():
+    names = declared_functions()
+    for n in ("dlm_sample_t", "dlm_corrupt", "dlm_loss_fwd_bwd", "dlm_linear_loss_fwd_bwd"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert set(names) == set(dlm.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+    # nothing else leaks out of the library (hidden visibility)
+    out = os.popen(f"nm -D --defined-only {dlm.LIB_PATH}").read()
+    exported = set(re.findall(r"\bT (dlm_[a-z0-9_]+)", out))
+    assert exported == set(names)
+
+
+def test_status_strings_and_version(L):
+    assert L.dlm_status_string(0) == b"DLM_OK"
+    assert L.dlm_status_string(3) == b"DLM_ERR_WORKSPACE_TOO_SMALL"
+    assert L.dlm_status_string(99) == b"DLM_ERR_UNKNOWN"
+    assert L.dlm_version() >= 100
+
+
+def test_host_side_rejections(L):
+    # these all fail argument validation before any device query or launch
+    assert L.dlm_sample_t(0, -1, 0, 1e-3, None, None, None) == 1
+    assert L.dlm_sample_t(0, 4, 7, 1e-3, None, None, None) == 1
+    assert L.dlm_sample_t(0, 4, 0, 1.5, None, None, None) == 1
+    assert L.dlm_sample_t(0, 0, 0, 1e-3, None, None, None) == 0           # no-op
+    bad = dlm.Layout(2, 10, 21, None, None)                              # 2*10 != 21
+    assert L.dlm_corrupt(ctypes.byref(bad), None, None, 0, 0, 0, 0, None, None, None, None) == 1
+    lay = dlm.Layout(2, 10, 20, None, None)
+    assert L.dlm_corrupt(ctypes.byref(lay), None, None, 0, 0, 0, 0, None, None, None, None) == 1
+    # loss: ld < vocab, bad mode, encoder with absorbing noise, small workspace
+    args = [ctypes.byref(lay), 16, 32, 32, 16, 16, 16, 0, 0, None, None, 0, None, 0.0, 1.0, 16,
+            None, 16, None, 256, 1 << 20, None]
+    a = list(args); a[2] = 16
+    assert L.dlm_loss_fwd_bwd(*a) == 1                                    # ld < vocab
+    a = list(args); a[7] = 5
+    assert L.dlm_loss_fwd_bwd(*a) == 1                                    # mode
+    a = list(args); a[8] = 9
+    assert L.dlm_loss_fwd_bwd(*a) == 1                                    # align
+    a = list(args); a[10] = 16
+    assert L.dlm_loss_fwd_bwd(*a) == 1                                    # encoder w/ absorbing
+    a = list(args); a[20] = 4
+    assert L.dlm_loss_fwd_bwd(*a) == 3                                    # workspace too small
+    a = list(args); a[19] = 100
+    assert L.dlm_loss_fwd_bwd(*a) == 1                                    # misaligned workspace
+
+
+def test_workspace_size_grows_with_rows(L):
+    a = dlm.Layout(1, 4096, 4096, None, None)
+    b = dlm.Layout(1, 8192, 8192, None, None)
+    sa = L.dlm_loss_workspace_size(ctypes.byref(a), None)
+    sb = L.dlm_loss_workspace_size(ctypes.byref(b), None)
+    assert sa > 4096 * 16 and sb > sa and sa % 256 == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises((ValueError, TypeError)):
+        dlm.corrupt(dlm.Layout(1, 4, 4, None, None), torch.zeros(4, dtype=torch.int32),
+                    torch.zeros(1, dtype=torch.float32))
+
+
+def test_oracle_and_product_share_no_code():
+    """Neither side imports the other; the oracle has no CUDA, the package no
+    oracle."""
+    pkg = os.path.join(ROOT, "diffusion_lm_loss_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt and "dlm_oracle" not in txt
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        if f.endswith((".py", ".c")):
+            txt = open(os.path.join(ROOT, "oracle", f)).read()
+            assert "diffusion_lm_loss_b200" not in txt and "dlm.h" not in txt
