@@ -37,14 +37,14 @@ STATUS = {0: "DLM_OK", 1: "DLM_ERR_INVALID_ARGUMENT", 2: "DLM_ERR_UNSUPPORTED",
           3: "DLM_ERR_WORKSPACE_TOO_SMALL", 4: "DLM_ERR_CUDA"}
 
 # every symbol include/dlm.h declares
-EXPORTS = ("dlm_status_string", "dlm_version", "dlm_sample_t", "dlm_corrupt",
+EXPORTS = ("dlm_status_string", "dlm_last_cuda_error", "dlm_version", "dlm_sample_t", "dlm_corrupt",
            "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_linear_loss_workspace_size",
            "dlm_linear_loss_fwd_bwd", "dlm_get_device_status")
 
 
 class DlmError(RuntimeError):
-    def __init__(self, code: int, where: str):
-        super().__init__(f"{where}: {STATUS.get(code, code)}")
+    def __init__(self, code: int, where: str, detail: str = ""):
+        super().__init__(f"{where}: {STATUS.get(code, code)}" + (f" [{detail}]" if detail else ""))
         self.code = code
 
 
@@ -91,6 +91,8 @@ def lib():
     lp = ctypes.POINTER(Layout)
     L.dlm_status_string.restype = ctypes.c_char_p
     L.dlm_status_string.argtypes = [ctypes.c_int]
+    L.dlm_last_cuda_error.restype = ctypes.c_char_p
+    L.dlm_last_cuda_error.argtypes = []
     L.dlm_version.restype = ctypes.c_int
     L.dlm_version.argtypes = []
     L.dlm_sample_t.restype = ctypes.c_int
@@ -130,7 +132,8 @@ def _stream():
 
 def _ok(code: int, where: str):
     if code != 0:
-        raise DlmError(code, where)
+        detail = lib().dlm_last_cuda_error().decode() if code == 4 else ""
+        raise DlmError(code, where, detail)
 
 
 def _bits(t: torch.Tensor) -> torch.Tensor:

@@ -47,18 +47,20 @@ def _stale(target, inputs):
     return any(os.path.getmtime(i) > t for i in inputs)
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = False,
+          lib_path: str = LIB, build_dir: str = BUILD, defines=()) -> str:
+    """Compile (incrementally) into lib_path; `defines` are extra -D flags."""
+    os.makedirs(build_dir, exist_ok=True)
     cc = nvcc()
     deps = _deps()
     objs = []
     jobs = []
     for src in _sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + deps):
-            cmd = [cc] + ARCH + NVCC_FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + \
-                  ["-c", src, "-o", obj]
+            cmd = [cc] + ARCH + NVCC_FLAGS + ["-D" + d for d in defines] + \
+                  (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", src, "-o", obj]
             jobs.append(cmd)
 
     def run(cmd):
@@ -74,11 +76,11 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     if ptxas_verbose:
         for l in logs:
             print(l)
-    if force or jobs or _stale(LIB, objs):
-        cmd = [cc] + ARCH + ["-shared", "-cudart", "static", "-o", LIB + ".tmp"] + objs
+    if force or jobs or _stale(lib_path, objs):
+        cmd = [cc] + ARCH + ["-shared", "-cudart", "static", "-o", lib_path + ".tmp"] + objs
         run(cmd)
-        os.replace(LIB + ".tmp", LIB)
-    return LIB
+        os.replace(lib_path + ".tmp", lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":

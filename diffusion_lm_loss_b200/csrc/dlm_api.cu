@@ -4,14 +4,24 @@
 
 #include "dlm_host.h"
 
+#include <cstdio>
+
 namespace dlm {
+
+static thread_local char g_last_error[256] = "";
+
+void record_cuda_error(cudaError_t e, const char* where) {
+    std::snprintf(g_last_error, sizeof g_last_error, "%s: %s (%s)", where, cudaGetErrorString(e),
+                  cudaGetErrorName(e));
+}
 
 dlm_status_t check_device() {
     // compute capability 10.0 (B200) only; cached per device ordinal
     static std::mutex mu;
     static int known[64];   // 0 = unknown, 1 = ok, 2 = unsupported
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return DLM_ERR_CUDA; }
+    cudaError_t e0 = cudaGetDevice(&dev);
+    if (e0 != cudaSuccess) { cudaGetLastError(); return cuda_status(e0, "cudaGetDevice"); }
     if (dev < 0 || dev >= 64) return DLM_ERR_UNSUPPORTED;
     std::lock_guard<std::mutex> g(mu);
     if (known[dev] == 0) {
@@ -41,14 +51,14 @@ extern "C" const char* dlm_status_string(dlm_status_t status) {
 
 extern "C" int dlm_version(void) { return 100; }   // 0.1.0
 
+extern "C" const char* dlm_last_cuda_error(void) { return dlm::g_last_error; }
+
 extern "C" dlm_status_t dlm_get_device_status(const void* workspace, uint32_t* host_status,
                                               dlm_stream_t stream) {
     if (!workspace || !host_status) return DLM_ERR_INVALID_ARGUMENT;
     cudaStream_t s = (cudaStream_t)stream;
-    if (cudaMemcpyAsync(host_status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess) {
-        cudaGetLastError();
-        return DLM_ERR_CUDA;
-    }
-    return DLM_OK;
+    cudaError_t e = cudaMemcpyAsync(host_status, workspace, sizeof(uint32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) cudaGetLastError();
+    return dlm::cuda_status(e, "dlm_get_device_status");
 }

@@ -12,20 +12,19 @@
 //                 target, unit and weight), counts N, and writes a row list
 //                 with the scored rows first -- so the CE kernel can deal the
 //                 expensive rows out evenly.
-//   2. k_ce_*     the hot kernel.  HBM-bound: each scored row is read once
-//                 (V*2 bytes) and each row's gradient written once (V*2 bytes).
-//                 Fast path (k_ce_cluster): a cluster of K CTAs owns one row at
-//                 a time, CTA j holding columns [j*S, (j+1)*S) -- the row does
-//                 not fit one SM's shared memory for V >= ~110k, so it is split
-//                 across the cluster.  Each CTA streams its slice with a bulk
-//                 async copy (TMA engine, no multicast) into a ring of shared
-//                 buffers, pulls it into registers, computes its (max, sum of
-//                 exp) pair, exchanges the pair with the other K-1 CTAs through
-//                 distributed shared memory (st.async + mbarrier), and writes
-//                 grad = g*w*(softmax - onehot) as bf16 with 128-bit streaming
-//                 stores.  Unscored rows are zero-filled with the same stores.
+//   2. k_ce_*     the hot kernel, HBM-bound: every scored row must be read
+//                 (V*2 bytes) and every row's gradient written (V*2 bytes).
+//                 Fast path (k_ce_stream): one CTA per SM, a TMA producer warp
+//                 and 16 consumer warps; each scored row is streamed twice
+//                 through a shared-memory ring -- pass 1 from HBM (kept in L2
+//                 with an evict_last policy) for the online max / sum of exp,
+//                 pass 2 from L2 for the bf16 gradient -- and unscored rows are
+//                 zero-filled by bulk shared->global copies from the producer.
+//                 A row of 126k-262k bf16 columns (253-524 KB) does not fit in
+//                 one SM's shared memory, so it is not held on chip between the
+//                 passes; L2 holds it instead.
 //                 General path (k_ce_generic): any V / ld / alignment, one CTA
-//                 per row, two passes over the row (the second hits L2).
+//                 per row, two passes over the row with plain loads.
 //   3. k_reduce   one CTA: per-unit sums and the total, fixed order, double.
 #include <mutex>
 
@@ -47,6 +46,7 @@ struct WsHeader {
     int32_t n_nonpad;     // N of the diffusion layout
     int32_t n_scored_a;   // scored diffusion rows
     int32_t n_scored_b;   // scored encoder rows
+    uint32_t ticket;      // completion counter of k_reduce (zeroed by k_plan)
 };
 static_assert(sizeof(WsHeader) <= kWsAlign, "header");
 
@@ -232,6 +232,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(PlanParams P) {
         P.hdr->n_nonpad = N;
         P.hdr->n_scored_a = n_a;
         P.hdr->n_scored_b = n_b;
+        P.hdr->ticket = 0u;
     }
 }
 
@@ -247,9 +248,6 @@ struct CeParams {
     int vocab;
     float grad_scale;
     float* row_loss;
-    // cluster path
-    int slice;       // S: columns per CTA (multiple of 8)
-    int nbuf;        // shared-memory ring depth
 };
 
 // (max, sum exp(x - max)) pairs combine associatively; an empty side has
@@ -273,205 +271,248 @@ __device__ __forceinline__ void row_ptrs(const CeParams& P, int q, const uint16_
     }
 }
 
-constexpr int kCeThreads = 512;
-constexpr int kCeWarps = kCeThreads / 32;
-constexpr int kMaxCluster = 8;
-constexpr int kMaxBuf = 4;
+// Fast path.  One CTA per SM, 16 consumer warps + 1 producer warp.  Each
+// CTA takes every G-th scored row of the list (G = grid size) and streams it
+// twice through a ring of kStages shared-memory chunks of kChunk elements:
+//   pass 1: bulk loads from HBM with an L2 evict_last policy; per-thread
+//           online (max, sum exp) -> one block combine -> lse of the row;
+//   pass 2: the same chunks again (L2 hits), loaded evict_first; the
+//           gradient g*w*(exp(x - lse) - [v == y]) goes out as 128-bit
+//           stores with an L2 evict_first policy.
+// The producer warp also zero-fills this CTA's share of the unscored rows
+// with bulk shared->global copies from a zeroed shared block, interleaved with
+// the scored rows so the zero stream overlaps the consumers' work.
+#ifndef DLM_CE_WARPS
+#define DLM_CE_WARPS 16
+#endif
+#ifndef DLM_CE_CHUNK
+#define DLM_CE_CHUNK 8192
+#endif
+#ifndef DLM_CE_STAGES
+#define DLM_CE_STAGES 8
+#endif
+#ifndef DLM_CE_CTAS_PER_SM
+#define DLM_CE_CTAS_PER_SM 1
+#endif
+constexpr int kConsumerWarps = DLM_CE_WARPS;
+constexpr int kConsumers = kConsumerWarps * 32;
+constexpr int kStreamThreads = kConsumers + 32;
+constexpr int kChunk = DLM_CE_CHUNK;         // bf16 elements per stage
+constexpr int kStages = DLM_CE_STAGES;       // ring depth
+constexpr int kCtasPerSm = DLM_CE_CTAS_PER_SM;
+#ifndef DLM_CE_ZERO
+#define DLM_CE_ZERO 16384
+#endif
+#ifndef DLM_CE_HINTS
+#define DLM_CE_HINTS 1
+#endif
+constexpr int kZeroBytes = DLM_CE_ZERO;
+constexpr int kVecPerThread = kChunk / 8 / kConsumers;   // 16-byte vectors per thread per chunk
+static_assert(kVecPerThread * 8 * kConsumers == kChunk, "chunk split");
 
-struct __align__(16) CeSmemTail {
-    uint64_t full[kMaxBuf];
-    uint64_t xbar[2];
-    float4 xslot[2][kMaxCluster];
-    float red_m[kCeWarps];
-    float red_s[kCeWarps];
-    float xy;
+struct __align__(128) StreamSmem {
+    uint4 ring[kStages][kChunk / 8];
+    uint4 zero[kZeroBytes / 16];
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    float red_m[2][kConsumerWarps];
+    float red_s[2][kConsumerWarps];
+    float xy[2];
     int abort;
 };
 
-template <int CHUNKS>
-__global__ void __launch_bounds__(kCeThreads, 1) k_ce_cluster(const CeParams P) {
-    extern __shared__ __align__(128) uint8_t smem[];
+__global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const CeParams P) {
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    StreamSmem& S = *reinterpret_cast<StreamSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int K = int(cluster_dims_x());
-    const int rank = int(cluster_ctarank());
-    const int cid = int(cluster_id_x()), C = int(nclusters_x());
-    const int S = P.slice;
-    const int c0 = rank * S;
-    const int c1 = min(P.vocab, c0 + S);
-    const int ncols = c1 - c0;                // multiple of 8 on this path
-    const int nch = ncols >> 3;
-    const int nbuf = P.nbuf;
-    CeSmemTail* tail = reinterpret_cast<CeSmemTail*>(smem + size_t(nbuf) * S * 2);
-    const uint32_t buf0 = smem_addr(smem);
+    const int V = P.vocab;
+    const int nch = (V + kChunk - 1) / kChunk;
+    const int G = gridDim.x;
+    volatile int* abort = &S.abort;
 
+    for (int i = tid; i < kZeroBytes / 16; i += kStreamThreads) S.zero[i] = make_uint4(0, 0, 0, 0);
     if (tid == 0) {
-        for (int b = 0; b < nbuf; ++b) mbar_init(smem_addr(&tail->full[b]), 1);
-        mbar_init(smem_addr(&tail->xbar[0]), 1);
-        mbar_init(smem_addr(&tail->xbar[1]), 1);
-        tail->abort = 0;
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(smem_addr(&S.full[i]), 1);
+            mbar_init(smem_addr(&S.empty[i]), kConsumerWarps);
+        }
+        S.abort = 0;
         fence_mbar_init_cluster();
     }
-    // peers' barriers must exist before any remote arrive
-    cluster_sync_all();
+    fence_proxy_async_smem();   // zero block visible to the bulk-copy engine
+    __syncthreads();
 
     const int n_scored = P.hdr->n_scored;
     const int n_rows = P.hdr->n_rows;
-    const int my_scored = cid < n_scored ? (n_scored - cid + C - 1) / C : 0;
+    const int my_scored = blockIdx.x < n_scored ? (n_scored - blockIdx.x + G - 1) / G : 0;
+    const int n_unscored = n_rows - n_scored;
+    const int my_unscored = blockIdx.x < n_unscored ? (n_unscored - blockIdx.x + G - 1) / G : 0;
 
-    auto issue = [&](int k) {
-        const int4 e = P.list[cid + k * C];
-        const uint16_t* x;
-        uint16_t* d;
-        row_ptrs(P, e.x, x, d);
-        const int b = k % nbuf;
-        const uint32_t bar = smem_addr(&tail->full[b]);
-        mbar_arrive_expect_tx(bar, uint32_t(ncols) * 2u);
-        bulk_g2s(buf0 + uint32_t(b) * uint32_t(S) * 2u, x + c0, uint32_t(ncols) * 2u, bar);
-    };
-
-    int issued = 0;      // meaningful in thread 0 only
-    int waited = 0;      // full-barrier waits completed
-    if (tid == 0) {
-        const int pre = min(nbuf, my_scored);
-        for (; issued < pre; ++issued) issue(issued);
+    if (warp == kConsumerWarps) {
+        // ------------------------------ producer ------------------------------
+        if (lane == 0) {
+            const uint64_t pol_keep = DLM_CE_HINTS ? policy_evict_last() : policy_evict_normal();
+            const uint64_t pol_drop = DLM_CE_HINTS ? policy_evict_first() : policy_evict_normal();
+            int seq = 0, zdone = 0;
+            auto zero_row = [&](int j) {
+                const int q = P.list[n_scored + blockIdx.x + j * G].x;
+                const uint16_t* xr;
+                uint16_t* dr;
+                row_ptrs(P, q, xr, dr);
+                const uint32_t bytes = uint32_t(V) * 2u;
+                for (uint32_t off = 0; off < bytes; off += kZeroBytes) {
+                    const uint32_t n = bytes - off < uint32_t(kZeroBytes) ? bytes - off : uint32_t(kZeroBytes);
+                    bulk_s2g_hint(reinterpret_cast<uint8_t*>(dr) + off, smem_addr(S.zero), n, pol_drop);
+                }
+                bulk_commit_group();
+                P.row_loss[q] = 0.f;
+            };
+            bool ok = true;
+            for (int k = 0; k < my_scored && ok; ++k) {
+                const int q = P.list[blockIdx.x + k * G].x;
+                const uint16_t* xr;
+                uint16_t* dr;
+                row_ptrs(P, q, xr, dr);
+                for (int pass = 0; pass < 2 && ok; ++pass) {
+                    for (int c = 0; c < nch; ++c, ++seq) {
+                        const int st = seq % kStages;
+                        if (!mbar_wait_or_abort(smem_addr(&S.empty[st]), ((seq / kStages) & 1) ^ 1, P.status,
+                                                abort)) { ok = false; break; }
+                        const int e0 = c * kChunk;
+                        const uint32_t bytes = uint32_t(min(kChunk, V - e0)) * 2u;
+                        const uint32_t fb = smem_addr(&S.full[st]);
+                        mbar_arrive_expect_tx(fb, bytes);
+                        bulk_g2s_hint(smem_addr(S.ring[st]), xr + e0, bytes, fb, pass == 0 ? pol_keep : pol_drop);
+                    }
+                }
+                // spread the zero rows evenly over the scored ones
+                const int want = my_scored ? int((int64_t(k + 1) * my_unscored) / my_scored) : 0;
+                while (ok && zdone < want) zero_row(zdone++);
+            }
+            while (ok && zdone < my_unscored) zero_row(zdone++);
+            bulk_wait_group_read<0>();   // shared zero block no longer read
+        }
+        return;
     }
 
-    int k = 0;
-    bool ok = true;
-    for (; k < my_scored; ++k) {
-        const int4 e = P.list[cid + k * C];
+    // ------------------------------ consumers ------------------------------
+    const uint64_t pol_drop = DLM_CE_HINTS ? policy_evict_first() : policy_evict_normal();
+    int seq = 0;
+    int4 e_next = my_scored > 0 ? P.list[blockIdx.x] : make_int4(0, -1, 0, 0);
+    for (int k = 0; k < my_scored; ++k) {
+        const int4 e = e_next;
+        if (k + 1 < my_scored) e_next = P.list[blockIdx.x + (k + 1) * G];
         const int q = e.x, y = e.y;
         const float w = __int_as_float(e.z);
-        const int b = k % nbuf;
-        if (!mbar_wait_bounded<false>(smem_addr(&tail->full[b]), uint32_t(k / nbuf) & 1u, P.status)) {
-            ok = false;
-        }
-        if (__syncthreads_or(!ok)) { ok = false; break; }
-        waited = k + 1;
+        const int par = k & 1;
+        const uint16_t* xr;
+        uint16_t* dr;
+        row_ptrs(P, q, xr, dr);
 
-        // registers <- shared slice
-        const uint4* sb = reinterpret_cast<const uint4*>(smem + size_t(b) * S * 2);
-        uint4 raw[CHUNKS];
-        #pragma unroll
-        for (int c = 0; c < CHUNKS; ++c) {
-            const int ci = tid + c * kCeThreads;
-            raw[c] = ci < nch ? sb[ci] : make_uint4(0, 0, 0, 0);
-        }
-        if (tid == 0) {
-            tail->xy = (y >= c0 && y < c1)
-                ? bf16_bits_to_float(reinterpret_cast<const uint16_t*>(sb)[y - c0]) : -INFINITY;
-        }
-        // per-thread max over its columns
-        float m = -INFINITY;
-        #pragma unroll
-        for (int c = 0; c < CHUNKS; ++c) {
-            if (tid + c * kCeThreads < nch) {
-                const uint32_t wv[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
-                #pragma unroll
-                for (int h = 0; h < 4; ++h) m = fmaxf(m, fmaxf(bf16lo(wv[h]), bf16hi(wv[h])));
+        // pass 1: online (max, sum exp)
+        float m = -INFINITY, s = 0.f;
+        bool ok = true;
+        for (int c = 0; c < nch; ++c, ++seq) {
+            const int st = seq % kStages;
+            if (!mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort)) {
+                ok = false;
+                break;
             }
-        }
-        // e_v = exp(x_v - m), kept in registers until the row's lse is known
-        float ev[CHUNKS * 8];
-        float s = 0.f;
-        const float mb = m * kLog2e;
-        #pragma unroll
-        for (int c = 0; c < CHUNKS; ++c) {
-            const bool valid = tid + c * kCeThreads < nch;
-            const uint32_t wv[4] = {raw[c].x, raw[c].y, raw[c].z, raw[c].w};
+            const int e0 = c * kChunk;
+            float x[kVecPerThread * 8];
+            float cm = -INFINITY;
             #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-                const float a0 = valid ? exp2f(fmaf(bf16lo(wv[h]), kLog2e, -mb)) : 0.f;
-                const float a1 = valid ? exp2f(fmaf(bf16hi(wv[h]), kLog2e, -mb)) : 0.f;
-                ev[c * 8 + 2 * h] = a0;
-                ev[c * 8 + 2 * h + 1] = a1;
-                s += a0 + a1;
+            for (int j = 0; j < kVecPerThread; ++j) {
+                const int vi = tid + j * kConsumers;
+                const int col = e0 + vi * 8;
+                if (col < V) {
+                    const uint4 r = S.ring[st][vi];
+                    const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
+                    #pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        x[j * 8 + 2 * h] = bf16lo(wv[h]);
+                        x[j * 8 + 2 * h + 1] = bf16hi(wv[h]);
+                    }
+                    #pragma unroll
+                    for (int h = 0; h < 8; ++h)
+                        if (y == col + h) S.xy[par] = x[j * 8 + h];
+                } else {
+                    #pragma unroll
+                    for (int h = 0; h < 8; ++h) x[j * 8 + h] = -INFINITY;
+                }
+                #pragma unroll
+                for (int h = 0; h < 8; ++h) cm = fmaxf(cm, x[j * 8 + h]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&S.empty[st]));
+            if (cm > m) {
+                s = (m == -INFINITY) ? 0.f : s * exp2f((m - cm) * kLog2e);
+                m = cm;
+            }
+            if (m != -INFINITY) {
+                const float mb = m * kLog2e;
+                #pragma unroll
+                for (int h = 0; h < kVecPerThread * 8; ++h) s += exp2f(fmaf(x[h], kLog2e, -mb));
             }
         }
-        // warp, then block combine of (m, s)
-        float wm = m, ws = s;
+        // block combine among the consumer warps
         #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-            const float m2 = __shfl_xor_sync(0xffffffffu, wm, o);
-            const float s2 = __shfl_xor_sync(0xffffffffu, ws, o);
-            lse_combine(wm, ws, m2, s2);
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+            const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+            lse_combine(m, s, m2, s2);
         }
-        if (lane == 0) { tail->red_m[warp] = wm; tail->red_s[warp] = ws; }
-        __syncthreads();   // all threads are done with buffer b and wrote red_*
-
-        const int xs = k;  // exchange index (every scored row exchanges once)
-        const uint32_t xbar = smem_addr(&tail->xbar[xs & 1]);
-        if (tid == 0) {
-            if (issued < my_scored) issue(issued++);
-            float bm = tail->red_m[0], bs = tail->red_s[0];
-            for (int i = 1; i < kCeWarps; ++i) lse_combine(bm, bs, tail->red_m[i], tail->red_s[i]);
-            mbar_arrive_expect_tx(xbar, uint32_t(K) * 16u);
-            const uint32_t slot = smem_addr(&tail->xslot[xs & 1][rank]);
-            for (int r = 0; r < K; ++r) {
-                st_async_v4(mapa_shared(slot, uint32_t(r)), bm, bs, tail->xy, 0.f,
-                            mapa_shared(xbar, uint32_t(r)));
-            }
-        }
-        if (!mbar_wait_bounded<true>(xbar, uint32_t(xs >> 1) & 1u, P.status)) ok = false;
-        if (__syncthreads_or(!ok)) { ok = false; break; }
-
-        float M = -INFINITY, Ssum = 0.f, XY = -INFINITY;
-        for (int r = 0; r < K; ++r) {
-            const float4 v = tail->xslot[xs & 1][r];
-            lse_combine(M, Ssum, v.x, v.y);
-            XY = fmaxf(XY, v.z);
-        }
-        const float lse = M + logf(Ssum);
-        const float coef = P.grad_scale * w;
-        const float sc = m == -INFINITY ? 0.f : coef * exp2f((m - lse) * kLog2e);
-
-        const uint16_t* xrow;
-        uint16_t* drow;
-        row_ptrs(P, q, xrow, drow);
-        uint4* dst = reinterpret_cast<uint4*>(drow + c0);
+        if (lane == 0) { S.red_m[par][warp] = m; S.red_s[par][warp] = s; }
+        ok = ok && !*abort;
+        named_barrier_sync(1, kConsumers);
+        if (!ok || *abort) break;
+        float M = S.red_m[par][0], Ssum = S.red_s[par][0];
         #pragma unroll
-        for (int c = 0; c < CHUNKS; ++c) {
-            const int ci = tid + c * kCeThreads;
-            if (ci < nch) {
-                float g[8];
-                #pragma unroll
-                for (int h = 0; h < 8; ++h) g[h] = ev[c * 8 + h] * sc;
-                const int col = c0 + ci * 8;
-                if (y >= col && y < col + 8) g[y - col] -= coef;
-                uint4 o;
-                o.x = pack_bf16x2(g[0], g[1]);
-                o.y = pack_bf16x2(g[2], g[3]);
-                o.z = pack_bf16x2(g[4], g[5]);
-                o.w = pack_bf16x2(g[6], g[7]);
-                __stcs(dst + ci, o);
-            }
-        }
-        if (rank == 0 && tid == 0) P.row_loss[q] = w * (lse - XY);
-    }
+        for (int i = 1; i < kConsumerWarps; ++i) lse_combine(M, Ssum, S.red_m[par][i], S.red_s[par][i]);
+        const float lse = M + logf(Ssum);
+        const float lb = lse * kLog2e;
+        const float coef = P.grad_scale * w;
 
-    if (ok) {
-        // unscored rows: exact zeros
-        const uint4 z = make_uint4(0, 0, 0, 0);
-        for (int i = n_scored + cid; i < n_rows; i += C) {
-            const int q = P.list[i].x;
-            const uint16_t* xrow;
-            uint16_t* drow;
-            row_ptrs(P, q, xrow, drow);
-            uint4* dst = reinterpret_cast<uint4*>(drow + c0);
-            #pragma unroll
-            for (int c = 0; c < CHUNKS; ++c) {
-                const int ci = tid + c * kCeThreads;
-                if (ci < nch) __stcs(dst + ci, z);
+        // pass 2: gradient
+        for (int c = 0; c < nch; ++c, ++seq) {
+            const int st = seq % kStages;
+            if (!mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort)) {
+                ok = false;
+                break;
             }
-            if (rank == 0 && tid == 0) P.row_loss[q] = 0.f;
+            const int e0 = c * kChunk;
+            uint4 outv[kVecPerThread];
+            #pragma unroll
+            for (int j = 0; j < kVecPerThread; ++j) {
+                const int vi = tid + j * kConsumers;
+                const int col = e0 + vi * 8;
+                if (col < V) {
+                    const uint4 r = S.ring[st][vi];
+                    const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
+                    float g[8];
+                    #pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        g[2 * h] = coef * exp2f(fmaf(bf16lo(wv[h]), kLog2e, -lb));
+                        g[2 * h + 1] = coef * exp2f(fmaf(bf16hi(wv[h]), kLog2e, -lb));
+                    }
+                    #pragma unroll
+                    for (int h = 0; h < 8; ++h)
+                        if (y == col + h) g[h] -= coef;
+                    outv[j] = make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]),
+                                         pack_bf16x2(g[4], g[5]), pack_bf16x2(g[6], g[7]));
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&S.empty[st]));
+            #pragma unroll
+            for (int j = 0; j < kVecPerThread; ++j) {
+                const int col = e0 + (tid + j * kConsumers) * 8;
+                if (col < V) st_global_v4_hint(dr + col, outv[j], pol_drop);
+            }
         }
-    } else if (tid == 0) {
-        // drain this CTA's own copies still in flight before leaving
-        for (int j = waited; j < issued; ++j)
-            mbar_wait_bounded<false>(smem_addr(&tail->full[j % nbuf]), uint32_t(j / nbuf) & 1u, P.status);
+        if (!ok) break;
+        if (tid == 0) P.row_loss[q] = w * (lse - S.xy[par]);
     }
-    // no CTA leaves while a peer may still write into its shared memory
-    cluster_sync_all();
 }
 
 // General path: one CTA per row (grid-stride), any vocab / stride / alignment.
@@ -538,9 +579,10 @@ struct ReduceParams {
     double* unit_acc;        // [n_units]
     float* unit_loss;        // may be null
     float* loss;
+    unsigned int* ticket;    // zero on entry (the plan kernel clears it); left zero
 };
 
-constexpr int kRedThreads = 1024;
+constexpr int kRedThreads = 256;
 
 __device__ __forceinline__ void unit_range(const LayoutDev& L, int u, int64_t& lo, int64_t& hi) {
     if (L.n_tokens == 0) { lo = hi = 0; return; }
@@ -554,115 +596,78 @@ __device__ __forceinline__ void unit_range(const LayoutDev& L, int u, int64_t& l
     }
 }
 
+// Fixed-order block sum of double values (one per thread).
+__device__ __forceinline__ double block_sum(double v, double* red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[warp] = v;
+    __syncthreads();
+    double t = 0.0;
+    if (warp == 0) {
+        t = lane < int(blockDim.x >> 5) ? red[lane] : 0.0;
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    }
+    __syncthreads();
+    return t;   // valid in warp 0
+}
+
+// One CTA per unit (grid-stride for very many units): the unit's rows of both
+// terms summed in a fixed order; the CTA that finishes last adds the units up
+// in a fixed order.  Bitwise reproducible.
 __global__ void __launch_bounds__(kRedThreads) k_reduce(ReduceParams R) {
     __shared__ double red[kRedThreads / 32];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ bool last;
+    const int tid = threadIdx.x;
     const int U = R.a.n_units;
-    for (int u = warp; u < U; u += kRedThreads / 32) {
+    for (int u = blockIdx.x; u < U; u += gridDim.x) {
         double acc = 0.0;
         int64_t lo, hi;
         unit_range(R.a, u, lo, hi);
-        for (int64_t i = lo + lane; i < hi; i += 32) acc += double(R.row_loss[i]);
+        for (int64_t i = lo + tid; i < hi; i += kRedThreads) acc += double(R.row_loss[i]);
         unit_range(R.b, u, lo, hi);
-        for (int64_t i = lo + lane; i < hi; i += 32) acc += double(R.row_loss[R.a.n_tokens + i]);
-        #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) {
-            R.unit_acc[u] = acc;
-            if (R.unit_loss) R.unit_loss[u] = float(acc);
+        for (int64_t i = lo + tid; i < hi; i += kRedThreads) acc += double(R.row_loss[R.a.n_tokens + i]);
+        const double t = block_sum(acc, red);
+        if (tid == 0) {
+            R.unit_acc[u] = t;
+            if (R.unit_loss) R.unit_loss[u] = float(t);
         }
     }
+    // last CTA: the total
+    if (tid == 0) {
+        __threadfence();
+        last = atomicAdd(R.ticket, 1u) == gridDim.x - 1;
+    }
     __syncthreads();
-    // total: each thread a contiguous run of units, then a fixed tree
+    if (!last) return;
+    __threadfence();
     const int per = (U + kRedThreads - 1) / kRedThreads;
     double acc = 0.0;
-    for (int u = tid * per; u < min(U, (tid + 1) * per); ++u) acc += R.unit_acc[u];
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) red[warp] = acc;
-    __syncthreads();
-    if (warp == 0) {
-        double v = red[lane];
-        #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) R.loss[0] = float(v);
+    for (int u = tid * per; u < min(U, (tid + 1) * per); ++u) acc += __ldcg(R.unit_acc + u);
+    const double t = block_sum(acc, red);
+    if (tid == 0) {
+        R.loss[0] = float(t);
+        *R.ticket = 0u;
     }
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-constexpr size_t kSmemBudget = 227 * 1024;
-
-struct ClusterCfg {
-    int K = 0, S = 0, chunks = 0, nbuf = 0;
-    size_t smem = 0;
-};
-
-// Smallest cluster K (1..8) whose per-CTA slice fits CHUNKS <= 8 per thread
-// and leaves room for at least two shared buffers.
-static ClusterCfg pick_cluster(int V) {
-    ClusterCfg c;
-    for (int K = 1; K <= kMaxCluster; ++K) {
-        const int S = int(align_up(size_t((V + K - 1) / K), 8));
-        if ((K - 1) * S >= V) break;
-        const int chunks = (S / 8 + kCeThreads - 1) / kCeThreads;
-        if (chunks > 8) continue;
-        const size_t tail = sizeof(CeSmemTail);
-        int nbuf = int((kSmemBudget - tail - 128) / (size_t(S) * 2));
-        nbuf = nbuf > kMaxBuf ? kMaxBuf : nbuf;
-        if (nbuf < 2) continue;
-        c.K = K; c.S = S; c.chunks = chunks; c.nbuf = nbuf;
-        c.smem = size_t(nbuf) * S * 2 + tail;
-        return c;
-    }
-    return c;
-}
-
-using CeKernel = void (*)(const CeParams);
-
-static CeKernel cluster_kernel(int chunks) {
-    switch (chunks) {
-        case 1: return k_ce_cluster<1>;
-        case 2: return k_ce_cluster<2>;
-        case 3: return k_ce_cluster<3>;
-        case 4: return k_ce_cluster<4>;
-        case 5: return k_ce_cluster<5>;
-        case 6: return k_ce_cluster<6>;
-        case 7: return k_ce_cluster<7>;
-        case 8: return k_ce_cluster<8>;
-        default: return nullptr;
-    }
-}
-
-// Occupancy of a cluster configuration, cached per (device, K, chunks, smem).
-static int max_active_clusters(int dev, CeKernel kern, const ClusterCfg& c) {
-    struct Entry { int dev, K, chunks; size_t smem; int n; };
+// Shared-memory attribute of the streaming kernel, set once per device.
+static bool stream_kernel_ready(int dev) {
     static std::mutex mu;
-    static Entry cache[64];
-    static int n_cache = 0;
+    static int state[64];   // 0 unknown, 1 ok, 2 failed
+    if (dev < 0 || dev >= 64) return false;
     std::lock_guard<std::mutex> g(mu);
-    for (int i = 0; i < n_cache; ++i)
-        if (cache[i].dev == dev && cache[i].K == c.K && cache[i].chunks == c.chunks && cache[i].smem == c.smem)
-            return cache[i].n;
-    int n = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(c.smem)) == cudaSuccess) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(c.K * 148, 1, 1);
-        cfg.blockDim = dim3(kCeThreads, 1, 1);
-        cfg.dynamicSmemBytes = c.smem;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = c.K;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+    if (state[dev] == 0) {
+        const cudaError_t e = cudaFuncSetAttribute(k_ce_stream, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   int(sizeof(StreamSmem)));
+        if (e != cudaSuccess) cudaGetLastError();
+        state[dev] = e == cudaSuccess ? 1 : 2;
     }
-    cudaGetLastError();
-    if (n_cache < 64) cache[n_cache++] = Entry{dev, c.K, c.chunks, c.smem, n};
-    return n;
+    return state[dev] == 1;
 }
 
 static LayoutDev to_dev(const dlm_layout_t* L) {
@@ -744,7 +749,7 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
     pp.hdr = hdr;
     pp.list = list;
     k_plan<<<1, kPlanThreads, 0, s>>>(pp);
-    if ((st = last_launch_status()) != DLM_OK) return st;
+    if ((st = last_launch_status("k_plan launch")) != DLM_OK) return st;
 
     // ---- 2. CE ----
     if (R > 0) {
@@ -761,43 +766,17 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
         bool fast = (vocab % 8 == 0) && (ld % 8 == 0) && vocab >= 4096 &&
                     (rows_a == 0 || (aligned16(logits) && aligned16(dlogits)));
         if (has_enc) fast = fast && (enc_ld % 8 == 0) && aligned16(enc_logits) && aligned16(enc_dlogits);
-        ClusterCfg cc;
-        int n_clusters = 0;
-        CeKernel kern = nullptr;
-        if (fast) {
-            cc = pick_cluster(vocab);
-            kern = cc.K ? cluster_kernel(cc.chunks) : nullptr;
-            if (kern) {
-                int dev = 0;
-                cudaGetDevice(&dev);
-                n_clusters = max_active_clusters(dev, kern, cc);
-            }
-            fast = kern && n_clusters > 0;
-        }
-        if (fast) {
-            if (n_clusters > R) n_clusters = int(R);
-            cp.slice = cc.S;
-            cp.nbuf = cc.nbuf;
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(unsigned(n_clusters * cc.K), 1, 1);
-            cfg.blockDim = dim3(kCeThreads, 1, 1);
-            cfg.dynamicSmemBytes = cc.smem;
-            cfg.stream = s;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = cc.K;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            if (cudaLaunchKernelEx(&cfg, kern, cp) != cudaSuccess) { cudaGetLastError(); return DLM_ERR_CUDA; }
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (fast && stream_kernel_ready(dev)) {
+            const int64_t grid = R < int64_t(sms) * kCtasPerSm ? R : int64_t(sms) * kCtasPerSm;
+            k_ce_stream<<<unsigned(grid), kStreamThreads, sizeof(StreamSmem), s>>>(cp);
+            if ((st = last_launch_status("k_ce_stream launch")) != DLM_OK) return st;
         } else {
-            int dev = 0, sms = 148;
-            cudaGetDevice(&dev);
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
             const int64_t grid = R < int64_t(sms) * 8 ? R : int64_t(sms) * 8;
             k_ce_generic<<<unsigned(grid), kGenThreads, 0, s>>>(cp);
-            if ((st = last_launch_status()) != DLM_OK) return st;
+            if ((st = last_launch_status("k_ce_generic launch")) != DLM_OK) return st;
         }
     }
 
@@ -809,6 +788,9 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
     rp.unit_acc = unit_acc;
     rp.unit_loss = unit_loss;
     rp.loss = loss;
-    k_reduce<<<1, kRedThreads, 0, s>>>(rp);
-    return last_launch_status();
+    rp.ticket = &hdr->ticket;
+    const int U = layout->n_units;
+    const int rgrid = U < 1 ? 1 : (U > 65536 ? 65536 : U);
+    k_reduce<<<rgrid, kRedThreads, 0, s>>>(rp);
+    return last_launch_status("k_reduce launch");
 }

@@ -19,9 +19,17 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // The library is built for sm_100a only: refuse anything else up front.
 dlm_status_t check_device();
 
-inline dlm_status_t last_launch_status() {
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? DLM_OK : DLM_ERR_CUDA;
+// Remember the text of a CUDA error for dlm_last_cuda_error().
+void record_cuda_error(cudaError_t e, const char* where);
+
+inline dlm_status_t cuda_status(cudaError_t e, const char* where) {
+    if (e == cudaSuccess) return DLM_OK;
+    record_cuda_error(e, where);
+    return DLM_ERR_CUDA;
+}
+
+inline dlm_status_t last_launch_status(const char* where = "kernel launch") {
+    return cuda_status(cudaGetLastError(), where);
 }
 
 // Layout sanity that the host can see (the device checks cu_seqlens itself).

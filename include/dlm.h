@@ -106,6 +106,11 @@ typedef struct dlm_layout {
 /* Human-readable name of a status code (static string, never NULL). */
 DLM_API const char *dlm_status_string(dlm_status_t status);
 
+/* Text of the last CUDA error this library saw on the calling host thread
+ * (a DLM_ERR_CUDA return), or "" if none.  Static/thread-local storage owned
+ * by the library; valid until the next failing call on the same thread. */
+DLM_API const char *dlm_last_cuda_error(void);
+
 /* Library version: major * 10000 + minor * 100 + patch. */
 DLM_API int dlm_version(void);
 
