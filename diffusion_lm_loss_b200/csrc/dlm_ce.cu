@@ -39,17 +39,6 @@ constexpr float kLn2 = 0.6931471805599453f;
 // ---------------------------------------------------------------------------
 // workspace layout
 // ---------------------------------------------------------------------------
-struct WsHeader {
-    uint32_t status;
-    int32_t n_scored;     // scored rows, both terms
-    int32_t n_rows;       // rows, both terms
-    int32_t n_nonpad;     // N of the diffusion layout
-    int32_t n_scored_a;   // scored diffusion rows
-    int32_t n_scored_b;   // scored encoder rows
-    uint32_t ticket;      // completion counter of k_reduce (zeroed by k_plan)
-};
-static_assert(sizeof(WsHeader) <= kWsAlign, "header");
-
 struct WsLayout {
     size_t list, row_loss, unit_acc, total;
 };
@@ -271,7 +260,7 @@ __device__ __forceinline__ void row_ptrs(const CeParams& P, int q, const uint16_
     }
 }
 
-// Fast path.  One CTA per SM, 16 consumer warps + 1 producer warp.  Each
+// Fast path.  Two CTAs per SM, each 8 consumer warps + 1 producer warp.  Each
 // CTA takes every G-th scored row of the list (G = grid size) and streams it
 // twice through a ring of kStages shared-memory chunks of kChunk elements:
 //   pass 1: bulk loads from HBM with an L2 evict_last policy; per-thread
@@ -283,16 +272,16 @@ __device__ __forceinline__ void row_ptrs(const CeParams& P, int q, const uint16_
 // with bulk shared->global copies from a zeroed shared block, interleaved with
 // the scored rows so the zero stream overlaps the consumers' work.
 #ifndef DLM_CE_WARPS
-#define DLM_CE_WARPS 16
+#define DLM_CE_WARPS 8
 #endif
 #ifndef DLM_CE_CHUNK
 #define DLM_CE_CHUNK 8192
 #endif
 #ifndef DLM_CE_STAGES
-#define DLM_CE_STAGES 8
+#define DLM_CE_STAGES 6
 #endif
 #ifndef DLM_CE_CTAS_PER_SM
-#define DLM_CE_CTAS_PER_SM 1
+#define DLM_CE_CTAS_PER_SM 2
 #endif
 constexpr int kConsumerWarps = DLM_CE_WARPS;
 constexpr int kConsumers = kConsumerWarps * 32;
@@ -301,7 +290,7 @@ constexpr int kChunk = DLM_CE_CHUNK;         // bf16 elements per stage
 constexpr int kStages = DLM_CE_STAGES;       // ring depth
 constexpr int kCtasPerSm = DLM_CE_CTAS_PER_SM;
 #ifndef DLM_CE_ZERO
-#define DLM_CE_ZERO 16384
+#define DLM_CE_ZERO 4096
 #endif
 #ifndef DLM_CE_HINTS
 #define DLM_CE_HINTS 1
@@ -390,6 +379,11 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
                 while (ok && zdone < want) zero_row(zdone++);
             }
             while (ok && zdone < my_unscored) zero_row(zdone++);
+            if (!ok) {
+                // let the copies already issued land before this thread leaves
+                for (int j = seq - 1; j >= 0 && j >= seq - kStages; --j)
+                    mbar_wait_bounded<false>(smem_addr(&S.full[j % kStages]), (j / kStages) & 1, nullptr);
+            }
             bulk_wait_group_read<0>();   // shared zero block no longer read
         }
         return;
@@ -409,15 +403,13 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
         uint16_t* dr;
         row_ptrs(P, q, xr, dr);
 
-        // pass 1: online (max, sum exp)
+        // pass 1: online (max, sum exp).  After an abort (a bounded wait gave
+        // up somewhere in the CTA) the waits return at once and the loops run
+        // on with garbage, so every consumer still meets every barrier.
         float m = -INFINITY, s = 0.f;
-        bool ok = true;
         for (int c = 0; c < nch; ++c, ++seq) {
             const int st = seq % kStages;
-            if (!mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort)) {
-                ok = false;
-                break;
-            }
+            mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort);
             const int e0 = c * kChunk;
             float x[kVecPerThread * 8];
             float cm = -INFINITY;
@@ -463,9 +455,7 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
             lse_combine(m, s, m2, s2);
         }
         if (lane == 0) { S.red_m[par][warp] = m; S.red_s[par][warp] = s; }
-        ok = ok && !*abort;
         named_barrier_sync(1, kConsumers);
-        if (!ok || *abort) break;
         float M = S.red_m[par][0], Ssum = S.red_s[par][0];
         #pragma unroll
         for (int i = 1; i < kConsumerWarps; ++i) lse_combine(M, Ssum, S.red_m[par][i], S.red_s[par][i]);
@@ -476,10 +466,7 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
         // pass 2: gradient
         for (int c = 0; c < nch; ++c, ++seq) {
             const int st = seq % kStages;
-            if (!mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort)) {
-                ok = false;
-                break;
-            }
+            mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort);
             const int e0 = c * kChunk;
             uint4 outv[kVecPerThread];
             #pragma unroll
@@ -510,7 +497,6 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
                 if (col < V) st_global_v4_hint(dr + col, outv[j], pol_drop);
             }
         }
-        if (!ok) break;
         if (tid == 0) P.row_loss[q] = w * (lse - S.xy[par]);
     }
 }
@@ -681,6 +667,44 @@ static LayoutDev to_dev(const dlm_layout_t* L) {
     return d;
 }
 
+dlm_status_t launch_plan(const dlm_layout_t* a, const int32_t* clean, const uint8_t* corrupted,
+                         const float* p, int mode, int align, const dlm_layout_t* b,
+                         const int32_t* ids_b, float lam, int vocab, WsHeader* hdr, int4* list,
+                         cudaStream_t s) {
+    PlanParams pp{};
+    pp.a = to_dev(a);
+    pp.clean_a = clean;
+    pp.corrupted = corrupted;
+    pp.p = p;
+    pp.mode = mode;
+    pp.align = align;
+    pp.b = to_dev(b);
+    pp.ids_b = ids_b;
+    pp.lam = lam;
+    pp.vocab = vocab;
+    pp.hdr = hdr;
+    pp.list = list;
+    k_plan<<<1, kPlanThreads, 0, s>>>(pp);
+    return last_launch_status("k_plan launch");
+}
+
+dlm_status_t launch_reduce(const dlm_layout_t* a, const dlm_layout_t* b, const float* row_loss,
+                           double* unit_acc, float* unit_loss, float* loss, WsHeader* hdr,
+                           cudaStream_t s) {
+    ReduceParams rp{};
+    rp.a = to_dev(a);
+    rp.b = to_dev(b);
+    rp.row_loss = row_loss;
+    rp.unit_acc = unit_acc;
+    rp.unit_loss = unit_loss;
+    rp.loss = loss;
+    rp.ticket = &hdr->ticket;
+    const int U = a->n_units;
+    const int rgrid = U < 1 ? 1 : (U > 65536 ? 65536 : U);
+    k_reduce<<<rgrid, kRedThreads, 0, s>>>(rp);
+    return last_launch_status("k_reduce launch");
+}
+
 }  // namespace dlm
 
 using namespace dlm;
@@ -735,21 +759,9 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
     double* unit_acc = reinterpret_cast<double*>(ws + W.unit_acc);
 
     // ---- 1. plan ----
-    PlanParams pp{};
-    pp.a = to_dev(layout);
-    pp.clean_a = clean_ids;
-    pp.corrupted = corrupted;
-    pp.p = p;
-    pp.mode = mode;
-    pp.align = align;
-    pp.b = to_dev(lb);
-    pp.ids_b = enc_ids;
-    pp.lam = enc_ar_weight;
-    pp.vocab = vocab;
-    pp.hdr = hdr;
-    pp.list = list;
-    k_plan<<<1, kPlanThreads, 0, s>>>(pp);
-    if ((st = last_launch_status("k_plan launch")) != DLM_OK) return st;
+    if ((st = launch_plan(layout, clean_ids, corrupted, p, mode, align, lb, enc_ids, enc_ar_weight, vocab,
+                          hdr, list, s)) != DLM_OK)
+        return st;
 
     // ---- 2. CE ----
     if (R > 0) {
@@ -781,16 +793,5 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
     }
 
     // ---- 3. reduce ----
-    ReduceParams rp{};
-    rp.a = to_dev(layout);
-    rp.b = to_dev(lb);
-    rp.row_loss = row_loss;
-    rp.unit_acc = unit_acc;
-    rp.unit_loss = unit_loss;
-    rp.loss = loss;
-    rp.ticket = &hdr->ticket;
-    const int U = layout->n_units;
-    const int rgrid = U < 1 ? 1 : (U > 65536 ? 65536 : U);
-    k_reduce<<<rgrid, kRedThreads, 0, s>>>(rp);
-    return last_launch_status("k_reduce launch");
+    return launch_reduce(layout, lb, row_loss, unit_acc, unit_loss, loss, hdr, s);
 }

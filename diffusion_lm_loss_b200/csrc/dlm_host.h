@@ -47,6 +47,33 @@ inline bool layout_ok(const dlm_layout_t* L) {
     return true;
 }
 
+// Header of a loss workspace (first 256 bytes), written by the row-plan
+// kernel and read by the kernels after it.
+struct WsHeader {
+    uint32_t status;      // DLM_DEV_* bits of this call
+    int32_t n_scored;     // scored rows, both terms
+    int32_t n_rows;       // rows, both terms
+    int32_t n_nonpad;     // N of the diffusion layout
+    int32_t n_scored_a;   // scored diffusion rows
+    int32_t n_scored_b;   // scored encoder rows
+    uint32_t ticket;      // completion counter of the unit reduction (zeroed by the plan)
+};
+static_assert(sizeof(WsHeader) <= kWsAlign, "header");
+
+// Row plan (one CTA): classifies every row of `a` (and of the encoder
+// layout `b`, rows after a's), writes list[] = {row, target, weight bits,
+// unit} with the scored rows first in row order, and fills *hdr.
+dlm_status_t launch_plan(const dlm_layout_t* a, const int32_t* clean, const uint8_t* corrupted,
+                         const float* p, int mode, int align, const dlm_layout_t* b,
+                         const int32_t* ids_b, float lam, int vocab, WsHeader* hdr, int4* list,
+                         cudaStream_t s);
+
+// Per-unit sums of row_loss over a's rows (and b's rows, indexed after a's)
+// and their total, in a fixed order.  Uses hdr->ticket (zeroed by the plan).
+dlm_status_t launch_reduce(const dlm_layout_t* a, const dlm_layout_t* b, const float* row_loss,
+                           double* unit_acc, float* unit_loss, float* loss, WsHeader* hdr,
+                           cudaStream_t s);
+
 // Number of logits rows described by a layout (one per token).
 inline int64_t layout_rows(const dlm_layout_t* L) { return L ? L->n_tokens : 0; }
 

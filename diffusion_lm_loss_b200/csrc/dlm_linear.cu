@@ -1,12 +1,640 @@
-// dlm_linear.cu -- fused lm_head + loss (placeholder until the tensor-core
-// path is in place: refuses every call).
+// dlm_linear.cu -- the absorbing-mask loss computed from hidden states and a
+// linear output head, logits never written to memory ("Native diffusion
+// language-model training", Adapters, merging and inference: Cut Cross
+// Entropy -- full-vocabulary CE from hidden states, aligned targets, plain
+// linear head).  The head is a dense contraction, so it runs on the 5th-gen
+// tensor cores: tcgen05.mma from shared memory into tensor-memory
+// accumulators, operands brought in by TMA tile loads (no multicast).
+//
+// With H_M = the M masked rows of H (gathered), W the [V, D] head:
+//   forward   Z = H_M W^T, tile by tile; the epilogue reads each 128x256
+//             accumulator tile out of tensor memory and keeps only per-row
+//             (max, sum exp) partials and the target logit -> lse per row.
+//   backward  per vocabulary chunk of kVc columns (a bounded buffer, never a
+//             [M, V] tensor): Z_c recomputed, dZ_c = w (softmax - onehot) in
+//             bf16; dH_M += dZ_c W_c; dW_c = dZ_c^T H_M.
+// Executed flops 8 M D V (the recompute adds 2 M D V to the 6 M D V the
+// method needs); every GEMM is the same warp-specialized persistent kernel:
+//   warp 0   TMA producer (one thread), 4-stage ring of 128x64 A + 256x64 B
+//   warp 1   MMA issuer (one thread), 128x256x16 bf16 MMAs, two 256-column
+//            accumulators in tensor memory (epilogue of tile i overlaps the
+//            main loop of tile i+1)
+//   warps 2-5  epilogue: tensor memory -> registers -> (partials | dZ |
+//            dH accumulate | dW store)
+// Every wait is bounded (a broken pipeline sets DLM_DEV_WAIT_TIMEOUT and the
+// kernel winds down instead of hanging).
+#include <cstdio>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "dlm_device.cuh"
 #include "dlm_host.h"
+#include "dlm_tc.cuh"
 
-extern "C" size_t dlm_linear_loss_workspace_size(const dlm_layout_t*, int32_t, int32_t) { return 0; }
+namespace dlm {
 
-extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t*, const uint16_t*, const uint16_t*,
-                                                int32_t, int32_t, const int32_t*, const uint8_t*,
-                                                const float*, float, float*, float*, uint16_t*,
-                                                uint16_t*, void*, size_t, dlm_stream_t) {
-    return DLM_ERR_UNSUPPORTED;
+constexpr int kBM = 128, kBN = 256, kBK = 64;
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kStageA = kBM * kBK * 2;   // 16 KB
+constexpr uint32_t kStageB = kBN * kBK * 2;   // 32 KB
+constexpr int kVc = 16384;                    // vocabulary chunk of the backward pass
+
+enum Epi { EPI_LSE = 0, EPI_DZ = 1, EPI_DH = 2, EPI_DW = 3 };
+
+struct GemmArgs {
+    const WsHeader* hdr;     // hdr->n_scored = M (masked rows)
+    uint32_t* status;
+    const int4* list;        // row plan: {token row, target, weight bits, unit}
+    int m_dev;               // 1: C rows = round_up(M, 128); 0: m_rows
+    int m_rows;
+    int n_cols;              // C columns
+    int k_dev;               // 1: K = round_up(M, 128); 0: k_len
+    int k_len;
+    int b_off;               // row offset of W (forward / dZ) or K offset into W rows (dH)
+    int col0;                // vocabulary index of C column 0 (LSE, DZ) or C row 0 (DW)
+    int vocab;
+    int d_model;
+    float grad_scale;
+    float2* part;            // LSE: [Mp, part_ld] (max, sum exp)
+    int part_ld;
+    float* xy;               // LSE: target logit per masked row
+    const float* lse;        // DZ
+    uint16_t* dz;            // DZ out: [Mp, dz_ld] bf16
+    int dz_ld;
+    float* dh;               // DH: [Mp, D] f32
+    int accumulate;
+    uint16_t* dw;            // DW: [V, D] bf16
+};
+
+struct __align__(1024) GemmSmem {
+    uint8_t a[kGemmStages][kStageA];
+    uint8_t b[kGemmStages][kStageB];
+    uint64_t full[kGemmStages];
+    uint64_t empty[kGemmStages];
+    uint64_t tfull[2];
+    uint64_t tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ int round_up_dev(int x, int a) { return (x + a - 1) / a * a; }
+
+template <int EPI, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_addr(smem_raw);
+    GemmSmem& S = *reinterpret_cast<GemmSmem*>(smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* abort = &S.abort;
+
+    const int M = g.hdr->n_scored;
+    const int Mp = round_up_dev(M, kBM);
+    const int rows = g.m_dev ? Mp : g.m_rows;
+    const int K = g.k_dev ? Mp : g.k_len;
+    const int m_tiles = rows / kBM;
+    const int n_tiles = (g.n_cols + kBN - 1) / kBN;
+    const int tiles = m_tiles * n_tiles;
+    const int nkb = K / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kGemmStages; ++i) {
+            mbar_init(smem_addr(&S.full[i]), 1);
+            mbar_init(smem_addr(&S.empty[i]), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_addr(&S.tfull[i]), 1);
+            mbar_init(smem_addr(&S.tempty[i]), 4);
+        }
+        mbar_init(smem_addr(&S.drain), 1);
+        S.abort = 0;
+        fence_mbar_init_cluster();
+        tc::prefetch_tensormap(&tmA);
+        tc::prefetch_tensormap(&tmB);
+    }
+    if (warp == 1) {
+        tc::tmem_alloc(smem_addr(&S.tmem_base), 512);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_thread_sync();
+    __syncthreads();
+    tc::fence_after_thread_sync();
+    const uint32_t tmem = S.tmem_base;
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        uint64_t pol_a, pol_b;
+        if (EPI == EPI_LSE || EPI == EPI_DZ) { pol_a = policy_evict_last(); pol_b = policy_evict_first(); }
+        else                                 { pol_a = policy_evict_normal(); pol_b = policy_evict_normal(); }
+        int it = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+            const int m0 = (tile % m_tiles) * kBM;
+            const int n0 = (tile / m_tiles) * kBN;
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = it % kGemmStages;
+                if (!mbar_wait_or_abort(smem_addr(&S.empty[s]), ((it / kGemmStages) & 1) ^ 1, g.status, abort)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = smem_addr(&S.full[s]);
+                mbar_arrive_expect_tx(fb, kStageA + kStageB);
+                const int k0 = kb * kBK;
+                const uint32_t a_s = smem_addr(S.a[s]), b_s = smem_addr(S.b[s]);
+                if (!A_MN) {
+                    tc::tma_load_2d(a_s, &tmA, k0, m0, fb, pol_a);
+                } else {
+                    tc::tma_load_2d(a_s, &tmA, m0, k0, fb, pol_a);
+                    tc::tma_load_2d(a_s + 8192, &tmA, m0 + 64, k0, fb, pol_a);
+                }
+                if (!B_MN) {
+                    tc::tma_load_2d(b_s, &tmB, k0, n0 + g.b_off, fb, pol_b);
+                } else {
+                    #pragma unroll
+                    for (int j = 0; j < 4; ++j) tc::tma_load_2d(b_s + 8192 * j, &tmB, n0 + 64 * j, k0 + g.b_off, fb, pol_b);
+                }
+            }
+        }
+        if (!ok) {
+            // let the copies already issued land before the CTA can exit
+            for (int j = it - 1; j >= 0 && j >= it - kGemmStages; --j)
+                mbar_wait_bounded<false>(smem_addr(&S.full[j % kGemmStages]), (j / kGemmStages) & 1, nullptr);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------ MMA issuer ------------------------------
+        constexpr uint32_t idesc = tc::idesc_bf16(kBM, kBN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+        int it = 0, lt = 0;
+        bool ok = nkb > 0;
+        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++lt) {
+            const int acc = lt & 1;
+            if (!mbar_wait_or_abort(smem_addr(&S.tempty[acc]), ((lt >> 1) & 1) ^ 1, g.status, abort)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_thread_sync();
+            const uint32_t d_tmem = tmem + uint32_t(acc * kBN);
+            for (int kb = 0; kb < nkb; ++kb, ++it) {
+                const int s = it % kGemmStages;
+                if (!mbar_wait_or_abort(smem_addr(&S.full[s]), (it / kGemmStages) & 1, g.status, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_thread_sync();
+                const uint32_t a_s = smem_addr(S.a[s]), b_s = smem_addr(S.b[s]);
+                #pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk) {
+                    const uint64_t ad = A_MN ? tc::smem_desc_sw128(a_s + kk * 2048, 8192, 1024)
+                                             : tc::smem_desc_sw128(a_s + kk * 32, 16, 1024);
+                    const uint64_t bd = B_MN ? tc::smem_desc_sw128(b_s + kk * 2048, 8192, 1024)
+                                             : tc::smem_desc_sw128(b_s + kk * 32, 16, 1024);
+                    tc::mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                }
+                tc::mma_commit(smem_addr(&S.empty[s]));   // stage reusable once these MMAs retire
+            }
+            if (!ok) break;
+            tc::mma_commit(smem_addr(&S.tfull[acc]));     // accumulator ready for the epilogue
+        }
+        // no MMA may still be running when tensor memory is released
+        tc::mma_commit(smem_addr(&S.drain));
+        mbar_wait_bounded<false>(smem_addr(&S.drain), 0, nullptr);
+    } else if (warp >= 2) {
+        // ------------------------------ epilogue ------------------------------
+        const int quarter = warp & 3;               // tensor-memory lanes 32*quarter .. +31
+        const int r_in_tile = quarter * 32 + lane;
+        const bool kempty = nkb == 0;
+        int lt = 0;
+        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
+            const int acc = lt & 1;
+            const int m0 = (tile % m_tiles) * kBM;
+            const int nt = tile / m_tiles;
+            const int n0 = nt * kBN;
+            const int m = m0 + r_in_tile;
+            if (!kempty) {
+                // warp-uniform exit: tcgen05.ld below needs all 32 lanes
+                const bool got = mbar_wait_or_abort(smem_addr(&S.tfull[acc]), (lt >> 1) & 1, g.status, abort);
+                if (__any_sync(0xffffffffu, !got)) break;
+                tc::fence_after_thread_sync();
+            }
+            const uint32_t taddr = tmem + uint32_t(acc * kBN) + (uint32_t(quarter * 32) << 16);
+
+            if (EPI == EPI_LSE) {
+                const bool rv = m < M;
+                const int tg = rv ? __ldg(&g.list[m].y) : -1;
+                float mx = -INFINITY, sm = 0.f, xyv = 0.f;
+                bool have_xy = false;
+                for (int c = 0; c < kBN / 32; ++c) {
+                    uint32_t r[32];
+                    tc::tmem_ld_32x32b_x32(taddr + c * 32, r);
+                    tc::tmem_ld_wait();
+                    const int cb = g.col0 + n0 + c * 32;
+                    float cm = -INFINITY;
+                    #pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float f = __uint_as_float(r[j]);
+                        if (cb + j < g.vocab) cm = fmaxf(cm, f);
+                        if (cb + j == tg) { xyv = f; have_xy = true; }
+                    }
+                    if (cm > mx) {
+                        sm = (mx == -INFINITY) ? 0.f : sm * exp2f((mx - cm) * 1.4426950408889634f);
+                        mx = cm;
+                    }
+                    if (mx != -INFINITY) {
+                        const float mb = mx * 1.4426950408889634f;
+                        #pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (cb + j < g.vocab) sm += exp2f(fmaf(__uint_as_float(r[j]), 1.4426950408889634f, -mb));
+                    }
+                }
+                tc::fence_before_thread_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
+                if (rv) {
+                    g.part[size_t(m) * g.part_ld + nt] = make_float2(mx, sm);
+                    if (have_xy) g.xy[m] = xyv;
+                }
+            } else if (EPI == EPI_DZ) {
+                const bool rv = m < M;
+                int tg = -1;
+                float coef = 0.f, lb = 0.f;
+                if (rv) {
+                    const int4 e = __ldg(&g.list[m]);
+                    tg = e.y;
+                    coef = g.grad_scale * __int_as_float(e.z);
+                    lb = g.lse[m] * 1.4426950408889634f;
+                }
+                uint16_t* drow = g.dz + size_t(m) * g.dz_ld + n0;
+                for (int c = 0; c < kBN / 32; ++c) {
+                    uint32_t r[32];
+                    tc::tmem_ld_32x32b_x32(taddr + c * 32, r);
+                    tc::tmem_ld_wait();
+                    const int cb = g.col0 + n0 + c * 32;
+                    uint32_t pk[16];
+                    #pragma unroll
+                    for (int j = 0; j < 32; j += 2) {
+                        float v0 = 0.f, v1 = 0.f;
+                        if (rv && cb + j < g.vocab)
+                            v0 = coef * exp2f(fmaf(__uint_as_float(r[j]), 1.4426950408889634f, -lb)) - (cb + j == tg ? coef : 0.f);
+                        if (rv && cb + j + 1 < g.vocab)
+                            v1 = coef * exp2f(fmaf(__uint_as_float(r[j + 1]), 1.4426950408889634f, -lb)) - (cb + j + 1 == tg ? coef : 0.f);
+                        pk[j / 2] = pack_bf16x2(v0, v1);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(drow + c * 32);
+                    #pragma unroll
+                    for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                }
+                tc::fence_before_thread_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
+            } else if (EPI == EPI_DH) {
+                float* hrow = g.dh + size_t(m) * g.d_model + n0;
+                for (int c = 0; c < kBN / 32; ++c) {
+                    uint32_t r[32];
+                    if (!kempty) {
+                        tc::tmem_ld_32x32b_x32(taddr + c * 32, r);
+                        tc::tmem_ld_wait();
+                    } else {
+                        #pragma unroll
+                        for (int j = 0; j < 32; ++j) r[j] = 0u;
+                    }
+                    if (n0 + c * 32 < g.d_model) {
+                        float4* dst = reinterpret_cast<float4*>(hrow + c * 32);
+                        #pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            float4 v = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                                   __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+                            if (g.accumulate) {
+                                const float4 o = dst[j];
+                                v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
+                            }
+                            dst[j] = v;
+                        }
+                    }
+                }
+                if (!kempty) {
+                    tc::fence_before_thread_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
+                }
+            } else {  // EPI_DW
+                const int vrow = g.col0 + m;
+                uint16_t* wrow = g.dw + size_t(vrow) * g.d_model + n0;
+                for (int c = 0; c < kBN / 32; ++c) {
+                    uint32_t r[32];
+                    if (!kempty) {
+                        tc::tmem_ld_32x32b_x32(taddr + c * 32, r);
+                        tc::tmem_ld_wait();
+                    } else {
+                        #pragma unroll
+                        for (int j = 0; j < 32; ++j) r[j] = 0u;
+                    }
+                    if (vrow < g.vocab && n0 + c * 32 < g.d_model) {
+                        uint32_t pk[16];
+                        #pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                        uint4* dst = reinterpret_cast<uint4*>(wrow + c * 32);
+                        #pragma unroll
+                        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    }
+                }
+                if (!kempty) {
+                    tc::fence_before_thread_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
+                }
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc::fence_after_thread_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// small kernels around the GEMMs
+// ---------------------------------------------------------------------------
+// H_M[m] = H[list[m].row] for m < M, zero rows up to round_up(M, 128).
+__global__ void k_gather(const WsHeader* hdr, const int4* list, const uint16_t* __restrict__ H, int D,
+                         uint16_t* __restrict__ HM) {
+    const int M = hdr->n_scored;
+    const int Mp = round_up_dev(M, kBM);
+    const int vecs = D / 8;
+    for (int r = blockIdx.x; r < Mp; r += gridDim.x) {
+        uint4* dst = reinterpret_cast<uint4*>(HM + size_t(r) * D);
+        if (r < M) {
+            const uint4* src = reinterpret_cast<const uint4*>(H + size_t(__ldg(&list[r].x)) * D);
+            for (int i = threadIdx.x; i < vecs; i += blockDim.x) dst[i] = __ldg(src + i);
+        } else {
+            for (int i = threadIdx.x; i < vecs; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+// lse per masked row from the per-tile partials (fixed order), row losses:
+// row_loss[row] = w (lse - z_target) for masked rows, 0 for all other rows.
+__global__ void k_lse(const WsHeader* hdr, const int4* list, const float2* __restrict__ part, int part_ld,
+                      const float* __restrict__ xy, float* __restrict__ lse, float* __restrict__ row_loss) {
+    const int M = hdr->n_scored;
+    const int R = hdr->n_rows;
+    const int warp_g = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nwarps = (gridDim.x * blockDim.x) >> 5;
+    for (int m = warp_g; m < R; m += nwarps) {
+        const int4 e = list[m];
+        if (m >= M) {
+            if (lane == 0) row_loss[e.x] = 0.f;
+            continue;
+        }
+        float mx = -INFINITY, s = 0.f;
+        for (int t = lane; t < part_ld; t += 32) {
+            const float2 v = part[size_t(m) * part_ld + t];
+            if (v.x == -INFINITY) continue;
+            if (v.x > mx) { s = (mx == -INFINITY ? 0.f : s * exp2f((mx - v.x) * 1.4426950408889634f)) + v.y; mx = v.x; }
+            else          { s += v.y * exp2f((v.x - mx) * 1.4426950408889634f); }
+        }
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, mx, o);
+            const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+            if (m2 != -INFINITY) {
+                if (mx == -INFINITY) { mx = m2; s = s2; }
+                else {
+                    const float Mx = fmaxf(mx, m2);
+                    s = s * exp2f((mx - Mx) * 1.4426950408889634f) + s2 * exp2f((m2 - Mx) * 1.4426950408889634f);
+                    mx = Mx;
+                }
+            }
+        }
+        if (lane == 0) {
+            const float l = mx + logf(s);
+            lse[m] = l;
+            row_loss[e.x] = __int_as_float(e.z) * (l - xy[m]);
+        }
+    }
+}
+
+// d_hidden[row] = bf16(dH_M[m]) for the masked rows, 0 for all other rows.
+__global__ void k_scatter_dh(const WsHeader* hdr, const int4* list, const float* __restrict__ dh, int D,
+                             uint16_t* __restrict__ d_hidden) {
+    const int M = hdr->n_scored;
+    const int R = hdr->n_rows;
+    const int vecs = D / 8;
+    for (int i = blockIdx.x; i < R; i += gridDim.x) {
+        const int row = list[i].x;
+        uint4* dst = reinterpret_cast<uint4*>(d_hidden + size_t(row) * D);
+        if (i < M) {
+            const float4* src = reinterpret_cast<const float4*>(dh + size_t(i) * D);
+            for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
+                const float4 a = src[2 * v], b = src[2 * v + 1];
+                dst[v] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                                    pack_bf16x2(b.z, b.w));
+            }
+        } else {
+            for (int v = threadIdx.x; v < vecs; v += blockDim.x) dst[v] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+struct LinWs {
+    size_t list, row_loss, unit_acc, hm, part, xy, lse, dz, dh, total;
+    int tpad, n_tiles;
+};
+
+static LinWs lin_ws(int64_t T, int64_t units, int D, int V) {
+    LinWs w;
+    w.tpad = int(align_up(size_t(T > 0 ? T : 1), kBM));
+    w.n_tiles = (V + kBN - 1) / kBN;
+    size_t o = kWsAlign;
+    w.list = o;     o = align_up(o + size_t(T) * 16, kWsAlign);
+    w.row_loss = o; o = align_up(o + size_t(T) * 4, kWsAlign);
+    w.unit_acc = o; o = align_up(o + size_t(units) * 8, kWsAlign);
+    w.hm = o;       o = align_up(o + size_t(w.tpad) * D * 2, 1024);
+    w.part = o;     o = align_up(o + size_t(w.tpad) * w.n_tiles * 8, kWsAlign);
+    w.xy = o;       o = align_up(o + size_t(w.tpad) * 4, kWsAlign);
+    w.lse = o;      o = align_up(o + size_t(w.tpad) * 4, kWsAlign);
+    w.dz = o;       o = align_up(o + size_t(w.tpad) * kVc * 2, 1024);
+    w.dh = o;       o = align_up(o + size_t(w.tpad) * D * 4, kWsAlign);
+    w.total = o;
+    return w;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::mutex mu;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::lock_guard<std::mutex> g(mu);
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    }
+    return fn;
+}
+
+// 2-D bf16 tensor [outer, inner] (row stride `stride_elems`), box
+// [box_outer, box_inner] with 128-byte swizzle (box_inner * 2 must be 128).
+static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t stride_elems,
+                     uint32_t box_inner, uint32_t box_outer) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {stride_elems * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int EPI, bool A_MN, bool B_MN>
+static dlm_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g, int grid,
+                                cudaStream_t s) {
+    auto kern = k_gemm<EPI, A_MN, B_MN>;
+    const size_t smem = sizeof(GemmSmem) + 1024;
+    static std::mutex mu;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+            if (e != cudaSuccess) return cuda_status(e, "k_gemm smem attribute");
+            attr_done[dev] = true;
+        }
+    }
+    kern<<<grid, kGemmThreads, smem, s>>>(a, b, g);
+    return last_launch_status("k_gemm launch");
+}
+
+}  // namespace dlm
+
+using namespace dlm;
+
+extern "C" size_t dlm_linear_loss_workspace_size(const dlm_layout_t* layout, int32_t d_model, int32_t vocab) {
+    if (!layout || d_model <= 0 || vocab <= 0) return 0;
+    return lin_ws(layout->n_tokens, layout->n_units, d_model, vocab).total;
+}
+
+extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16_t* hidden,
+                                                const uint16_t* weight, int32_t d_model, int32_t vocab,
+                                                const int32_t* clean_ids, const uint8_t* corrupted,
+                                                const float* p, float grad_scale, float* loss,
+                                                float* unit_loss, uint16_t* d_hidden, uint16_t* d_weight,
+                                                void* workspace, size_t workspace_bytes, dlm_stream_t stream) {
+    if (!layout_ok(layout)) return DLM_ERR_INVALID_ARGUMENT;
+    if (d_model <= 0 || d_model % 64 != 0 || vocab <= 0 || vocab % 8 != 0) return DLM_ERR_INVALID_ARGUMENT;
+    if (!loss || !workspace) return DLM_ERR_INVALID_ARGUMENT;
+    const int64_t T = layout->n_tokens;
+    if (T > 0 && (!hidden || !weight || !clean_ids || !corrupted || !p || !d_hidden)) return DLM_ERR_INVALID_ARGUMENT;
+    if (T > 0 && !layout->cu_seqlens && layout->seq_len == 0) return DLM_ERR_INVALID_ARGUMENT;
+    if (!aligned16(hidden) || !aligned16(weight) || !aligned16(d_hidden) || (d_weight && !aligned16(d_weight)))
+        return DLM_ERR_INVALID_ARGUMENT;
+    if (reinterpret_cast<uintptr_t>(workspace) % 1024) return DLM_ERR_INVALID_ARGUMENT;
+    const LinWs W = lin_ws(T, layout->n_units, d_model, vocab);
+    if (workspace_bytes < W.total) return DLM_ERR_WORKSPACE_TOO_SMALL;
+    dlm_status_t st = check_device();
+    if (st != DLM_OK) return st;
+
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+    int4* list = reinterpret_cast<int4*>(ws + W.list);
+    float* row_loss = reinterpret_cast<float*>(ws + W.row_loss);
+    double* unit_acc = reinterpret_cast<double*>(ws + W.unit_acc);
+    uint16_t* HM = reinterpret_cast<uint16_t*>(ws + W.hm);
+    float2* part = reinterpret_cast<float2*>(ws + W.part);
+    float* xy = reinterpret_cast<float*>(ws + W.xy);
+    float* lse = reinterpret_cast<float*>(ws + W.lse);
+    uint16_t* dz = reinterpret_cast<uint16_t*>(ws + W.dz);
+    float* dh = reinterpret_cast<float*>(ws + W.dh);
+
+    // 1. which rows are scored, their targets and weights (absorbing, aligned)
+    if ((st = launch_plan(layout, clean_ids, corrupted, p, DLM_ABSORBING, DLM_ALIGNED, nullptr, nullptr, 0.f,
+                          vocab, hdr, list, s)) != DLM_OK)
+        return st;
+    if (T == 0) {
+        if (d_weight) {
+            cudaError_t e = cudaMemsetAsync(d_weight, 0, size_t(vocab) * d_model * 2, s);
+            if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync d_weight");
+        }
+        return launch_reduce(layout, nullptr, row_loss, unit_acc, unit_loss, loss, hdr, s);
+    }
+
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+
+    // 2. gather the masked rows of H (zero padding to a 128-row tile)
+    k_gather<<<sms * 4, 256, 0, s>>>(hdr, list, hidden, d_model, HM);
+    if ((st = last_launch_status("k_gather launch")) != DLM_OK) return st;
+
+    // tensor maps (shapes are host-known upper bounds; the kernels read M)
+    CUtensorMap mHM_K, mW_K, mDZ_K, mW_MN, mDZ_MN, mHM_MN;
+    bool ok = make_map(&mHM_K, HM, d_model, W.tpad, d_model, 64, kBM) &&
+              make_map(&mW_K, weight, d_model, vocab, d_model, 64, kBN) &&
+              make_map(&mDZ_K, dz, kVc, W.tpad, kVc, 64, kBM) &&
+              make_map(&mW_MN, weight, d_model, vocab, d_model, 64, 64) &&
+              make_map(&mDZ_MN, dz, kVc, W.tpad, kVc, 64, 64) &&
+              make_map(&mHM_MN, HM, d_model, W.tpad, d_model, 64, 64);
+    if (!ok) {
+        record_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+        return DLM_ERR_CUDA;
+    }
+
+    GemmArgs g{};
+    g.hdr = hdr;
+    g.status = &hdr->status;
+    g.list = list;
+    g.vocab = vocab;
+    g.d_model = d_model;
+    g.grad_scale = grad_scale;
+
+    // 3. forward: lse partials over the whole vocabulary
+    {
+        GemmArgs a = g;
+        a.m_dev = 1; a.n_cols = vocab; a.k_dev = 0; a.k_len = d_model; a.b_off = 0; a.col0 = 0;
+        a.part = part; a.part_ld = W.n_tiles; a.xy = xy;
+        if ((st = launch_gemm<EPI_LSE, false, false>(mHM_K, mW_K, a, sms, s)) != DLM_OK) return st;
+    }
+    k_lse<<<sms, 256, 0, s>>>(hdr, list, part, W.n_tiles, xy, lse, row_loss);
+    if ((st = last_launch_status("k_lse launch")) != DLM_OK) return st;
+
+    // 4. backward, one vocabulary chunk at a time
+    for (int c0 = 0; c0 < vocab; c0 += kVc) {
+        const int vc = vocab - c0 < kVc ? vocab - c0 : kVc;
+        GemmArgs a = g;
+        a.m_dev = 1; a.n_cols = int(align_up(vc, kBN)); a.k_dev = 0; a.k_len = d_model; a.b_off = c0; a.col0 = c0;
+        a.lse = lse; a.dz = dz; a.dz_ld = kVc;
+        if ((st = launch_gemm<EPI_DZ, false, false>(mHM_K, mW_K, a, sms, s)) != DLM_OK) return st;
+
+        GemmArgs h = g;
+        h.m_dev = 1; h.n_cols = d_model; h.k_dev = 0; h.k_len = int(align_up(vc, kBK)); h.b_off = c0;
+        h.dh = dh; h.accumulate = c0 > 0;
+        if ((st = launch_gemm<EPI_DH, false, true>(mDZ_K, mW_MN, h, sms, s)) != DLM_OK) return st;
+
+        if (d_weight) {
+            GemmArgs w = g;
+            w.m_dev = 0; w.m_rows = int(align_up(vc, kBM)); w.n_cols = d_model; w.k_dev = 1; w.b_off = 0;
+            w.col0 = c0; w.dw = d_weight;
+            if ((st = launch_gemm<EPI_DW, true, true>(mDZ_MN, mHM_MN, w, sms, s)) != DLM_OK) return st;
+        }
+    }
+
+    // 5. d_hidden (zero rows for unscored tokens) and the reductions
+    k_scatter_dh<<<sms * 4, 256, 0, s>>>(hdr, list, dh, d_model, d_hidden);
+    if ((st = last_launch_status("k_scatter_dh launch")) != DLM_OK) return st;
+    return launch_reduce(layout, nullptr, row_loss, unit_acc, unit_loss, loss, hdr, s);
 }
