@@ -411,29 +411,23 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
             const int st = seq % kStages;
             mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort);
             const int e0 = c * kChunk;
-            float x[kVecPerThread * 8];
+            uint4 raw[kVecPerThread];
             float cm = -INFINITY;
             #pragma unroll
             for (int j = 0; j < kVecPerThread; ++j) {
                 const int vi = tid + j * kConsumers;
                 const int col = e0 + vi * 8;
                 if (col < V) {
-                    const uint4 r = S.ring[st][vi];
-                    const uint32_t wv[4] = {r.x, r.y, r.z, r.w};
-                    #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        x[j * 8 + 2 * h] = bf16lo(wv[h]);
-                        x[j * 8 + 2 * h + 1] = bf16hi(wv[h]);
+                    raw[j] = S.ring[st][vi];
+                    cm = fmaxf(cm, bf16x8_max(raw[j]));
+                    const unsigned dy = unsigned(y - col);
+                    if (dy < 8u) {
+                        const uint32_t wv = dy < 2u ? raw[j].x : dy < 4u ? raw[j].y : dy < 6u ? raw[j].z : raw[j].w;
+                        S.xy[par] = (dy & 1u) ? bf16hi(wv) : bf16lo(wv);
                     }
-                    #pragma unroll
-                    for (int h = 0; h < 8; ++h)
-                        if (y == col + h) S.xy[par] = x[j * 8 + h];
                 } else {
-                    #pragma unroll
-                    for (int h = 0; h < 8; ++h) x[j * 8 + h] = -INFINITY;
+                    raw[j] = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);   // bf16 -inf
                 }
-                #pragma unroll
-                for (int h = 0; h < 8; ++h) cm = fmaxf(cm, x[j * 8 + h]);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&S.empty[st]));
@@ -444,7 +438,14 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
             if (m != -INFINITY) {
                 const float mb = m * kLog2e;
                 #pragma unroll
-                for (int h = 0; h < kVecPerThread * 8; ++h) s += exp2f(fmaf(x[h], kLog2e, -mb));
+                for (int j = 0; j < kVecPerThread; ++j) {
+                    const uint32_t wv[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
+                    #pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        s += exp2f(fmaf(bf16lo(wv[h]), kLog2e, -mb));
+                        s += exp2f(fmaf(bf16hi(wv[h]), kLog2e, -mb));
+                    }
+                }
             }
         }
         // block combine among the consumer warps
@@ -460,8 +461,12 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
         #pragma unroll
         for (int i = 1; i < kConsumerWarps; ++i) lse_combine(M, Ssum, S.red_m[par][i], S.red_s[par][i]);
         const float lse = M + logf(Ssum);
-        const float lb = lse * kLog2e;
         const float coef = P.grad_scale * w;
+        // g = coef * 2^(x log2e - lse log2e); for coef > 0 the factor folds
+        // into the exponent (one FFMA + one exp2 per element)
+        const bool fold = coef > 0.f;
+        const float lb = lse * kLog2e - (fold ? log2f(coef) : 0.f);
+        const float mul = fold ? 1.f : coef;
 
         // pass 2: gradient
         for (int c = 0; c < nch; ++c, ++seq) {
@@ -479,12 +484,19 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
                     float g[8];
                     #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        g[2 * h] = coef * exp2f(fmaf(bf16lo(wv[h]), kLog2e, -lb));
-                        g[2 * h + 1] = coef * exp2f(fmaf(bf16hi(wv[h]), kLog2e, -lb));
+                        g[2 * h] = exp2f(fmaf(bf16lo(wv[h]), kLog2e, -lb));
+                        g[2 * h + 1] = exp2f(fmaf(bf16hi(wv[h]), kLog2e, -lb));
                     }
-                    #pragma unroll
-                    for (int h = 0; h < 8; ++h)
-                        if (y == col + h) g[h] -= coef;
+                    if (!fold) {
+                        #pragma unroll
+                        for (int h = 0; h < 8; ++h) g[h] *= mul;
+                    }
+                    const unsigned dy = unsigned(y - col);
+                    if (dy < 8u) {
+                        #pragma unroll
+                        for (int h = 0; h < 8; ++h)
+                            if (dy == unsigned(h)) g[h] -= coef;
+                    }
                     outv[j] = make_uint4(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]),
                                          pack_bf16x2(g[4], g[5]), pack_bf16x2(g[6], g[7]));
                 }

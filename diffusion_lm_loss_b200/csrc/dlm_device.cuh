@@ -48,6 +48,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t b) { return __uint_as_float(uint32_t(b) << 16); }
+// max of the 8 bf16 values of a 16-byte vector (packed max, then one unpack)
+__device__ __forceinline__ float bf16x8_max(uint4 r) {
+    const __nv_bfloat162 a = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&r.x),
+                                     *reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    const __nv_bfloat162 b = __hmax2(*reinterpret_cast<const __nv_bfloat162*>(&r.z),
+                                     *reinterpret_cast<const __nv_bfloat162*>(&r.w));
+    const __nv_bfloat162 c = __hmax2(a, b);
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(&c);
+    return fmaxf(bf16lo(w), bf16hi(w));
+}
 
 // ---------------------------------------------------------------------------
 // PTX wrappers
@@ -92,6 +102,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Same, but the thread may sleep (up to `ns`) until the phase completes
+// instead of spinning: the hardware wakes it when the barrier flips, so a
+// waiting warp takes no issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -107,16 +130,16 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // pipeline ends the kernel instead of hanging the GPU.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s; a healthy wait is microseconds
 
+constexpr uint32_t kSleepHintNs = 20000;
+
 template <bool kCluster>
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, uint32_t* status) {
-    #pragma unroll 1
-    for (int i = 0; i < 32; ++i) {
-        if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
-    }
+    if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     #pragma unroll 1
     while (true) {
-        if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
+        if (kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait_sleep(bar, parity, kSleepHintNs))
+            return true;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             if (status) atomicOr(status, DLM_DEV_WAIT_TIMEOUT);
             return false;
@@ -234,13 +257,11 @@ __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t count) 
 // raised `abort` (shared flag).  Returns false on timeout or abort.
 __device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t parity, uint32_t* status,
                                                    volatile int* abort) {
-    #pragma unroll 1
-    for (int i = 0; i < 64; ++i)
-        if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     #pragma unroll 1
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, kSleepHintNs)) return true;
         if (*abort) return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             if (status) atomicOr(status, DLM_DEV_WAIT_TIMEOUT);
