@@ -142,6 +142,21 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+def reduce_over_ranks(ms: float, loss_ms: float, scored: float, device):
+    """Whole-job numbers: the slowest rank's times (max) and the scored
+    tokens of all ranks (sum).  Plumbing only (a few scalars); no-op on one
+    rank."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([ms, loss_ms], dtype=torch.float64, device=device)
+    n = torch.tensor([scored], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t[0]), float(t[1]), float(n[0])
+
+
 def algorithmic_ce_bytes(rows: int, scored: int, vocab: int) -> int:
     """Bytes the weighted-CE fwd+bwd must move per launch: each scored row is
     read once (2V) and every row's bf16 gradient written once (2V); plus the
@@ -239,13 +254,7 @@ def run_ours(args):
                 tot += corr.sum(dtype=torch.int64)
         scored = int(tot.item())
 
-    t_all = torch.tensor([ms, loss_ms], dtype=torch.float64, device=dev)
-    n_all = torch.tensor([scored], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_all, op=dist.ReduceOp.MAX)
-        dist.all_reduce(n_all, op=dist.ReduceOp.SUM)
-    ms, loss_ms = float(t_all[0]), float(t_all[1])
-    scored_all = float(n_all[0])
+    ms, loss_ms, scored_all = reduce_over_ranks(ms, loss_ms, scored, dev)
     value = scored_all / (ms / 1e3)
 
     # e2e: inputs from pinned host memory, H2D + step + D2H of the loss
