@@ -38,7 +38,8 @@ STATUS = {0: "DLM_OK", 1: "DLM_ERR_INVALID_ARGUMENT", 2: "DLM_ERR_UNSUPPORTED",
 
 # every symbol include/dlm.h declares
 EXPORTS = ("dlm_status_string", "dlm_last_cuda_error", "dlm_version", "dlm_sample_t", "dlm_corrupt",
-           "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_linear_loss_workspace_size",
+           "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_loss_fwd_bwd_static",
+           "dlm_linear_loss_workspace_size",
            "dlm_linear_loss_fwd_bwd", "dlm_get_device_status")
 
 
@@ -104,6 +105,9 @@ def lib():
     L.dlm_loss_fwd_bwd.restype = ctypes.c_int
     L.dlm_loss_fwd_bwd.argtypes = [lp, vp, i64, i32, vp, vp, vp, i32, i32, lp, vp, i64, vp, f32,
                                    f32, vp, vp, vp, vp, vp, sz, vp]
+    L.dlm_loss_fwd_bwd_static.restype = ctypes.c_int
+    L.dlm_loss_fwd_bwd_static.argtypes = [lp, vp, i64, i32, vp, vp, vp, i32, i32, lp, vp, i64, vp, f32,
+                                          f32, vp, vp, vp, vp, vp]
     L.dlm_linear_loss_workspace_size.restype = sz
     L.dlm_linear_loss_workspace_size.argtypes = [lp, i32, i32]
     L.dlm_linear_loss_fwd_bwd.restype = ctypes.c_int

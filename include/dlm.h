@@ -197,6 +197,40 @@ DLM_API dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t *layout, const uint16_t
                               void *workspace, size_t workspace_bytes, dlm_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * dlm_loss_fwd_bwd_static -- dlm_loss_fwd_bwd without a caller workspace.
+ * No counterpart on the pages: this entry point exists for callers that are
+ * not allowed to call cudaMalloc (code handed only its input and output
+ * buffers by a host program that owns all device memory, e.g. a plugin in
+ * another framework or a process held to a fixed memory pool), and that
+ * therefore cannot provide the workspace dlm_loss_fwd_bwd takes.
+ *
+ * Same arguments and results as dlm_loss_fwd_bwd, minus the workspace.  The
+ * scratch is a fixed device array of DLM_STATIC_SCRATCH_BYTES inside this
+ * library, held by every GPU that loads the library until the process exits;
+ * the call allocates nothing.  A problem whose dlm_loss_workspace_size()
+ * exceeds DLM_STATIC_SCRATCH_BYTES is refused with
+ * DLM_ERR_WORKSPACE_TOO_SMALL before anything is enqueued (2 MiB fits about
+ * 100,000 logits rows, diffusion plus encoder, over a few thousand units).
+ * The first call on a device looks up the array's device address with that
+ * device current and caches it; make that first call before any stream
+ * capture.  All calls share the one array: calls that overlap on the GPU (on
+ * different streams, or from different host threads without ordering) race
+ * and corrupt each other's results; order them on one stream.  Each call
+ * re-initialises what it needs, so contents left by an earlier call are
+ * harmless.  The device status word of these calls is not readable from
+ * outside (use dlm_loss_fwd_bwd with a workspace when you need it).
+ * ---------------------------------------------------------------------- */
+#define DLM_STATIC_SCRATCH_BYTES (2u << 20)
+
+DLM_API dlm_status_t dlm_loss_fwd_bwd_static(const dlm_layout_t *layout, const uint16_t *logits,
+                              int64_t ld, int32_t vocab, const int32_t *clean_ids,
+                              const uint8_t *corrupted, const float *p, int32_t mode, int32_t align,
+                              const dlm_layout_t *enc_layout, const uint16_t *enc_logits,
+                              int64_t enc_ld, const int32_t *enc_ids, float enc_ar_weight,
+                              float grad_scale, float *loss, float *unit_loss,
+                              uint16_t *dlogits, uint16_t *enc_dlogits, dlm_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * dlm_linear_loss_fwd_bwd -- the absorbing, aligned loss above with
  * logits = hidden @ weight^T formed tile by tile on the tensor cores and never
  * written to memory ("Native diffusion language-model training", Adapters,
