@@ -21,6 +21,9 @@
 //            main loop of tile i+1)
 //   warps 2-5  epilogue: tensor memory -> registers -> (partials | dZ |
 //            dH accumulate | dW store)
+// Tile raster: the forward and dZ GEMMs walk M fastest (H_M, the small
+// operand, stays in L2 while W streams once); the dH and dW GEMMs walk N
+// fastest so the dZ chunk (the large operand) streams once per wave.
 // Every wait is bounded (a broken pipeline sets DLM_DEV_WAIT_TIMEOUT and the
 // kernel winds down instead of hanging).
 #include <cstdio>
@@ -52,6 +55,7 @@ struct GemmArgs {
     int n_cols;              // C columns
     int k_dev;               // 1: K = round_up(M, 128); 0: k_len
     int k_len;
+    int n_fastest;           // tile raster: 0 = consecutive tiles share the B tile, 1 = share the A tile
     int b_off;               // row offset of W (forward / dZ) or K offset into W rows (dH)
     int col0;                // vocabulary index of C column 0 (LSE, DZ) or C row 0 (DW)
     int vocab;
@@ -132,8 +136,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         int it = 0;
         bool ok = true;
         for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-            const int m0 = (tile % m_tiles) * kBM;
-            const int n0 = (tile / m_tiles) * kBN;
+            const int m0 = (g.n_fastest ? tile / n_tiles : tile % m_tiles) * kBM;
+            const int n0 = (g.n_fastest ? tile % n_tiles : tile / m_tiles) * kBN;
             for (int kb = 0; kb < nkb; ++kb, ++it) {
                 const int s = it % kGemmStages;
                 if (!mbar_wait_or_abort(smem_addr(&S.empty[s]), ((it / kGemmStages) & 1) ^ 1, g.status, abort)) {
@@ -208,8 +212,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         int lt = 0;
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
             const int acc = lt & 1;
-            const int m0 = (tile % m_tiles) * kBM;
-            const int nt = tile / m_tiles;
+            const int m0 = (g.n_fastest ? tile / n_tiles : tile % m_tiles) * kBM;
+            const int nt = g.n_fastest ? tile % n_tiles : tile / m_tiles;
             const int n0 = nt * kBN;
             const int m = m0 + r_in_tile;
             if (!kempty) {
@@ -622,13 +626,13 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, cons
 
         GemmArgs h = g;
         h.m_dev = 1; h.n_cols = d_model; h.k_dev = 0; h.k_len = int(align_up(vc, kBK)); h.b_off = c0;
-        h.dh = dh; h.accumulate = c0 > 0;
+        h.dh = dh; h.accumulate = c0 > 0; h.n_fastest = 1;
         if ((st = launch_gemm<EPI_DH, false, true>(mDZ_K, mW_MN, h, sms, s)) != DLM_OK) return st;
 
         if (d_weight) {
             GemmArgs w = g;
             w.m_dev = 0; w.m_rows = int(align_up(vc, kBM)); w.n_cols = d_model; w.k_dev = 1; w.b_off = 0;
-            w.col0 = c0; w.dw = d_weight;
+            w.col0 = c0; w.dw = d_weight; w.n_fastest = 1;
             if ((st = launch_gemm<EPI_DW, true, true>(mDZ_MN, mHM_MN, w, sms, s)) != DLM_OK) return st;
         }
     }

@@ -92,6 +92,13 @@ WORKLOADS = {
         h_std=1.0, w_std=0.02, data_seed=5,
         description="packed documents (lengths geometric, mean 296, 16..4096) through a fused "
                     "lm_head, T=16384 D=4096 V=126464"),
+    # a smaller case of the same kernels, sized for detailed profiling (W is
+    # still larger than L2)
+    "lin_t4096_d4096_v32768": Spec(
+        "lin_t4096_d4096_v32768", "linear", ABSORBING, ALIGNED, vocab=32768,
+        mask_id=32767, ids_high=32000, n_tokens_packed=4096, d_model=4096,
+        h_std=1.0, w_std=0.02, data_seed=5,
+        description="packed documents through a fused lm_head, T=4096 D=4096 V=32768"),
 }
 
 
