@@ -88,36 +88,32 @@ __device__ __forceinline__ void unit_pos(const LayoutDev& L, int64_t i, int& u, 
     }
 }
 
-// Target of row q (or -1) and its unit.  Rows [0, a.n_tokens) are diffusion
-// rows, the rest encoder rows.
+// Target of row q (or -1), its unit, and the row's unit's p (absorbing
+// weight).  Rows [0, a.n_tokens) are diffusion rows, the rest encoder rows.
+// All loads are issued unconditionally (in bounds), so the loads of several
+// rows can be in flight together.
 __device__ __forceinline__ void classify(const PlanParams& P, int64_t q, int& target, int& unit,
                                          bool& bad_id) {
     target = -1;
     bad_id = false;
-    if (q < P.a.n_tokens) {
-        int64_t end;
-        unit_pos(P.a, q, unit, end);
-        int64_t j = P.align == DLM_ALIGNED ? q : q + 1;
-        if (j >= end || j >= P.a.n_tokens) return;
-        if (P.a.pad && P.a.pad[j]) return;
-        if (P.mode == DLM_ABSORBING && !P.corrupted[j]) return;
-        int y = P.clean_a[j];
-        if (y < 0 || y >= P.vocab) { bad_id = true; return; }
-        target = y;
-    } else {
-        const int64_t i = q - P.a.n_tokens;
-        int64_t end;
-        unit_pos(P.b, i, unit, end);
-        const int64_t j = i + 1;
-        if (j >= end || j >= P.b.n_tokens) return;
-        if (P.b.pad && P.b.pad[j]) return;
-        int y = P.ids_b[j];
-        if (y < 0 || y >= P.vocab) { bad_id = true; return; }
-        target = y;
-    }
+    const bool in_a = q < P.a.n_tokens;
+    const LayoutDev& L = in_a ? P.a : P.b;
+    const int64_t i = in_a ? q : q - P.a.n_tokens;
+    int64_t end;
+    unit_pos(L, i, unit, end);
+    const int64_t j = (in_a && P.align == DLM_ALIGNED) ? i : i + 1;
+    const bool inr = j < end && j < L.n_tokens;
+    const int64_t jj = inr ? j : 0;
+    const bool pad = inr && L.pad && L.pad[jj];
+    const bool cor = !(in_a && P.mode == DLM_ABSORBING) || (inr && P.corrupted[jj]);
+    const int y = inr ? (in_a ? P.clean_a[jj] : P.ids_b[jj]) : -1;
+    if (!inr || pad || !cor) return;
+    if (y < 0 || y >= P.vocab) { bad_id = true; return; }
+    target = y;
 }
 
-constexpr int kPlanThreads = 1024;
+constexpr int kPlanThreads = 512;
+constexpr int kPlanWarps = kPlanThreads / 32;
 
 __device__ __forceinline__ bool layout_bad(const LayoutDev& L) {
     // every thread checks a strided part of cu_seqlens
@@ -132,64 +128,82 @@ __device__ __forceinline__ bool layout_bad(const LayoutDev& L) {
     return bad;
 }
 
-__global__ void __launch_bounds__(kPlanThreads) k_plan(PlanParams P) {
-    __shared__ int s_cnt[kPlanThreads];
-    __shared__ int s_red[4][32];
-    __shared__ int s_tot[4];
+constexpr int kPlanCacheRows = 16384;   // rows whose classification is kept in shared memory
+
+// Exclusive block scan of one int per thread (kPlanThreads threads): warp
+// shuffles, then one pass over the warp totals.  Also returns the block total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+    #pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < kPlanWarps ? s_warp[lane] : 0;
+        #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < kPlanWarps) s_warp[lane] = w;   // inclusive over warps
+    }
+    __syncthreads();
+    total = s_warp[kPlanWarps - 1];
+    return (warp ? s_warp[warp - 1] : 0) + x - v;
+}
+
+__global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
+    __shared__ int s_warp[32];
+    __shared__ int s_sum[3][kPlanWarps];
     __shared__ uint32_t s_status;
-    const int tid = threadIdx.x;
+    pdl_launch_dependents();   // the CE kernel may start its prologue now
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     if (tid == 0) s_status = 0;
+    pdl_wait();                // inputs written by earlier kernels are visible
     __syncthreads();
     if (layout_bad(P.a) || layout_bad(P.b)) atomicOr(&s_status, DLM_DEV_BAD_LAYOUT);
 
     const int64_t R = P.a.n_tokens + P.b.n_tokens;
     const int64_t chunk = (R + kPlanThreads - 1) / kPlanThreads;
     const int64_t r0 = min(R, int64_t(tid) * chunk), r1 = min(R, r0 + chunk);
+    const bool cached = R <= kPlanCacheRows;
+    extern __shared__ int2 s_rows[];   // {target, unit} per row when cached
 
-    // pass 1: counts
+    // pass 1: classify (kept in shared memory when R is small enough) and count
     int na = 0, nb = 0, nonpad = 0;
     bool any_bad = false;
+    #pragma unroll 4
     for (int64_t q = r0; q < r1; ++q) {
         int tg, u;
         bool bad;
         classify(P, q, tg, u, bad);
         any_bad |= bad;
         if (tg >= 0) { if (q < P.a.n_tokens) ++na; else ++nb; }
-        if (q < P.a.n_tokens && !(P.a.pad && P.a.pad[q])) ++nonpad;
+        if (cached) s_rows[q] = make_int2(tg, u);
     }
+    for (int64_t q = r0; q < r1 && q < P.a.n_tokens; ++q) nonpad += !(P.a.pad && P.a.pad[q]);
     if (any_bad) atomicOr(&s_status, DLM_DEV_BAD_TOKEN_ID);
-    s_cnt[tid] = na + nb;
-    // block sums of na, nb, nonpad
+
+    // block totals (na, nb, nonpad) and the exclusive scan of scored rows
     {
         int v0 = na, v1 = nb, v2 = nonpad;
+        #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             v0 += __shfl_xor_sync(0xffffffffu, v0, o);
             v1 += __shfl_xor_sync(0xffffffffu, v1, o);
             v2 += __shfl_xor_sync(0xffffffffu, v2, o);
         }
-        if ((tid & 31) == 0) { s_red[0][tid >> 5] = v0; s_red[1][tid >> 5] = v1; s_red[2][tid >> 5] = v2; }
+        if (lane == 0) { s_sum[0][warp] = v0; s_sum[1][warp] = v1; s_sum[2][warp] = v2; }
     }
-    __syncthreads();
-    if (tid < 32) {
-        int v0 = s_red[0][tid], v1 = s_red[1][tid], v2 = s_red[2][tid];
-        for (int o = 16; o > 0; o >>= 1) {
-            v0 += __shfl_xor_sync(0xffffffffu, v0, o);
-            v1 += __shfl_xor_sync(0xffffffffu, v1, o);
-            v2 += __shfl_xor_sync(0xffffffffu, v2, o);
-        }
-        if (tid == 0) { s_tot[0] = v0; s_tot[1] = v1; s_tot[2] = v2; }
-    }
-    // exclusive scan of per-thread scored counts (Hillis-Steele, in place)
-    for (int o = 1; o < kPlanThreads; o <<= 1) {
-        __syncthreads();
-        const int add = tid >= o ? s_cnt[tid - o] : 0;
-        __syncthreads();
-        s_cnt[tid] += add;
-    }
-    __syncthreads();
-    const int n_a = s_tot[0], n_b = s_tot[1], N = s_tot[2];
-    const int n_scored = n_a + n_b;
-    const int scored_before = s_cnt[tid] - (na + nb);
+    int n_scored;
+    const int scored_before = block_exclusive_scan(na + nb, s_warp, n_scored);
+    int n_a = 0, n_b = 0, N = 0;
+    #pragma unroll
+    for (int w = 0; w < kPlanWarps; ++w) { n_a += s_sum[0][w]; n_b += s_sum[1][w]; N += s_sum[2][w]; }
     int64_t so = scored_before;                          // next scored slot
     int64_t uo = n_scored + (r0 - scored_before);        // next unscored slot
 
@@ -197,10 +211,7 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(PlanParams P) {
     const float w_enc = n_b > 0 ? P.lam / float(n_b) : 0.0f;
 
     // pass 2: weights and the row list
-    for (int64_t q = r0; q < r1; ++q) {
-        int tg, u;
-        bool bad;
-        classify(P, q, tg, u, bad);
+    auto emit = [&](int64_t q, int tg, int u) {
         if (tg >= 0) {
             float w;
             if (q < P.a.n_tokens) {
@@ -211,6 +222,19 @@ __global__ void __launch_bounds__(kPlanThreads) k_plan(PlanParams P) {
             P.list[so++] = make_int4(int(q), tg, __float_as_int(w), u);
         } else {
             P.list[uo++] = make_int4(int(q), -1, 0, u);
+        }
+    };
+    if (cached) {
+        for (int64_t q = r0; q < r1; ++q) {
+            const int2 c = s_rows[q];
+            emit(q, c.x, c.y);
+        }
+    } else {
+        for (int64_t q = r0; q < r1; ++q) {
+            int tg, u;
+            bool bad;
+            classify(P, q, tg, u, bad);
+            emit(q, tg, u);
         }
     }
     __syncthreads();
@@ -245,7 +269,7 @@ __device__ __forceinline__ void lse_combine(float& m, float& s, float m2, float 
     if (m2 == -INFINITY) return;
     if (m == -INFINITY) { m = m2; s = s2; return; }
     const float M = fmaxf(m, m2);
-    s = s * exp2f((m - M) * kLog2e) + s2 * exp2f((m2 - M) * kLog2e);
+    s = s * ex2((m - M) * kLog2e) + s2 * ex2((m2 - M) * kLog2e);
     m = M;
 }
 
@@ -330,6 +354,8 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
     }
     fence_proxy_async_smem();   // zero block visible to the bulk-copy engine
     __syncthreads();
+    pdl_wait();                 // the row plan (previous kernel) is complete
+    pdl_launch_dependents();    // the reduction may start its prologue
 
     const int n_scored = P.hdr->n_scored;
     const int n_rows = P.hdr->n_rows;
@@ -432,7 +458,7 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&S.empty[st]));
             if (cm > m) {
-                s = (m == -INFINITY) ? 0.f : s * exp2f((m - cm) * kLog2e);
+                s = (m == -INFINITY) ? 0.f : s * ex2((m - cm) * kLog2e);
                 m = cm;
             }
             if (m != -INFINITY) {
@@ -442,8 +468,8 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
                     const uint32_t wv[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
                     #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        s += exp2f(fmaf(bf16lo(wv[h]), kLog2e, -mb));
-                        s += exp2f(fmaf(bf16hi(wv[h]), kLog2e, -mb));
+                        s += ex2(fmaf(bf16lo(wv[h]), kLog2e, -mb));
+                        s += ex2(fmaf(bf16hi(wv[h]), kLog2e, -mb));
                     }
                 }
             }
@@ -484,8 +510,8 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
                     float g[8];
                     #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        g[2 * h] = exp2f(fmaf(bf16lo(wv[h]), kLog2e, -lb));
-                        g[2 * h + 1] = exp2f(fmaf(bf16hi(wv[h]), kLog2e, -lb));
+                        g[2 * h] = ex2(fmaf(bf16lo(wv[h]), kLog2e, -lb));
+                        g[2 * h + 1] = ex2(fmaf(bf16hi(wv[h]), kLog2e, -lb));
                     }
                     if (!fold) {
                         #pragma unroll
@@ -520,6 +546,8 @@ __global__ void __launch_bounds__(kGenThreads) k_ce_generic(const CeParams P) {
     __shared__ float red_m[kGenThreads / 32], red_s[kGenThreads / 32];
     __shared__ float s_lse;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    pdl_launch_dependents();
     const int n_rows = P.hdr->n_rows;
     const int V = P.vocab;
     for (int i = blockIdx.x; i < n_rows; i += gridDim.x) {
@@ -537,8 +565,8 @@ __global__ void __launch_bounds__(kGenThreads) k_ce_generic(const CeParams P) {
         float m = -INFINITY, s = 0.f;
         for (int v = tid; v < V; v += kGenThreads) {
             const float xv = bf16_bits_to_float(x[v]);
-            if (xv > m) { s = s * exp2f((m - xv) * kLog2e) + 1.f; m = xv; }
-            else        { s += exp2f((xv - m) * kLog2e); }
+            if (xv > m) { s = s * ex2((m - xv) * kLog2e) + 1.f; m = xv; }
+            else        { s += ex2((xv - m) * kLog2e); }
         }
         #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -560,7 +588,7 @@ __global__ void __launch_bounds__(kGenThreads) k_ce_generic(const CeParams P) {
         const float coef = P.grad_scale * w;
         for (int v = tid; v < V; v += kGenThreads) {
             const float xv = bf16_bits_to_float(x[v]);
-            float g = coef * exp2f((xv - lse) * kLog2e);
+            float g = coef * ex2((xv - lse) * kLog2e);
             if (v == y) g -= coef;
             d[v] = __bfloat16_as_ushort(__float2bfloat16_rn(g));
         }
@@ -619,14 +647,32 @@ __global__ void __launch_bounds__(kRedThreads) k_reduce(ReduceParams R) {
     __shared__ bool last;
     const int tid = threadIdx.x;
     const int U = R.a.n_units;
+    pdl_wait();   // row losses of the CE kernel are complete
     for (int u = blockIdx.x; u < U; u += gridDim.x) {
-        double acc = 0.0;
+        // four independent accumulators (loads in flight together), combined
+        // in a fixed order
+        double acc[4] = {0.0, 0.0, 0.0, 0.0};
         int64_t lo, hi;
         unit_range(R.a, u, lo, hi);
-        for (int64_t i = lo + tid; i < hi; i += kRedThreads) acc += double(R.row_loss[i]);
+        {
+            int64_t i = lo + tid;
+            for (; i + 3 * kRedThreads < hi; i += 4 * kRedThreads) {
+                #pragma unroll
+                for (int k = 0; k < 4; ++k) acc[k] += double(R.row_loss[i + k * kRedThreads]);
+            }
+            for (; i < hi; i += kRedThreads) acc[0] += double(R.row_loss[i]);
+        }
         unit_range(R.b, u, lo, hi);
-        for (int64_t i = lo + tid; i < hi; i += kRedThreads) acc += double(R.row_loss[R.a.n_tokens + i]);
-        const double t = block_sum(acc, red);
+        {
+            const float* rb = R.row_loss + R.a.n_tokens;
+            int64_t i = lo + tid;
+            for (; i + 3 * kRedThreads < hi; i += 4 * kRedThreads) {
+                #pragma unroll
+                for (int k = 0; k < 4; ++k) acc[k] += double(rb[i + k * kRedThreads]);
+            }
+            for (; i < hi; i += kRedThreads) acc[0] += double(rb[i]);
+        }
+        const double t = block_sum((acc[0] + acc[1]) + (acc[2] + acc[3]), red);
         if (tid == 0) {
             R.unit_acc[u] = t;
             if (R.unit_loss) R.unit_loss[u] = float(t);
@@ -696,8 +742,22 @@ dlm_status_t launch_plan(const dlm_layout_t* a, const int32_t* clean, const uint
     pp.vocab = vocab;
     pp.hdr = hdr;
     pp.list = list;
-    k_plan<<<1, kPlanThreads, 0, s>>>(pp);
-    return last_launch_status("k_plan launch");
+    const int64_t R = (a ? a->n_tokens : 0) + (b ? b->n_tokens : 0);
+    const size_t smem = R <= kPlanCacheRows ? size_t(R) * sizeof(int2) : 0;
+    static std::mutex mu;
+    static bool attr[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> g(mu);
+        if (dev >= 0 && dev < 64 && !attr[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(k_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 int(kPlanCacheRows * sizeof(int2)));
+            if (e != cudaSuccess) return cuda_status(e, "k_plan smem attribute");
+            attr[dev] = true;
+        }
+    }
+    return launch_pdl(k_plan, dim3(1), dim3(kPlanThreads), smem, s, "k_plan launch", pp);
 }
 
 dlm_status_t launch_reduce(const dlm_layout_t* a, const dlm_layout_t* b, const float* row_loss,
@@ -713,8 +773,7 @@ dlm_status_t launch_reduce(const dlm_layout_t* a, const dlm_layout_t* b, const f
     rp.ticket = &hdr->ticket;
     const int U = a->n_units;
     const int rgrid = U < 1 ? 1 : (U > 65536 ? 65536 : U);
-    k_reduce<<<rgrid, kRedThreads, 0, s>>>(rp);
-    return last_launch_status("k_reduce launch");
+    return launch_pdl(k_reduce, dim3(rgrid), dim3(kRedThreads), 0, s, "k_reduce launch", rp);
 }
 
 }  // namespace dlm
@@ -795,12 +854,14 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (fast && stream_kernel_ready(dev)) {
             const int64_t grid = R < int64_t(sms) * kCtasPerSm ? R : int64_t(sms) * kCtasPerSm;
-            k_ce_stream<<<unsigned(grid), kStreamThreads, sizeof(StreamSmem), s>>>(cp);
-            if ((st = last_launch_status("k_ce_stream launch")) != DLM_OK) return st;
+            if ((st = launch_pdl(k_ce_stream, dim3(unsigned(grid)), dim3(kStreamThreads), sizeof(StreamSmem), s,
+                                 "k_ce_stream launch", cp)) != DLM_OK)
+                return st;
         } else {
             const int64_t grid = R < int64_t(sms) * 8 ? R : int64_t(sms) * 8;
-            k_ce_generic<<<unsigned(grid), kGenThreads, 0, s>>>(cp);
-            if ((st = last_launch_status("k_ce_generic launch")) != DLM_OK) return st;
+            if ((st = launch_pdl(k_ce_generic, dim3(unsigned(grid)), dim3(kGenThreads), 0, s,
+                                 "k_ce_generic launch", cp)) != DLM_OK)
+                return st;
         }
     }
 

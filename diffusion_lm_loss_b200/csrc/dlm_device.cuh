@@ -38,6 +38,16 @@ __device__ __forceinline__ int find_unit(const int32_t* __restrict__ cu, int n_u
     return lo;
 }
 
+// Base-2 exponential by the hardware instruction (PTX ex2.approx.ftz.f32:
+// one MUFU op, relative error about 2^-22; results below 2^-126 flush to 0).
+// The losses' exponents are x - max <= 0, so the flush only drops terms
+// smaller than 1e-38 of the row's largest.
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ---------------------------------------------------------------------------
 // bf16 helpers
 // ---------------------------------------------------------------------------
@@ -194,6 +204,15 @@ __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, float a, float
     asm volatile(
         "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
         :: "r"(remote_addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar) : "memory");
+}
+
+// Programmatic dependent launch: a kernel launched with the programmatic
+// stream-serialization attribute may start before the previous kernel in the
+// stream ends; pdl_wait() blocks until that kernel has completed and its
+// writes are visible (a no-op for kernels launched without the attribute).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------

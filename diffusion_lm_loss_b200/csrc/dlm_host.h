@@ -5,6 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <utility>
 
 #include "../../include/dlm.h"
 
@@ -30,6 +31,27 @@ inline dlm_status_t cuda_status(cudaError_t e, const char* where) {
 
 inline dlm_status_t last_launch_status(const char* where = "kernel launch") {
     return cuda_status(cudaGetLastError(), where);
+}
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream is still running; it must call
+// pdl_wait() before reading that kernel's results.
+template <typename... KArgs, typename... Args>
+inline dlm_status_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                               const char* what, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    if (e != cudaSuccess) cudaGetLastError();
+    return cuda_status(e, what);
 }
 
 // Layout sanity that the host can see (the device checks cu_seqlens itself).

@@ -242,14 +242,14 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                         if (cb + j == tg) { xyv = f; have_xy = true; }
                     }
                     if (cm > mx) {
-                        sm = (mx == -INFINITY) ? 0.f : sm * exp2f((mx - cm) * 1.4426950408889634f);
+                        sm = (mx == -INFINITY) ? 0.f : sm * ex2((mx - cm) * 1.4426950408889634f);
                         mx = cm;
                     }
                     if (mx != -INFINITY) {
                         const float mb = mx * 1.4426950408889634f;
                         #pragma unroll
                         for (int j = 0; j < 32; ++j)
-                            if (cb + j < g.vocab) sm += exp2f(fmaf(__uint_as_float(r[j]), 1.4426950408889634f, -mb));
+                            if (cb + j < g.vocab) sm += ex2(fmaf(__uint_as_float(r[j]), 1.4426950408889634f, -mb));
                     }
                 }
                 tc::fence_before_thread_sync();
@@ -280,9 +280,9 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                     for (int j = 0; j < 32; j += 2) {
                         float v0 = 0.f, v1 = 0.f;
                         if (rv && cb + j < g.vocab)
-                            v0 = coef * exp2f(fmaf(__uint_as_float(r[j]), 1.4426950408889634f, -lb)) - (cb + j == tg ? coef : 0.f);
+                            v0 = coef * ex2(fmaf(__uint_as_float(r[j]), 1.4426950408889634f, -lb)) - (cb + j == tg ? coef : 0.f);
                         if (rv && cb + j + 1 < g.vocab)
-                            v1 = coef * exp2f(fmaf(__uint_as_float(r[j + 1]), 1.4426950408889634f, -lb)) - (cb + j + 1 == tg ? coef : 0.f);
+                            v1 = coef * ex2(fmaf(__uint_as_float(r[j + 1]), 1.4426950408889634f, -lb)) - (cb + j + 1 == tg ? coef : 0.f);
                         pk[j / 2] = pack_bf16x2(v0, v1);
                     }
                     uint4* dst = reinterpret_cast<uint4*>(drow + c * 32);
@@ -398,8 +398,8 @@ __global__ void k_lse(const WsHeader* hdr, const int4* list, const float2* __res
         for (int t = lane; t < part_ld; t += 32) {
             const float2 v = part[size_t(m) * part_ld + t];
             if (v.x == -INFINITY) continue;
-            if (v.x > mx) { s = (mx == -INFINITY ? 0.f : s * exp2f((mx - v.x) * 1.4426950408889634f)) + v.y; mx = v.x; }
-            else          { s += v.y * exp2f((v.x - mx) * 1.4426950408889634f); }
+            if (v.x > mx) { s = (mx == -INFINITY ? 0.f : s * ex2((mx - v.x) * 1.4426950408889634f)) + v.y; mx = v.x; }
+            else          { s += v.y * ex2((v.x - mx) * 1.4426950408889634f); }
         }
         #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -409,7 +409,7 @@ __global__ void k_lse(const WsHeader* hdr, const int4* list, const float2* __res
                 if (mx == -INFINITY) { mx = m2; s = s2; }
                 else {
                     const float Mx = fmaxf(mx, m2);
-                    s = s * exp2f((mx - Mx) * 1.4426950408889634f) + s2 * exp2f((m2 - Mx) * 1.4426950408889634f);
+                    s = s * ex2((mx - Mx) * 1.4426950408889634f) + s2 * ex2((m2 - Mx) * 1.4426950408889634f);
                     mx = Mx;
                 }
             }
