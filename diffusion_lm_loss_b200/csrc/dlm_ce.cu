@@ -14,8 +14,9 @@
 //                 expensive rows out evenly.
 //   2. k_ce_*     the hot kernel, HBM-bound: every scored row must be read
 //                 (V*2 bytes) and every row's gradient written (V*2 bytes).
-//                 Fast path (k_ce_stream): one CTA per SM, a TMA producer warp
-//                 and 16 consumer warps; each scored row is streamed twice
+//                 Fast path (k_ce_stream): per SM one or two CTAs of a TMA
+//                 producer warp and 16 or 8 consumer warps (chosen so that
+//                 the rows in flight fit in L2); each scored row is streamed twice
 //                 through a shared-memory ring -- pass 1 from HBM (kept in L2
 //                 with an evict_last policy) for the online max / sum of exp,
 //                 pass 2 from L2 for the bf16 gradient -- and unscored rows are
@@ -284,8 +285,8 @@ __device__ __forceinline__ void row_ptrs(const CeParams& P, int q, const uint16_
     }
 }
 
-// Fast path.  Two CTAs per SM, each 8 consumer warps + 1 producer warp.  Each
-// CTA takes every G-th scored row of the list (G = grid size) and streams it
+// Fast path.  Each CTA = one TMA producer warp + WARPS consumer warps; it
+// takes every G-th scored row of the list (G = grid size) and streams it
 // twice through a ring of kStages shared-memory chunks of kChunk elements:
 //   pass 1: bulk loads from HBM with an L2 evict_last policy; per-thread
 //           online (max, sum exp) -> one block combine -> lse of the row;
@@ -295,48 +296,45 @@ __device__ __forceinline__ void row_ptrs(const CeParams& P, int q, const uint16_
 // The producer warp also zero-fills this CTA's share of the unscored rows
 // with bulk shared->global copies from a zeroed shared block, interleaved with
 // the scored rows so the zero stream overlaps the consumers' work.
-#ifndef DLM_CE_WARPS
-#define DLM_CE_WARPS 8
-#endif
-#ifndef DLM_CE_CHUNK
-#define DLM_CE_CHUNK 8192
-#endif
-#ifndef DLM_CE_STAGES
-#define DLM_CE_STAGES 6
-#endif
-#ifndef DLM_CE_CTAS_PER_SM
-#define DLM_CE_CTAS_PER_SM 2
-#endif
-constexpr int kConsumerWarps = DLM_CE_WARPS;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kStreamThreads = kConsumers + 32;
-constexpr int kChunk = DLM_CE_CHUNK;         // bf16 elements per stage
-constexpr int kStages = DLM_CE_STAGES;       // ring depth
-constexpr int kCtasPerSm = DLM_CE_CTAS_PER_SM;
-#ifndef DLM_CE_ZERO
-#define DLM_CE_ZERO 4096
-#endif
-#ifndef DLM_CE_HINTS
-#define DLM_CE_HINTS 1
-#endif
-constexpr int kZeroBytes = DLM_CE_ZERO;
-constexpr int kVecPerThread = kChunk / 8 / kConsumers;   // 16-byte vectors per thread per chunk
-static_assert(kVecPerThread * 8 * kConsumers == kChunk, "chunk split");
+constexpr int kChunk = 8192;        // bf16 elements per ring stage (16 KB)
+constexpr int kZeroBytes = 4096;    // zero block the producer copies over unscored rows
 
+// Two shapes of the kernel, chosen per call from the L2 footprint (every row
+// in flight lives in L2 between its two passes, 2V bytes each):
+//   StreamShape<8, 6>   2 CTAs/SM x 8 consumer warps, 6-stage ring  (296 rows in flight)
+//   StreamShape<16, 12> 1 CTA/SM x 16 consumer warps, 12-stage ring (148 rows in flight)
+template <int WARPS, int STAGES>
+struct StreamShape {
+    static constexpr int kWarps = WARPS;
+    static constexpr int kConsumers = WARPS * 32;
+    static constexpr int kThreads = kConsumers + 32;
+    static constexpr int kStages = STAGES;
+    static constexpr int kVec = kChunk / 8 / kConsumers;   // 16-byte vectors per thread per chunk
+    static_assert(kVec * 8 * kConsumers == kChunk, "chunk split");
+};
+
+template <int WARPS, int STAGES>
 struct __align__(128) StreamSmem {
-    uint4 ring[kStages][kChunk / 8];
+    uint4 ring[STAGES][kChunk / 8];
     uint4 zero[kZeroBytes / 16];
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
-    float red_m[2][kConsumerWarps];
-    float red_s[2][kConsumerWarps];
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    float red_m[2][WARPS];
+    float red_s[2][WARPS];
     float xy[2];
     int abort;
 };
 
-__global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const CeParams P) {
+template <int WARPS, int STAGES, int CTAS>
+__global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_ce_stream(const CeParams P) {
+    using Sh = StreamShape<WARPS, STAGES>;
+    constexpr int kConsumerWarps = Sh::kWarps;
+    constexpr int kConsumers = Sh::kConsumers;
+    constexpr int kStreamThreads = Sh::kThreads;
+    constexpr int kStages = Sh::kStages;
+    constexpr int kVecPerThread = Sh::kVec;
     extern __shared__ __align__(128) uint8_t smem_raw[];
-    StreamSmem& S = *reinterpret_cast<StreamSmem*>(smem_raw);
+    StreamSmem<WARPS, STAGES>& S = *reinterpret_cast<StreamSmem<WARPS, STAGES>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int V = P.vocab;
     const int nch = (V + kChunk - 1) / kChunk;
@@ -366,8 +364,8 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
     if (warp == kConsumerWarps) {
         // ------------------------------ producer ------------------------------
         if (lane == 0) {
-            const uint64_t pol_keep = DLM_CE_HINTS ? policy_evict_last() : policy_evict_normal();
-            const uint64_t pol_drop = DLM_CE_HINTS ? policy_evict_first() : policy_evict_normal();
+            const uint64_t pol_keep = policy_evict_last();
+            const uint64_t pol_drop = policy_evict_first();
             int seq = 0, zdone = 0;
             auto zero_row = [&](int j) {
                 const int q = P.list[n_scored + blockIdx.x + j * G].x;
@@ -393,7 +391,8 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
                         const int st = seq % kStages;
                         if (!mbar_wait_or_abort(smem_addr(&S.empty[st]), ((seq / kStages) & 1) ^ 1, P.status,
                                                 abort)) { ok = false; break; }
-                        const int e0 = c * kChunk;
+                        const int cc = c;
+                        const int e0 = cc * kChunk;
                         const uint32_t bytes = uint32_t(min(kChunk, V - e0)) * 2u;
                         const uint32_t fb = smem_addr(&S.full[st]);
                         mbar_arrive_expect_tx(fb, bytes);
@@ -416,7 +415,7 @@ __global__ void __launch_bounds__(kStreamThreads, kCtasPerSm) k_ce_stream(const 
     }
 
     // ------------------------------ consumers ------------------------------
-    const uint64_t pol_drop = DLM_CE_HINTS ? policy_evict_first() : policy_evict_normal();
+    const uint64_t pol_drop = policy_evict_first();
     int seq = 0;
     int4 e_next = my_scored > 0 ? P.list[blockIdx.x] : make_int4(0, -1, 0, 0);
     for (int k = 0; k < my_scored; ++k) {
@@ -699,20 +698,36 @@ __global__ void __launch_bounds__(kRedThreads) k_reduce(ReduceParams R) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-// Shared-memory attribute of the streaming kernel, set once per device.
+// Shared-memory attribute of a streaming-kernel shape, set once per device.
+template <int WARPS, int STAGES, int CTAS>
 static bool stream_kernel_ready(int dev) {
     static std::mutex mu;
     static int state[64];   // 0 unknown, 1 ok, 2 failed
     if (dev < 0 || dev >= 64) return false;
     std::lock_guard<std::mutex> g(mu);
     if (state[dev] == 0) {
-        const cudaError_t e = cudaFuncSetAttribute(k_ce_stream, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   int(sizeof(StreamSmem)));
+        const cudaError_t e = cudaFuncSetAttribute(k_ce_stream<WARPS, STAGES, CTAS>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   int(sizeof(StreamSmem<WARPS, STAGES>)));
         if (e != cudaSuccess) cudaGetLastError();
         state[dev] = e == cudaSuccess ? 1 : 2;
     }
     return state[dev] == 1;
 }
+
+// Launch the streaming kernel of the given shape: CTAS CTAs per SM.
+template <int WARPS, int STAGES, int CTAS>
+static dlm_status_t launch_stream(const CeParams& cp, int64_t R, int sms, int dev, cudaStream_t s, bool& done) {
+    done = false;
+    if (!stream_kernel_ready<WARPS, STAGES, CTAS>(dev)) return DLM_OK;
+    const int64_t grid = R < int64_t(sms) * CTAS ? R : int64_t(sms) * CTAS;
+    done = true;
+    return launch_pdl(k_ce_stream<WARPS, STAGES, CTAS>, dim3(unsigned(grid)), dim3(StreamShape<WARPS, STAGES>::kThreads),
+                      sizeof(StreamSmem<WARPS, STAGES>), s, "k_ce_stream launch", cp);
+}
+
+// Rows in flight x 2V bytes must stay within this much L2 between the passes.
+constexpr double kL2RowBudget = 80e6;
 
 static LayoutDev to_dev(const dlm_layout_t* L) {
     LayoutDev d{};
@@ -852,12 +867,14 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
         int dev = 0, sms = 148;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (fast && stream_kernel_ready(dev)) {
-            const int64_t grid = R < int64_t(sms) * kCtasPerSm ? R : int64_t(sms) * kCtasPerSm;
-            if ((st = launch_pdl(k_ce_stream, dim3(unsigned(grid)), dim3(kStreamThreads), sizeof(StreamSmem), s,
-                                 "k_ce_stream launch", cp)) != DLM_OK)
-                return st;
-        } else {
+        bool launched = false;
+        if (fast) {
+            const bool two_per_sm = double(sms) * 2.0 * 2.0 * double(vocab) <= kL2RowBudget;
+            st = two_per_sm ? launch_stream<8, 6, 2>(cp, R, sms, dev, s, launched)
+                            : launch_stream<16, 12, 1>(cp, R, sms, dev, s, launched);
+            if (st != DLM_OK) return st;
+        }
+        if (!launched) {
             const int64_t grid = R < int64_t(sms) * 8 ? R : int64_t(sms) * 8;
             if ((st = launch_pdl(k_ce_generic, dim3(unsigned(grid)), dim3(kGenThreads), 0, s,
                                  "k_ce_generic launch", cp)) != DLM_OK)
