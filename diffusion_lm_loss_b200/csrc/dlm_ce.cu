@@ -461,16 +461,24 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
                 m = cm;
             }
             if (m != -INFINITY) {
-                const float mb = m * kLog2e;
+                // exp(x - m) for both halves of each bf16 pair: one packed FMA,
+                // two ex2, one packed add into the (even, odd) partial sums
+                const uint64_t l2e = f2pack(kLog2e, kLog2e);
+                const uint64_t nmb = f2pack(-m * kLog2e, -m * kLog2e);
+                uint64_t acc = f2pack(0.f, 0.f);
                 #pragma unroll
                 for (int j = 0; j < kVecPerThread; ++j) {
                     const uint32_t wv[4] = {raw[j].x, raw[j].y, raw[j].z, raw[j].w};
                     #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        s += ex2(fmaf(bf16lo(wv[h]), kLog2e, -mb));
-                        s += ex2(fmaf(bf16hi(wv[h]), kLog2e, -mb));
+                        float t0, t1;
+                        f2unpack(f2fma(f2pack(bf16lo(wv[h]), bf16hi(wv[h])), l2e, nmb), t0, t1);
+                        acc = f2add(acc, f2pack(ex2(t0), ex2(t1)));
                     }
                 }
+                float a0, a1;
+                f2unpack(acc, a0, a1);
+                s += a0 + a1;
             }
         }
         // block combine among the consumer warps
@@ -492,6 +500,8 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
         const bool fold = coef > 0.f;
         const float lb = lse * kLog2e - (fold ? log2f(coef) : 0.f);
         const float mul = fold ? 1.f : coef;
+        const uint64_t l2e = f2pack(kLog2e, kLog2e);
+        const uint64_t nlb = f2pack(-lb, -lb);
 
         // pass 2: gradient
         for (int c = 0; c < nch; ++c, ++seq) {
@@ -509,8 +519,10 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
                     float g[8];
                     #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        g[2 * h] = ex2(fmaf(bf16lo(wv[h]), kLog2e, -lb));
-                        g[2 * h + 1] = ex2(fmaf(bf16hi(wv[h]), kLog2e, -lb));
+                        float t0, t1;
+                        f2unpack(f2fma(f2pack(bf16lo(wv[h]), bf16hi(wv[h])), l2e, nlb), t0, t1);
+                        g[2 * h] = ex2(t0);
+                        g[2 * h + 1] = ex2(t1);
                     }
                     if (!fold) {
                         #pragma unroll
