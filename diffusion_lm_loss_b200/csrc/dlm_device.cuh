@@ -282,6 +282,13 @@ __device__ __forceinline__ void bulk_wait_group_read() {
     asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(N) : "memory");
 }
 
+// Wait until at most N bulk groups of this thread are still in flight
+// (fully complete, global writes included).
+template <int N>
+__device__ __forceinline__ void bulk_wait_group() {
+    asm volatile("cp.async.bulk.wait_group %0;" :: "n"(N) : "memory");
+}
+
 // 16-byte global store with an L2 cache policy.
 __device__ __forceinline__ void st_global_v4_hint(void* p, uint4 v, uint64_t policy) {
     asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;"

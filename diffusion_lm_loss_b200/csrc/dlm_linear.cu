@@ -72,9 +72,13 @@ struct GemmArgs {
     uint16_t* dw;            // DW: [V, D] bf16
 };
 
+constexpr uint32_t kStageRowBytes = 128;                // one staged row: 64 bf16 or 32 f32
+constexpr uint32_t kStageBytes = 32 * kStageRowBytes;   // 32 rows (one epilogue warp)
+
 struct __align__(1024) GemmSmem {
     uint8_t a[kGemmStages][kStageA];
     uint8_t b[kGemmStages][kStageB];
+    uint8_t stage[4][2][kStageBytes];   // per epilogue warp, double-buffered TMA-store staging
     uint64_t full[kGemmStages];
     uint64_t empty[kGemmStages];
     uint64_t tfull[2];
@@ -86,9 +90,20 @@ struct __align__(1024) GemmSmem {
 
 __device__ __forceinline__ int round_up_dev(int x, int a) { return (x + a - 1) / a * a; }
 
+// Write one 128-byte row (8 x 16 B) of lane `row` into a 32-row staging tile
+// laid out for a 128-byte-swizzled TMA box: 16-byte unit j of row r sits at
+// unit (j ^ (r % 8)) -- which also keeps the 32 lanes' stores bank-conflict
+// free.  The tile must be 1024-byte aligned.
+__device__ __forceinline__ void stage_row(uint8_t* tile, int row, const uint4 (&v)[8]) {
+    uint4* r = reinterpret_cast<uint4*>(tile + row * kStageRowBytes);
+    #pragma unroll
+    for (int j = 0; j < 8; ++j) r[j ^ (row & 7)] = v[j];
+}
+
 template <int EPI, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs g) {
+k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+       const __grid_constant__ CUtensorMap tmC, const GemmArgs g) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
     GemmSmem& S = *reinterpret_cast<GemmSmem*>(smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr));
@@ -118,6 +133,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         fence_mbar_init_cluster();
         tc::prefetch_tensormap(&tmA);
         tc::prefetch_tensormap(&tmB);
+        if (EPI != EPI_LSE) tc::prefetch_tensormap(&tmC);
     }
     if (warp == 1) {
         tc::tmem_alloc(smem_addr(&S.tmem_base), 512);
@@ -210,6 +226,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         const int r_in_tile = quarter * 32 + lane;
         const bool kempty = nkb == 0;
         int lt = 0;
+        int sc = 0;   // staging boxes written by this warp (buffer parity)
         for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
             const int acc = lt & 1;
             const int m0 = (g.n_fastest ? tile / n_tiles : tile % m_tiles) * kBM;
@@ -259,98 +276,99 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                     g.part[size_t(m) * g.part_ld + nt] = make_float2(mx, sm);
                     if (have_xy) g.xy[m] = xyv;
                 }
-            } else if (EPI == EPI_DZ) {
+            } else {
+                // stores go out through TMA from a per-warp staging tile:
+                // 64 bf16 columns (dZ, dW) or 32 f32 columns (dH) per box
+                constexpr int kColsPerBox = EPI == EPI_DH ? 32 : 64;
+                constexpr int kBoxes = kBN / kColsPerBox;
                 const bool rv = m < M;
                 int tg = -1;
                 float coef = 0.f, lb = 0.f;
-                if (rv) {
+                if (EPI == EPI_DZ && rv) {
                     const int4 e = __ldg(&g.list[m]);
                     tg = e.y;
                     coef = g.grad_scale * __int_as_float(e.z);
                     lb = g.lse[m] * 1.4426950408889634f;
                 }
-                uint16_t* drow = g.dz + size_t(m) * g.dz_ld + n0;
-                for (int c = 0; c < kBN / 32; ++c) {
-                    uint32_t r[32];
-                    tc::tmem_ld_32x32b_x32(taddr + c * 32, r);
-                    tc::tmem_ld_wait();
-                    const int cb = g.col0 + n0 + c * 32;
-                    uint32_t pk[16];
-                    #pragma unroll
-                    for (int j = 0; j < 32; j += 2) {
-                        float v0 = 0.f, v1 = 0.f;
-                        if (rv && cb + j < g.vocab)
-                            v0 = coef * ex2(fmaf(__uint_as_float(r[j]), 1.4426950408889634f, -lb)) - (cb + j == tg ? coef : 0.f);
-                        if (rv && cb + j + 1 < g.vocab)
-                            v1 = coef * ex2(fmaf(__uint_as_float(r[j + 1]), 1.4426950408889634f, -lb)) - (cb + j + 1 == tg ? coef : 0.f);
-                        pk[j / 2] = pack_bf16x2(v0, v1);
-                    }
-                    uint4* dst = reinterpret_cast<uint4*>(drow + c * 32);
-                    #pragma unroll
-                    for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-                }
-                tc::fence_before_thread_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
-            } else if (EPI == EPI_DH) {
-                float* hrow = g.dh + size_t(m) * g.d_model + n0;
-                for (int c = 0; c < kBN / 32; ++c) {
-                    uint32_t r[32];
-                    if (!kempty) {
-                        tc::tmem_ld_32x32b_x32(taddr + c * 32, r);
-                        tc::tmem_ld_wait();
-                    } else {
-                        #pragma unroll
-                        for (int j = 0; j < 32; ++j) r[j] = 0u;
-                    }
-                    if (n0 + c * 32 < g.d_model) {
-                        float4* dst = reinterpret_cast<float4*>(hrow + c * 32);
-                        #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            float4 v = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
-                                                   __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
-                            if (g.accumulate) {
-                                const float4 o = dst[j];
-                                v.x += o.x; v.y += o.y; v.z += o.z; v.w += o.w;
-                            }
-                            dst[j] = v;
+                const int ew = warp - 2;                       // epilogue warp index 0..3
+                const int y0 = (EPI == EPI_DW ? g.col0 : 0) + m0 + quarter * 32;
+                for (int bx = 0; bx < kBoxes; ++bx) {
+                    uint4 v[8];
+                    if (EPI == EPI_DH) {
+                        uint32_t r[32];
+                        if (!kempty) {
+                            tc::tmem_ld_32x32b_x32(taddr + bx * 32, r);
+                            tc::tmem_ld_wait();
+                        } else {
+                            #pragma unroll
+                            for (int j = 0; j < 32; ++j) r[j] = 0u;
                         }
-                    }
-                }
-                if (!kempty) {
-                    tc::fence_before_thread_sync();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
-                }
-            } else {  // EPI_DW
-                const int vrow = g.col0 + m;
-                uint16_t* wrow = g.dw + size_t(vrow) * g.d_model + n0;
-                for (int c = 0; c < kBN / 32; ++c) {
-                    uint32_t r[32];
-                    if (!kempty) {
-                        tc::tmem_ld_32x32b_x32(taddr + c * 32, r);
-                        tc::tmem_ld_wait();
+                        #pragma unroll
+                        for (int j = 0; j < 8; ++j) v[j] = make_uint4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
                     } else {
+                        uint32_t pk[32];
                         #pragma unroll
-                        for (int j = 0; j < 32; ++j) r[j] = 0u;
+                        for (int half = 0; half < 2; ++half) {
+                            uint32_t r[32];
+                            if (!kempty) {
+                                tc::tmem_ld_32x32b_x32(taddr + bx * 64 + half * 32, r);
+                                tc::tmem_ld_wait();
+                            } else {
+                                #pragma unroll
+                                for (int j = 0; j < 32; ++j) r[j] = 0u;
+                            }
+                            if (EPI == EPI_DZ) {
+                                const int cb = g.col0 + n0 + bx * 64 + half * 32;
+                                #pragma unroll
+                                for (int j = 0; j < 32; j += 2) {
+                                    float v0 = 0.f, v1 = 0.f;
+                                    if (rv && cb + j < g.vocab)
+                                        v0 = coef * ex2(fmaf(__uint_as_float(r[j]), 1.4426950408889634f, -lb)) -
+                                             (cb + j == tg ? coef : 0.f);
+                                    if (rv && cb + j + 1 < g.vocab)
+                                        v1 = coef * ex2(fmaf(__uint_as_float(r[j + 1]), 1.4426950408889634f, -lb)) -
+                                             (cb + j + 1 == tg ? coef : 0.f);
+                                    pk[half * 16 + j / 2] = pack_bf16x2(v0, v1);
+                                }
+                            } else {
+                                #pragma unroll
+                                for (int j = 0; j < 16; ++j)
+                                    pk[half * 16 + j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                            }
+                        }
+                        #pragma unroll
+                        for (int j = 0; j < 8; ++j) v[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                     }
-                    if (vrow < g.vocab && n0 + c * 32 < g.d_model) {
-                        uint32_t pk[16];
-                        #pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            pk[j] = pack_bf16x2(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
-                        uint4* dst = reinterpret_cast<uint4*>(wrow + c * 32);
-                        #pragma unroll
-                        for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    if (bx == kBoxes - 1 && !kempty) {
+                        // all of this tile's accumulator is in registers: free it
+                        tc::fence_before_thread_sync();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
                     }
-                }
-                if (!kempty) {
-                    tc::fence_before_thread_sync();
+                    const int buf = sc & 1;
+                    if (lane == 0) bulk_wait_group_read<1>();   // the store from this buffer two boxes ago is done reading
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
+                    uint8_t* tile_s = S.stage[ew][buf];
+                    stage_row(tile_s, lane, v);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        // boxes that start outside the tensor are skipped (partial
+                        // boxes are clipped by the TMA unit); coordinates >= 0
+                        const int x = n0 + bx * kColsPerBox;
+                        const int xlim = EPI == EPI_DZ ? g.dz_ld : g.d_model;
+                        const int ylim = EPI == EPI_DW ? g.vocab : 0x7fffffff;
+                        if (x < xlim && y0 < ylim) {
+                            if (EPI == EPI_DH && g.accumulate) tc::tma_reduce_add_2d(&tmC, x, y0, smem_addr(tile_s));
+                            else                                tc::tma_store_2d(&tmC, x, y0, smem_addr(tile_s));
+                        }
+                        bulk_commit_group();
+                    }
+                    ++sc;
                 }
             }
         }
+        if (EPI != EPI_LSE && lane == 0) bulk_wait_group<0>();   // all stores complete before the CTA ends
     }
     __syncthreads();
     if (warp == 1) {
@@ -486,25 +504,28 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 2-D bf16 tensor [outer, inner] (row stride `stride_elems`), box
-// [box_outer, box_inner] with 128-byte swizzle (box_inner * 2 must be 128).
+// 2-D tensor [outer, inner] of bf16 (or f32), row stride `stride_elems`,
+// box [box_outer, box_inner] with 128-byte swizzle (box_inner * elem size must
+// be 128 bytes).
 static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t stride_elems,
-                     uint32_t box_inner, uint32_t box_outer) {
+                     uint32_t box_inner, uint32_t box_outer, bool f32 = false) {
     auto fn = encode_fn();
     if (!fn) return false;
+    const uint64_t esz = f32 ? 4 : 2;
     cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {stride_elems * 2};
+    cuuint64_t strides[1] = {stride_elems * esz};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 template <int EPI, bool A_MN, bool B_MN>
-static dlm_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const GemmArgs& g, int grid,
-                                cudaStream_t s) {
+static dlm_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
+                                const GemmArgs& g, int grid, cudaStream_t s) {
     auto kern = k_gemm<EPI, A_MN, B_MN>;
     const size_t smem = sizeof(GemmSmem) + 1024;
     static std::mutex mu;
@@ -519,7 +540,7 @@ static dlm_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, cons
             attr_done[dev] = true;
         }
     }
-    kern<<<grid, kGemmThreads, smem, s>>>(a, b, g);
+    kern<<<grid, kGemmThreads, smem, s>>>(a, b, c, g);
     return last_launch_status("k_gemm launch");
 }
 
@@ -586,13 +607,18 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, cons
     if ((st = last_launch_status("k_gather launch")) != DLM_OK) return st;
 
     // tensor maps (shapes are host-known upper bounds; the kernels read M)
-    CUtensorMap mHM_K, mW_K, mDZ_K, mW_MN, mDZ_MN, mHM_MN;
+    CUtensorMap mHM_K, mW_K, mDZ_K, mW_MN, mDZ_MN, mHM_MN, oDZ, oDH, oDW;
     bool ok = make_map(&mHM_K, HM, d_model, W.tpad, d_model, 64, kBM) &&
               make_map(&mW_K, weight, d_model, vocab, d_model, 64, kBN) &&
               make_map(&mDZ_K, dz, kVc, W.tpad, kVc, 64, kBM) &&
               make_map(&mW_MN, weight, d_model, vocab, d_model, 64, 64) &&
               make_map(&mDZ_MN, dz, kVc, W.tpad, kVc, 64, 64) &&
-              make_map(&mHM_MN, HM, d_model, W.tpad, d_model, 64, 64);
+              make_map(&mHM_MN, HM, d_model, W.tpad, d_model, 64, 64) &&
+              // epilogue outputs, 32-row boxes of 128 bytes
+              make_map(&oDZ, dz, kVc, W.tpad, kVc, 64, 32) &&
+              make_map(&oDH, dh, d_model, W.tpad, d_model, 32, 32, true) &&
+              (!d_weight || make_map(&oDW, d_weight, d_model, vocab, d_model, 64, 32));
+    if (!d_weight) oDW = oDZ;   // unused
     if (!ok) {
         record_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
         return DLM_ERR_CUDA;
@@ -611,7 +637,7 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, cons
         GemmArgs a = g;
         a.m_dev = 1; a.n_cols = vocab; a.k_dev = 0; a.k_len = d_model; a.b_off = 0; a.col0 = 0;
         a.part = part; a.part_ld = W.n_tiles; a.xy = xy;
-        if ((st = launch_gemm<EPI_LSE, false, false>(mHM_K, mW_K, a, sms, s)) != DLM_OK) return st;
+        if ((st = launch_gemm<EPI_LSE, false, false>(mHM_K, mW_K, mHM_K, a, sms, s)) != DLM_OK) return st;
     }
     k_lse<<<sms, 256, 0, s>>>(hdr, list, part, W.n_tiles, xy, lse, row_loss);
     if ((st = last_launch_status("k_lse launch")) != DLM_OK) return st;
@@ -622,18 +648,18 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, cons
         GemmArgs a = g;
         a.m_dev = 1; a.n_cols = int(align_up(vc, kBN)); a.k_dev = 0; a.k_len = d_model; a.b_off = c0; a.col0 = c0;
         a.lse = lse; a.dz = dz; a.dz_ld = kVc;
-        if ((st = launch_gemm<EPI_DZ, false, false>(mHM_K, mW_K, a, sms, s)) != DLM_OK) return st;
+        if ((st = launch_gemm<EPI_DZ, false, false>(mHM_K, mW_K, oDZ, a, sms, s)) != DLM_OK) return st;
 
         GemmArgs h = g;
         h.m_dev = 1; h.n_cols = d_model; h.k_dev = 0; h.k_len = int(align_up(vc, kBK)); h.b_off = c0;
         h.dh = dh; h.accumulate = c0 > 0; h.n_fastest = 1;
-        if ((st = launch_gemm<EPI_DH, false, true>(mDZ_K, mW_MN, h, sms, s)) != DLM_OK) return st;
+        if ((st = launch_gemm<EPI_DH, false, true>(mDZ_K, mW_MN, oDH, h, sms, s)) != DLM_OK) return st;
 
         if (d_weight) {
             GemmArgs w = g;
             w.m_dev = 0; w.m_rows = int(align_up(vc, kBM)); w.n_cols = d_model; w.k_dev = 1; w.b_off = 0;
             w.col0 = c0; w.dw = d_weight; w.n_fastest = 1;
-            if ((st = launch_gemm<EPI_DW, true, true>(mDZ_MN, mHM_MN, w, sms, s)) != DLM_OK) return st;
+            if ((st = launch_gemm<EPI_DW, true, true>(mDZ_MN, mHM_MN, oDW, w, sms, s)) != DLM_OK) return st;
         }
     }
 

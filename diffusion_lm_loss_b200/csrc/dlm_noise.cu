@@ -18,6 +18,8 @@ namespace dlm {
 __global__ void k_sample_t(uint64_t seed, int n_units, int mode, float eps,
                            float* __restrict__ t, float* __restrict__ p) {
     const int u = blockIdx.x * blockDim.x + threadIdx.x;
+    pdl_wait();   // earlier kernels may still read t / p
+    pdl_launch_dependents();
     if (u >= n_units) return;
     const uint32_t k = uint32_t(splitmix64_at(seed, rng_counter(0, uint32_t(u), 0)) >> 40);
     const float x = float(k) * (1.0f / 16777216.0f);            // exact
@@ -37,6 +39,8 @@ __global__ void k_corrupt(int n_units, int seq_len, const int32_t* __restrict__ 
                           int32_t* __restrict__ noisy, uint8_t* __restrict__ corrupted,
                           uint32_t* __restrict__ status) {
     const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+    pdl_wait();   // p comes from the previous kernel; outputs may still be read by earlier ones
+    pdl_launch_dependents();
     if (cu && i <= n_units && status) {
         const int32_t c = cu[i];
         bool bad = (i == 0 && c != 0) || (i == n_units && int64_t(c) != n_tokens);
@@ -82,9 +86,8 @@ extern "C" dlm_status_t dlm_sample_t(uint64_t seed, int32_t n_units, int32_t mod
     dlm_status_t s = check_device();
     if (s != DLM_OK) return s;
     const int threads = 128;
-    k_sample_t<<<(n_units + threads - 1) / threads, threads, 0, (cudaStream_t)stream>>>(
-        seed, n_units, mode, eps, t, p);
-    return last_launch_status();
+    return launch_pdl(k_sample_t, dim3((n_units + threads - 1) / threads), dim3(threads), 0,
+                      (cudaStream_t)stream, "k_sample_t launch", seed, n_units, mode, eps, t, p);
 }
 
 extern "C" dlm_status_t dlm_corrupt(const dlm_layout_t* layout, const int32_t* clean_ids,
@@ -103,8 +106,8 @@ extern "C" dlm_status_t dlm_corrupt(const dlm_layout_t* layout, const int32_t* c
     const int threads = 256;
     const int64_t work = n > layout->n_units + 1 ? n : int64_t(layout->n_units) + 1;
     const int64_t blocks = (work + threads - 1) / threads;
-    k_corrupt<<<unsigned(blocks), threads, 0, (cudaStream_t)stream>>>(
-        layout->n_units, layout->seq_len, layout->cu_seqlens, layout->pad_mask, n, clean_ids, p,
-        mode, mask_id, uint32_t(vocab), seed, noisy_ids, corrupted, dev_status);
-    return last_launch_status();
+    return launch_pdl(k_corrupt, dim3(unsigned(blocks)), dim3(threads), 0, (cudaStream_t)stream,
+                      "k_corrupt launch", layout->n_units, layout->seq_len, layout->cu_seqlens,
+                      layout->pad_mask, n, clean_ids, p, mode, mask_id, uint32_t(vocab), seed, noisy_ids,
+                      corrupted, dev_status);
 }
