@@ -40,7 +40,7 @@ STATUS = {0: "DLM_OK", 1: "DLM_ERR_INVALID_ARGUMENT", 2: "DLM_ERR_UNSUPPORTED",
 EXPORTS = ("dlm_status_string", "dlm_last_cuda_error", "dlm_version", "dlm_sample_t", "dlm_corrupt",
            "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_loss_fwd_bwd_static",
            "dlm_linear_loss_workspace_size",
-           "dlm_linear_loss_fwd_bwd", "dlm_get_device_status")
+           "dlm_linear_loss_fwd_bwd", "dlm_get_device_status", "dlm_selftest_bounded_wait")
 
 
 class DlmError(RuntimeError):
@@ -113,6 +113,8 @@ def lib():
     L.dlm_linear_loss_fwd_bwd.restype = ctypes.c_int
     L.dlm_linear_loss_fwd_bwd.argtypes = [lp, vp, vp, i32, i32, vp, vp, vp, f32, vp, vp, vp, vp,
                                           vp, sz, vp]
+    L.dlm_selftest_bounded_wait.restype = ctypes.c_int
+    L.dlm_selftest_bounded_wait.argtypes = [u64, vp, vp]
     L.dlm_get_device_status.restype = ctypes.c_int
     L.dlm_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), vp]
     _lib = L

@@ -2,6 +2,7 @@
 // device-status read-back of the C ABI.
 #include <mutex>
 
+#include "dlm_device.cuh"
 #include "dlm_host.h"
 
 #include <cstdio>
@@ -36,7 +37,27 @@ dlm_status_t check_device() {
     return known[dev] == 1 ? DLM_OK : DLM_ERR_UNSUPPORTED;
 }
 
+// One thread waits on an mbarrier phase that nothing completes; the bounded
+// wait gives up after `limit_ns`, records DLM_DEV_WAIT_TIMEOUT and the kernel
+// returns normally.
+__global__ void k_selftest_wait(uint64_t limit_ns, uint32_t* status) {
+    __shared__ uint64_t bar;
+    const uint32_t a = smem_addr(&bar);
+    mbar_init(a, 1);                      // expects one arrival that never comes
+    fence_mbar_init_cluster();
+    mbar_wait_limit(a, 0, limit_ns, status);
+}
+
 }  // namespace dlm
+
+extern "C" dlm_status_t dlm_selftest_bounded_wait(uint64_t limit_ns, uint32_t* dev_status,
+                                                  dlm_stream_t stream) {
+    if (!dev_status || limit_ns == 0 || limit_ns > 10000000000ull) return DLM_ERR_INVALID_ARGUMENT;
+    dlm_status_t st = dlm::check_device();
+    if (st != DLM_OK) return st;
+    dlm::k_selftest_wait<<<1, 1, 0, (cudaStream_t)stream>>>(limit_ns, dev_status);
+    return dlm::last_launch_status("k_selftest_wait launch");
+}
 
 extern "C" const char* dlm_status_string(dlm_status_t status) {
     switch (status) {

@@ -178,6 +178,20 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     }
 }
 
+// The same bounded wait with a caller-given limit in nanoseconds.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, uint64_t limit_ns, uint32_t* status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    #pragma unroll 1
+    while (true) {
+        if (mbar_try_wait_sleep(bar, parity, kSleepHintNs)) return true;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            if (status) atomicOr(status, DLM_DEV_WAIT_TIMEOUT);
+            return false;
+        }
+    }
+}
+
 // Bulk copy global -> this CTA's shared memory, completion on `bar`
 // (tx bytes).  dst, src 16-byte aligned; bytes a multiple of 16.  No
 // multicast.

@@ -262,6 +262,21 @@ DLM_API dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t *layout, const u
 DLM_API dlm_status_t dlm_get_device_status(const void *workspace, uint32_t *host_status,
                                    dlm_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * dlm_selftest_bounded_wait -- exercise the library's failure detection on
+ * the device.  Every on-chip wait of the kernels above (mbarrier phases of
+ * the TMA / tensor-core pipelines) gives up after a time limit, records
+ * DLM_DEV_WAIT_TIMEOUT in the status word and lets the kernel end, so a
+ * broken pipeline cannot hang the GPU.  This call launches one thread that
+ * waits, through the same bounded wait, on a barrier phase that nothing ever
+ * completes, with a limit of `limit_ns` nanoseconds (1 .. 1e10): on return of
+ * the kernel *dev_status (device uint32) has DLM_DEV_WAIT_TIMEOUT or'ed in and
+ * the CUDA context is still usable.  (The pages describe failure handling
+ * only at the level of the training loop; this is the library's own check.)
+ * ---------------------------------------------------------------------- */
+DLM_API dlm_status_t dlm_selftest_bounded_wait(uint64_t limit_ns, uint32_t *dev_status,
+                                               dlm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

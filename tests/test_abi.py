@@ -74,6 +74,10 @@ def test_host_side_rejections(L):
     assert L.dlm_loss_fwd_bwd(*a) == 3                                    # workspace too small
     a = list(args); a[19] = 100
     assert L.dlm_loss_fwd_bwd(*a) == 1                                    # misaligned workspace
+    # bounded-wait self-test: no status word, zero or over-long limit
+    assert L.dlm_selftest_bounded_wait(10, None, None) == 1
+    assert L.dlm_selftest_bounded_wait(0, 16, None) == 1
+    assert L.dlm_selftest_bounded_wait(20_000_000_000, 16, None) == 1
 
 
 def test_workspace_size_grows_with_rows(L):

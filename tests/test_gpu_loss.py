@@ -1,7 +1,7 @@
 """GPU parity of the weighted CE forward + backward against the CPU oracle.
 
-Element-by-element at sizes the oracle finishes in seconds (several cluster
-slices, ragged tails, packed documents, pads, empty documents); at the full
+Element-by-element at sizes the oracle finishes in seconds (more rows than
+CTAs, ragged vocabularies, packed documents, pads, empty documents); at the full
 workload sizes, in the launch configuration the benchmark times: the total
 loss and every per-unit sum over all rows, and the gradient on sampled rows.
 """
@@ -93,7 +93,7 @@ def test_tiny_absorbing_full():
 
 
 def test_llada_like_mid_size_elementwise():
-    """L=256 rows of V=126464: four cluster slices, every element checked."""
+    """L=256 rows of V=126464 (more rows than CTAs in flight at once), every element checked."""
     spec = di.WORKLOADS["abs_b1_l4096_v126464"].scaled(seq_len=256)
     case = di.make_case(spec, "cuda")
     run_absorbing(spec, case.logits, case.clean, n_units=1, seq_len=256, seed=0)
