@@ -332,6 +332,40 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t parity
     }
 }
 
+// Arrive on an mbarrier of another CTA of the cluster (shared::cluster
+// address from mapa_shared), releasing this thread's prior writes at cluster
+// scope.
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t bar_cluster) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar_cluster) : "memory");
+}
+
+// mbar_wait_or_abort for a barrier that threads of other CTAs of the cluster
+// arrive on: the wait acquires at cluster scope.
+__device__ __forceinline__ bool mbar_try_wait_cluster_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar), "r"(parity), "r"(ns) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_or_abort_cluster(uint32_t bar, uint32_t parity, uint32_t* status,
+                                                           volatile int* abort) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    #pragma unroll 1
+    while (true) {
+        if (mbar_try_wait_cluster_sleep(bar, parity, kSleepHintNs)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (status) atomicOr(status, DLM_DEV_WAIT_TIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
 __device__ __forceinline__ void cluster_sync_all() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
                  "barrier.cluster.wait.acquire.aligned;" ::: "memory");

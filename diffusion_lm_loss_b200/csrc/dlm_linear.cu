@@ -37,12 +37,23 @@
 
 namespace dlm {
 
-constexpr int kBM = 128, kBN = 256, kBK = 64;
-constexpr int kGemmStages = 4;
+constexpr int kBM = 128, kBN = 256, kBK = 64;   // per-CTA accumulator tile 128 x 256, K step 64
 constexpr int kGemmThreads = 192;
-constexpr uint32_t kStageA = kBM * kBK * 2;   // 16 KB
-constexpr uint32_t kStageB = kBN * kBK * 2;   // 32 KB
+constexpr uint32_t kStageA = kBM * kBK * 2;   // 16 KB: this CTA's 128 A rows x 64
 constexpr int kVc = 16384;                    // vocabulary chunk of the backward pass
+constexpr int kRowPad = 256;                  // masked-row buffers are padded to the paired tile height
+
+// PAIR = 2: a CTA pair (cluster of 2) computes a 256 x 256 tile with
+// cta_group::2 MMAs -- each CTA loads its own 128 A rows and half of the 256
+// B rows, so a CTA streams 32 KB per K step instead of 48 KB and the ring
+// holds 6 stages.  PAIR = 1: one CTA per 128 x 256 tile, 4 stages.
+template <int PAIR>
+struct GemmCfg {
+    static constexpr int kStages = PAIR == 2 ? 6 : 4;
+    static constexpr int kBRows = kBN / PAIR;                  // B rows (N) loaded by one CTA
+    static constexpr uint32_t kStageB = kBRows * kBK * 2;      // 16 or 32 KB
+    static constexpr int kTileM = kBM * PAIR;                  // C rows per tile
+};
 
 enum Epi { EPI_LSE = 0, EPI_DZ = 1, EPI_DH = 2, EPI_DW = 3 };
 
@@ -75,12 +86,13 @@ struct GemmArgs {
 constexpr uint32_t kStageRowBytes = 128;                // one staged row: 64 bf16 or 32 f32
 constexpr uint32_t kStageBytes = 32 * kStageRowBytes;   // 32 rows (one epilogue warp)
 
+template <int PAIR>
 struct __align__(1024) GemmSmem {
-    uint8_t a[kGemmStages][kStageA];
-    uint8_t b[kGemmStages][kStageB];
+    uint8_t a[GemmCfg<PAIR>::kStages][kStageA];
+    uint8_t b[GemmCfg<PAIR>::kStages][GemmCfg<PAIR>::kStageB];
     uint8_t stage[4][2][kStageBytes];   // per epilogue warp, double-buffered TMA-store staging
-    uint64_t full[kGemmStages];
-    uint64_t empty[kGemmStages];
+    uint64_t full[GemmCfg<PAIR>::kStages];
+    uint64_t empty[GemmCfg<PAIR>::kStages];
     uint64_t tfull[2];
     uint64_t tempty[2];
     uint64_t drain;
@@ -100,33 +112,41 @@ __device__ __forceinline__ void stage_row(uint8_t* tile, int row, const uint4 (&
     for (int j = 0; j < 8; ++j) r[j ^ (row & 7)] = v[j];
 }
 
-template <int EPI, bool A_MN, bool B_MN>
+template <int EPI, bool A_MN, bool B_MN, int PAIR>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
        const __grid_constant__ CUtensorMap tmC, const GemmArgs g) {
+    using Cfg = GemmCfg<PAIR>;
+    constexpr int kStages = Cfg::kStages;
+    constexpr uint32_t kStageB = Cfg::kStageB;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_addr(smem_raw);
-    GemmSmem& S = *reinterpret_cast<GemmSmem*>(smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr));
+    GemmSmem<PAIR>& S = *reinterpret_cast<GemmSmem<PAIR>*>(smem_raw + (((raw_addr + 1023u) & ~1023u) - raw_addr));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int* abort = &S.abort;
+    // the pair: rank 0 issues the MMAs for both CTAs; tiles go to clusters
+    const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit = PAIR == 2 ? int(cluster_id_x()) : int(blockIdx.x);
+    const int n_units = PAIR == 2 ? int(nclusters_x()) : int(gridDim.x);
 
     const int M = g.hdr->n_scored;
     const int Mp = round_up_dev(M, kBM);
     const int rows = g.m_dev ? Mp : g.m_rows;
     const int K = g.k_dev ? Mp : g.k_len;
-    const int m_tiles = rows / kBM;
+    const int m_tiles = (rows + Cfg::kTileM - 1) / Cfg::kTileM;
     const int n_tiles = (g.n_cols + kBN - 1) / kBN;
     const int tiles = m_tiles * n_tiles;
     const int nkb = K / kBK;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kGemmStages; ++i) {
+        for (int i = 0; i < kStages; ++i) {
             mbar_init(smem_addr(&S.full[i]), 1);
             mbar_init(smem_addr(&S.empty[i]), 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(smem_addr(&S.tfull[i]), 1);
-            mbar_init(smem_addr(&S.tempty[i]), 4);
+            mbar_init(smem_addr(&S.tempty[i]), 4 * PAIR);   // every epilogue warp of the pair
         }
         mbar_init(smem_addr(&S.drain), 1);
         S.abort = 0;
@@ -136,69 +156,92 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         if (EPI != EPI_LSE) tc::prefetch_tensormap(&tmC);
     }
     if (warp == 1) {
-        tc::tmem_alloc(smem_addr(&S.tmem_base), 512);
-        tc::tmem_relinquish();
+        if (PAIR == 2) { tc::tmem_alloc_pair(smem_addr(&S.tmem_base), 512); tc::tmem_relinquish_pair(); }
+        else           { tc::tmem_alloc(smem_addr(&S.tmem_base), 512);      tc::tmem_relinquish(); }
     }
     tc::fence_before_thread_sync();
     __syncthreads();
+    if (PAIR == 2) cluster_sync_all();   // the peer's barriers exist before anyone signals them
     tc::fence_after_thread_sync();
     const uint32_t tmem = S.tmem_base;
 
+    // tile -> (first C row of this CTA, first C column)
+    auto tile_coords = [&](int tile, int& m0, int& nt) {
+        const int mt = g.n_fastest ? tile / n_tiles : tile % m_tiles;
+        nt = g.n_fastest ? tile % n_tiles : tile / m_tiles;
+        m0 = mt * Cfg::kTileM + int(rank) * kBM;
+    };
+
     if (warp == 0 && lane == 0) {
         // ------------------------------ TMA producer ------------------------------
+        // Each CTA loads its own A rows and its share of the B rows; the bytes
+        // of both CTAs complete on the leader's full barrier.
         uint64_t pol_a, pol_b;
         if (EPI == EPI_LSE || EPI == EPI_DZ) { pol_a = policy_evict_last(); pol_b = policy_evict_first(); }
         else                                 { pol_a = policy_evict_normal(); pol_b = policy_evict_normal(); }
         int it = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-            const int m0 = (g.n_fastest ? tile / n_tiles : tile % m_tiles) * kBM;
-            const int n0 = (g.n_fastest ? tile % n_tiles : tile / m_tiles) * kBN;
+        for (int tile = unit; tile < tiles && ok; tile += n_units) {
+            int m0, nt;
+            tile_coords(tile, m0, nt);
+            const int nb = nt * kBN + int(rank) * Cfg::kBRows;   // this CTA's first B row (N)
             for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const int s = it % kGemmStages;
-                if (!mbar_wait_or_abort(smem_addr(&S.empty[s]), ((it / kGemmStages) & 1) ^ 1, g.status, abort)) {
+                const int s = it % kStages;
+                if (!mbar_wait_or_abort(smem_addr(&S.empty[s]), ((it / kStages) & 1) ^ 1, g.status, abort)) {
                     ok = false;
                     break;
                 }
                 const uint32_t fb = smem_addr(&S.full[s]);
-                mbar_arrive_expect_tx(fb, kStageA + kStageB);
+                const uint32_t fb_lead = PAIR == 2 ? mapa_shared(fb, 0) : fb;
+                if (leader) mbar_arrive_expect_tx(fb, PAIR * (kStageA + kStageB));
                 const int k0 = kb * kBK;
                 const uint32_t a_s = smem_addr(S.a[s]), b_s = smem_addr(S.b[s]);
+                auto load = [&](uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t pol) {
+                    if (PAIR == 2) tc::tma_load_2d_pair(dst, map, x, y, fb_lead, pol);
+                    else           tc::tma_load_2d(dst, map, x, y, fb, pol);
+                };
                 if (!A_MN) {
-                    tc::tma_load_2d(a_s, &tmA, k0, m0, fb, pol_a);
+                    load(a_s, &tmA, k0, m0, pol_a);
                 } else {
-                    tc::tma_load_2d(a_s, &tmA, m0, k0, fb, pol_a);
-                    tc::tma_load_2d(a_s + 8192, &tmA, m0 + 64, k0, fb, pol_a);
+                    load(a_s, &tmA, m0, k0, pol_a);
+                    load(a_s + 8192, &tmA, m0 + 64, k0, pol_a);
                 }
                 if (!B_MN) {
-                    tc::tma_load_2d(b_s, &tmB, k0, n0 + g.b_off, fb, pol_b);
+                    load(b_s, &tmB, k0, nb + g.b_off, pol_b);
                 } else {
                     #pragma unroll
-                    for (int j = 0; j < 4; ++j) tc::tma_load_2d(b_s + 8192 * j, &tmB, n0 + 64 * j, k0 + g.b_off, fb, pol_b);
+                    for (int j = 0; j < Cfg::kBRows / 64; ++j)
+                        load(b_s + 8192 * j, &tmB, nb + 64 * j, k0 + g.b_off, pol_b);
                 }
             }
         }
-        if (!ok) {
-            // let the copies already issued land before the CTA can exit
-            for (int j = it - 1; j >= 0 && j >= it - kGemmStages; --j)
-                mbar_wait_bounded<false>(smem_addr(&S.full[j % kGemmStages]), (j / kGemmStages) & 1, nullptr);
+        if (!ok && (PAIR == 1 || leader)) {
+            // let the copies already issued land before the CTA can exit (a
+            // pair's second CTA cannot observe its own copies -- they complete
+            // on the leader's barrier -- but it only gets here after a wait of
+            // seconds, long after any copy it issued has landed)
+            for (int j = it - 1; j >= 0 && j >= it - kStages; --j)
+                mbar_wait_bounded<false>(smem_addr(&S.full[j % kStages]), (j / kStages) & 1, nullptr);
         }
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1 && lane == 0 && leader) {
         // ------------------------------ MMA issuer ------------------------------
-        constexpr uint32_t idesc = tc::idesc_bf16(kBM, kBN, A_MN ? 1 : 0, B_MN ? 1 : 0);
+        constexpr uint32_t idesc = tc::idesc_bf16(Cfg::kTileM, kBN, A_MN ? 1 : 0, B_MN ? 1 : 0);
         int it = 0, lt = 0;
         bool ok = nkb > 0;
-        for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++lt) {
+        for (int tile = unit; tile < tiles && ok; tile += n_units, ++lt) {
             const int acc = lt & 1;
-            if (!mbar_wait_or_abort(smem_addr(&S.tempty[acc]), ((lt >> 1) & 1) ^ 1, g.status, abort)) {
+            const bool free_acc = PAIR == 2
+                ? mbar_wait_or_abort_cluster(smem_addr(&S.tempty[acc]), ((lt >> 1) & 1) ^ 1, g.status, abort)
+                : mbar_wait_or_abort(smem_addr(&S.tempty[acc]), ((lt >> 1) & 1) ^ 1, g.status, abort);
+            if (!free_acc) {
                 ok = false;
                 break;
             }
             tc::fence_after_thread_sync();
             const uint32_t d_tmem = tmem + uint32_t(acc * kBN);
             for (int kb = 0; kb < nkb; ++kb, ++it) {
-                const int s = it % kGemmStages;
-                if (!mbar_wait_or_abort(smem_addr(&S.full[s]), (it / kGemmStages) & 1, g.status, abort)) {
+                const int s = it % kStages;
+                if (!mbar_wait_or_abort(smem_addr(&S.full[s]), (it / kStages) & 1, g.status, abort)) {
                     ok = false;
                     break;
                 }
@@ -210,15 +253,25 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                                              : tc::smem_desc_sw128(a_s + kk * 32, 16, 1024);
                     const uint64_t bd = B_MN ? tc::smem_desc_sw128(b_s + kk * 2048, 8192, 1024)
                                              : tc::smem_desc_sw128(b_s + kk * 32, 16, 1024);
-                    tc::mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    if (PAIR == 2) tc::mma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    else           tc::mma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
                 }
-                tc::mma_commit(smem_addr(&S.empty[s]));   // stage reusable once these MMAs retire
+                // the stage is reusable (in both CTAs) once these MMAs retire
+                if (PAIR == 2) tc::mma_commit_pair(smem_addr(&S.empty[s]), 0x3);
+                else           tc::mma_commit(smem_addr(&S.empty[s]));
             }
             if (!ok) break;
-            tc::mma_commit(smem_addr(&S.tfull[acc]));     // accumulator ready for the epilogue
+            // accumulator ready for the epilogue (of both CTAs)
+            if (PAIR == 2) tc::mma_commit_pair(smem_addr(&S.tfull[acc]), 0x3);
+            else           tc::mma_commit(smem_addr(&S.tfull[acc]));
         }
         // no MMA may still be running when tensor memory is released
-        tc::mma_commit(smem_addr(&S.drain));
+        if (PAIR == 2) tc::mma_commit_pair(smem_addr(&S.drain), 0x3);
+        else           tc::mma_commit(smem_addr(&S.drain));
+        mbar_wait_bounded<false>(smem_addr(&S.drain), 0, nullptr);
+    } else if (warp == 1 && lane == 0) {
+        // the pair's second CTA: its tensor memory is written by the leader's
+        // MMAs; wait for the leader's final completion signal before release
         mbar_wait_bounded<false>(smem_addr(&S.drain), 0, nullptr);
     } else if (warp >= 2) {
         // ------------------------------ epilogue ------------------------------
@@ -227,10 +280,19 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         const bool kempty = nkb == 0;
         int lt = 0;
         int sc = 0;   // staging boxes written by this warp (buffer parity)
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
+        // accumulator release: the leader's barrier counts the epilogue warps of both CTAs
+        auto release_acc = [&](int acc) {
+            tc::fence_before_thread_sync();
+            __syncwarp();
+            if (lane == 0) {
+                if (PAIR == 2) mbar_arrive_remote(mapa_shared(smem_addr(&S.tempty[acc]), 0));
+                else           mbar_arrive(smem_addr(&S.tempty[acc]));
+            }
+        };
+        for (int tile = unit; tile < tiles; tile += n_units, ++lt) {
             const int acc = lt & 1;
-            const int m0 = (g.n_fastest ? tile / n_tiles : tile % m_tiles) * kBM;
-            const int nt = g.n_fastest ? tile % n_tiles : tile / m_tiles;
+            int m0, nt;
+            tile_coords(tile, m0, nt);
             const int n0 = nt * kBN;
             const int m = m0 + r_in_tile;
             if (!kempty) {
@@ -269,9 +331,7 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                             if (cb + j < g.vocab) sm += ex2(fmaf(__uint_as_float(r[j]), 1.4426950408889634f, -mb));
                     }
                 }
-                tc::fence_before_thread_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
+                release_acc(acc);
                 if (rv) {
                     g.part[size_t(m) * g.part_ld + nt] = make_float2(mx, sm);
                     if (have_xy) g.xy[m] = xyv;
@@ -339,12 +399,8 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
                         #pragma unroll
                         for (int j = 0; j < 8; ++j) v[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                     }
-                    if (bx == kBoxes - 1 && !kempty) {
-                        // all of this tile's accumulator is in registers: free it
-                        tc::fence_before_thread_sync();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(smem_addr(&S.tempty[acc]));
-                    }
+                    // all of this tile's accumulator is in registers: free it
+                    if (bx == kBoxes - 1 && !kempty) release_acc(acc);
                     const int buf = sc & 1;
                     if (lane == 0) bulk_wait_group_read<1>();   // the store from this buffer two boxes ago is done reading
                     __syncwarp();
@@ -371,20 +427,26 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
         if (EPI != EPI_LSE && lane == 0) bulk_wait_group<0>();   // all stores complete before the CTA ends
     }
     __syncthreads();
+    __syncwarp();
+    // neither CTA of a pair leaves (or frees tensor memory) while the other
+    // may still signal its barriers
+    if (PAIR == 2) cluster_sync_all();
     if (warp == 1) {
         tc::fence_after_thread_sync();
-        tc::tmem_dealloc(tmem, 512);
+        if (PAIR == 2) tc::tmem_dealloc_pair(tmem, 512);
+        else           tc::tmem_dealloc(tmem, 512);
     }
 }
 
 // ---------------------------------------------------------------------------
 // small kernels around the GEMMs
 // ---------------------------------------------------------------------------
-// H_M[m] = H[list[m].row] for m < M, zero rows up to round_up(M, 128).
+// H_M[m] = H[list[m].row] for m < M, zero rows up to round_up(M, 256) (the
+// height of a paired tile).
 __global__ void k_gather(const WsHeader* hdr, const int4* list, const uint16_t* __restrict__ H, int D,
                          uint16_t* __restrict__ HM) {
     const int M = hdr->n_scored;
-    const int Mp = round_up_dev(M, kBM);
+    const int Mp = round_up_dev(M, kRowPad);
     const int vecs = D / 8;
     for (int r = blockIdx.x; r < Mp; r += gridDim.x) {
         uint4* dst = reinterpret_cast<uint4*>(HM + size_t(r) * D);
@@ -472,7 +534,7 @@ struct LinWs {
 
 static LinWs lin_ws(int64_t T, int64_t units, int D, int V) {
     LinWs w;
-    w.tpad = int(align_up(size_t(T > 0 ? T : 1), kBM));
+    w.tpad = int(align_up(size_t(T > 0 ? T : 1), kRowPad));
     w.n_tiles = (V + kBN - 1) / kBN;
     size_t o = kWsAlign;
     w.list = o;     o = align_up(o + size_t(T) * 16, kWsAlign);
@@ -523,11 +585,20 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
     return r == CUDA_SUCCESS;
 }
 
+#ifndef DLM_GEMM_PAIR
+#define DLM_GEMM_PAIR 2
+#endif
+constexpr int kPair = DLM_GEMM_PAIR;   // CTAs per MMA tile (2: cta_group::2 pairs)
+static_assert(kPair == 1 || kPair == 2, "CTAs per tile");
+
+// One persistent CTA per SM (clusters of kPair CTAs; the grid is a multiple
+// of kPair).
 template <int EPI, bool A_MN, bool B_MN>
 static dlm_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& c,
                                 const GemmArgs& g, int grid, cudaStream_t s) {
-    auto kern = k_gemm<EPI, A_MN, B_MN>;
-    const size_t smem = sizeof(GemmSmem) + 1024;
+    auto kern = k_gemm<EPI, A_MN, B_MN, kPair>;
+    const size_t smem = sizeof(GemmSmem<kPair>) + 1024;
+    static_assert(sizeof(GemmSmem<kPair>) + 1024 <= 227 * 1024, "shared memory per CTA");
     static std::mutex mu;
     static bool attr_done[64] = {};
     int dev = 0;
@@ -540,8 +611,22 @@ static dlm_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, cons
             attr_done[dev] = true;
         }
     }
-    kern<<<grid, kGemmThreads, smem, s>>>(a, b, c, g);
-    return last_launch_status("k_gemm launch");
+    grid -= grid % kPair;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kPair;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, b, c, g);
+    if (e != cudaSuccess) return cuda_status(e, "k_gemm launch");
+    return DLM_OK;
 }
 
 }  // namespace dlm
@@ -609,7 +694,7 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, cons
     // tensor maps (shapes are host-known upper bounds; the kernels read M)
     CUtensorMap mHM_K, mW_K, mDZ_K, mW_MN, mDZ_MN, mHM_MN, oDZ, oDH, oDW;
     bool ok = make_map(&mHM_K, HM, d_model, W.tpad, d_model, 64, kBM) &&
-              make_map(&mW_K, weight, d_model, vocab, d_model, 64, kBN) &&
+              make_map(&mW_K, weight, d_model, vocab, d_model, 64, kBN / kPair) &&
               make_map(&mDZ_K, dz, kVc, W.tpad, kVc, 64, kBM) &&
               make_map(&mW_MN, weight, d_model, vocab, d_model, 64, 64) &&
               make_map(&mDZ_MN, dz, kVc, W.tpad, kVc, 64, 64) &&
