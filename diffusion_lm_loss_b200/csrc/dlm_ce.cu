@@ -84,7 +84,7 @@ __device__ __forceinline__ void unit_pos(const LayoutDev& L, int64_t i, int& u, 
         u = find_unit(L.cu, L.n_units, i);
         end = L.cu[u + 1];
     } else {
-        u = int(i / L.seq_len);
+        u = int(i) / L.seq_len;   // token indices are < 2^31
         end = int64_t(u + 1) * L.seq_len;
     }
 }
@@ -134,34 +134,29 @@ __device__ __forceinline__ bool layout_bad(const LayoutDev& L) {
 
 constexpr int kPlanCacheRows = 16384;   // rows whose classification is kept in shared memory
 
-// Exclusive block scan of one int per thread (kPlanThreads threads): warp
-// shuffles, then one pass over the warp totals.  Also returns the block total.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
+// Exclusive prefix over the warps of the CTA of one count per warp, and the
+// CTA total, from s_cnt[warp]; every lane of every warp gets the values for
+// its own warp.
+__device__ __forceinline__ void warp_prefix(const int* s_cnt, int warp, int lane, int& before, int& total) {
+    const int c = lane < kPlanWarps ? s_cnt[lane] : 0;
+    int x = c;
     #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < kPlanWarps ? s_warp[lane] : 0;
-        #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += y;
-        }
-        if (lane < kPlanWarps) s_warp[lane] = w;   // inclusive over warps
-    }
-    __syncthreads();
-    total = s_warp[kPlanWarps - 1];
-    return (warp ? s_warp[warp - 1] : 0) + x - v;
+    before = __shfl_sync(0xffffffffu, x - c, warp);
+    total = __shfl_sync(0xffffffffu, x, 31);
 }
 
+// One CTA.  Thread t takes rows t, t + T, t + 2T, ... (T = kPlanThreads), so
+// a warp always works on 32 consecutive rows: its loads are coalesced, and in
+// pass 2 its scored rows (and its other rows) land in consecutive list slots,
+// found from a warp ballot plus a prefix over the warps -- 16-byte list
+// stores that coalesce.  The list holds the scored rows in row order, then
+// all other rows in row order.
 __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
-    __shared__ int s_warp[32];
+    __shared__ int s_cnt[2][kPlanWarps];
     __shared__ int s_sum[3][kPlanWarps];
     __shared__ uint32_t s_status;
     pdl_launch_dependents();   // the CE kernel may start its prologue now
@@ -172,27 +167,22 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
     if (layout_bad(P.a) || layout_bad(P.b)) atomicOr(&s_status, DLM_DEV_BAD_LAYOUT);
 
     const int64_t R = P.a.n_tokens + P.b.n_tokens;
-    const int64_t chunk = (R + kPlanThreads - 1) / kPlanThreads;
-    const int64_t r0 = min(R, int64_t(tid) * chunk), r1 = min(R, r0 + chunk);
     const bool cached = R <= kPlanCacheRows;
     extern __shared__ int2 s_rows[];   // {target, unit} per row when cached
 
     // pass 1: classify (kept in shared memory when R is small enough) and count
     int na = 0, nb = 0, nonpad = 0;
     bool any_bad = false;
-    #pragma unroll 4
-    for (int64_t q = r0; q < r1; ++q) {
+    for (int64_t q = tid; q < R; q += kPlanThreads) {
         int tg, u;
         bool bad;
         classify(P, q, tg, u, bad);
         any_bad |= bad;
         if (tg >= 0) { if (q < P.a.n_tokens) ++na; else ++nb; }
+        if (q < P.a.n_tokens) nonpad += !(P.a.pad && P.a.pad[q]);
         if (cached) s_rows[q] = make_int2(tg, u);
     }
-    for (int64_t q = r0; q < r1 && q < P.a.n_tokens; ++q) nonpad += !(P.a.pad && P.a.pad[q]);
     if (any_bad) atomicOr(&s_status, DLM_DEV_BAD_TOKEN_ID);
-
-    // block totals (na, nb, nonpad) and the exclusive scan of scored rows
     {
         int v0 = na, v1 = nb, v2 = nonpad;
         #pragma unroll
@@ -203,43 +193,54 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
         }
         if (lane == 0) { s_sum[0][warp] = v0; s_sum[1][warp] = v1; s_sum[2][warp] = v2; }
     }
-    int n_scored;
-    const int scored_before = block_exclusive_scan(na + nb, s_warp, n_scored);
+    __syncthreads();
     int n_a = 0, n_b = 0, N = 0;
     #pragma unroll
     for (int w = 0; w < kPlanWarps; ++w) { n_a += s_sum[0][w]; n_b += s_sum[1][w]; N += s_sum[2][w]; }
-    int64_t so = scored_before;                          // next scored slot
-    int64_t uo = n_scored + (r0 - scored_before);        // next unscored slot
-
+    const int n_scored = n_a + n_b;
     const float w_canvas = n_a > 0 ? 1.0f / float(n_a) : 0.0f;
     const float w_enc = n_b > 0 ? P.lam / float(n_b) : 0.0f;
 
-    // pass 2: weights and the row list
-    auto emit = [&](int64_t q, int tg, int u) {
-        if (tg >= 0) {
-            float w;
-            if (q < P.a.n_tokens) {
-                w = P.mode == DLM_ABSORBING ? 1.0f / (__ldg(P.p + u) * float(N)) : w_canvas;
+    // pass 2: weights and the row list, T rows at a time in row order
+    int64_t base_s = 0, base_u = n_scored;   // next scored / unscored slot
+    const unsigned below = (1u << lane) - 1u;
+    for (int64_t t0 = 0; t0 < R; t0 += kPlanThreads) {
+        const int64_t q = t0 + tid;
+        const bool in = q < R;
+        int tg = -1, u = 0;
+        if (in) {
+            if (cached) {
+                const int2 c = s_rows[q];
+                tg = c.x;
+                u = c.y;
             } else {
-                w = w_enc;
+                bool bad;
+                classify(P, q, tg, u, bad);
             }
-            P.list[so++] = make_int4(int(q), tg, __float_as_int(w), u);
-        } else {
-            P.list[uo++] = make_int4(int(q), -1, 0, u);
         }
-    };
-    if (cached) {
-        for (int64_t q = r0; q < r1; ++q) {
-            const int2 c = s_rows[q];
-            emit(q, c.x, c.y);
+        const unsigned bs = __ballot_sync(0xffffffffu, in && tg >= 0);
+        const unsigned bu = __ballot_sync(0xffffffffu, in && tg < 0);
+        if (lane == 0) { s_cnt[0][warp] = __popc(bs); s_cnt[1][warp] = __popc(bu); }
+        __syncthreads();
+        int ps, ts, pu, tu;
+        warp_prefix(s_cnt[0], warp, lane, ps, ts);
+        warp_prefix(s_cnt[1], warp, lane, pu, tu);
+        __syncthreads();   // s_cnt is rewritten for the next rows
+        if (in) {
+            if (tg >= 0) {
+                float w;
+                if (q < P.a.n_tokens) {
+                    w = P.mode == DLM_ABSORBING ? 1.0f / (__ldg(P.p + u) * float(N)) : w_canvas;
+                } else {
+                    w = w_enc;
+                }
+                P.list[base_s + ps + __popc(bs & below)] = make_int4(int(q), tg, __float_as_int(w), u);
+            } else {
+                P.list[base_u + pu + __popc(bu & below)] = make_int4(int(q), -1, 0, u);
+            }
         }
-    } else {
-        for (int64_t q = r0; q < r1; ++q) {
-            int tg, u;
-            bool bad;
-            classify(P, q, tg, u, bad);
-            emit(q, tg, u);
-        }
+        base_s += ts;
+        base_u += tu;
     }
     __syncthreads();
     if (tid == 0) {
@@ -250,6 +251,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
         P.hdr->n_scored_a = n_a;
         P.hdr->n_scored_b = n_b;
         P.hdr->ticket = 0u;
+        P.hdr->next_s = 0u;
+        P.hdr->next_u = 0u;
     }
 }
 
@@ -337,6 +340,7 @@ struct StreamShape {
     static_assert(kVec * 8 * kConsumers == kChunk, "chunk split");
 };
 
+constexpr int kRowQ = 16;          // row entries in flight between producer and consumers (> stages / 2)
 constexpr int kMaxMine = 256;       // rows of each kind one CTA may take when it plans for itself
 // Below this many rows the one-CTA plan kernel (overlapped with the CE
 // kernel's launch) is cheaper than every CTA planning in its prologue;
@@ -352,6 +356,8 @@ struct __align__(128) StreamSmem {
     float red_m[2][WARPS];
     float red_s[2][WARPS];
     float xy[2];
+    int4 rowq[kRowQ];           // list entries of the rows the producer has started
+    int4 cur[2];                // the consumers' current row entry
     int abort;
     // self-planned share of the row list
     int4 mine_s[kMaxMine];      // scored rows {row, target, weight bits, unit}
@@ -540,12 +546,34 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
 
     if (warp == kConsumerWarps) {
         // ------------------------------ producer ------------------------------
+        // Rows come from the plan's list through two tickets in the workspace
+        // header (scored rows, unscored rows; zeroed by the plan kernel), so a
+        // CTA that streams faster simply takes more rows and all CTAs finish
+        // together; a self-planned CTA takes its own share.  Unscored rows are
+        // interleaved with the scored ones in the global ratio so the zero
+        // stream overlaps the consumers' work.  Each scored row's list entry
+        // is published in S.rowq before its first chunk's arrival, and an
+        // arrival without data (entry row -1) ends the consumers' loop.
         if (lane == 0) {
             const uint64_t pol_keep = policy_evict_last();
             const uint64_t pol_drop = policy_evict_first();
-            int seq = 0, zdone = 0;
-            auto zero_row = [&](int j) {
-                const int q = P.self_plan ? S.mine_u[j] : P.list[first_u + j * G].x;
+            const bool dyn = !P.self_plan;
+            const int n_uns = n_rows - n_scored;
+            const int64_t z_num = dyn ? n_uns : my_unscored, z_den = dyn ? n_scored : my_scored;
+            uint32_t* const tick_s = &P.hdr_w->next_s;
+            uint32_t* const tick_u = &P.hdr_w->next_u;
+            int seq = 0, k = 0, zdone = 0;
+            bool zleft = true, ok = true;
+            auto zero_next = [&]() {   // zero-fill one more unscored row, if any is left
+                int q;
+                if (dyn) {
+                    const int j = int(atomicAdd(tick_u, 1u));
+                    if (j >= n_uns) { zleft = false; return; }
+                    q = P.list[n_scored + j].x;
+                } else {
+                    if (zdone >= my_unscored) { zleft = false; return; }
+                    q = S.mine_u[zdone];
+                }
                 const uint16_t* xr;
                 uint16_t* dr;
                 row_ptrs(P, q, xr, dr);
@@ -556,31 +584,50 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
                 }
                 bulk_commit_group();
                 P.row_loss[q] = 0.f;
+                ++zdone;
             };
-            bool ok = true;
-            for (int k = 0; k < my_scored && ok; ++k) {
-                const int q = P.self_plan ? S.mine_s[k].x : P.list[blockIdx.x + k * G].x;
+            int i = dyn ? int(atomicAdd(tick_s, 1u)) : 0;
+            while (ok) {
+                int4 e;
+                if (dyn) {
+                    if (i >= n_scored) break;
+                    e = P.list[i];
+                    i = int(atomicAdd(tick_s, 1u));   // the next row's ticket, in flight meanwhile
+                } else {
+                    if (k >= my_scored) break;
+                    e = S.mine_s[k];
+                }
+                S.rowq[k % kRowQ] = e;
                 const uint16_t* xr;
                 uint16_t* dr;
-                row_ptrs(P, q, xr, dr);
+                row_ptrs(P, e.x, xr, dr);
                 for (int pass = 0; pass < 2 && ok; ++pass) {
                     for (int c = 0; c < nch; ++c, ++seq) {
                         const int st = seq % kStages;
                         if (!mbar_wait_or_abort(smem_addr(&S.empty[st]), ((seq / kStages) & 1) ^ 1, P.status,
                                                 abort)) { ok = false; break; }
-                        const int cc = c;
-                        const int e0 = cc * kChunk;
+                        const int e0 = c * kChunk;
                         const uint32_t bytes = uint32_t(min(kChunk, V - e0)) * 2u;
                         const uint32_t fb = smem_addr(&S.full[st]);
                         mbar_arrive_expect_tx(fb, bytes);
                         bulk_g2s_hint(smem_addr(S.ring[st]), xr + e0, bytes, fb, pass == 0 ? pol_keep : pol_drop);
                     }
                 }
-                // spread the zero rows evenly over the scored ones
-                const int want = my_scored ? int((int64_t(k + 1) * my_unscored) / my_scored) : 0;
-                while (ok && zdone < want) zero_row(zdone++);
+                ++k;
+                const int64_t want = z_den ? int64_t(k) * z_num / z_den : 0;
+                while (ok && zleft && zdone < want) zero_next();
             }
-            while (ok && zdone < my_unscored) zero_row(zdone++);
+            while (ok && zleft) zero_next();
+            if (ok) {
+                // end marker: the next stage arrives without data
+                const int st = seq % kStages;
+                if (mbar_wait_or_abort(smem_addr(&S.empty[st]), ((seq / kStages) & 1) ^ 1, P.status, abort)) {
+                    S.rowq[k % kRowQ] = make_int4(-1, -1, 0, 0);
+                    mbar_arrive(smem_addr(&S.full[st]));
+                } else {
+                    ok = false;
+                }
+            }
             if (!ok) {
                 // let the copies already issued land before this thread leaves
                 for (int j = seq - 1; j >= 0 && j >= seq - kStages; --j)
@@ -592,11 +639,20 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
     // ------------------------------ consumers ------------------------------
     const uint64_t pol_drop = policy_evict_first();
     int seq = 0;
-    auto entry = [&](int k) { return P.self_plan ? S.mine_s[k] : P.list[blockIdx.x + k * G]; };
-    int4 e_next = my_scored > 0 ? entry(0) : make_int4(0, -1, 0, 0);
-    for (int k = 0; k < my_scored; ++k) {
-        const int4 e = e_next;
-        if (k + 1 < my_scored) e_next = entry(k + 1);
+    for (int k = 0;; ++k) {
+        // The first chunk of the next row; its arrival also publishes the
+        // row's entry.  Thread 0 reads it (or decides to stop after an abort)
+        // and hands it to every consumer warp, so all of them leave the loop
+        // together and every barrier below is met by all.
+        mbar_wait_or_abort(smem_addr(&S.full[seq % kStages]), (seq / kStages) & 1, P.status, abort);
+        if (tid == 0) {
+            int4 e0 = S.rowq[k % kRowQ];
+            if (*abort) e0.x = -1;
+            S.cur[k & 1] = e0;
+        }
+        named_barrier_sync(2, kConsumers);
+        const int4 e = S.cur[k & 1];
+        if (e.x < 0) break;
         const int q = e.x, y = e.y;
         const float w = __int_as_float(e.z);
         const int par = k & 1;
@@ -610,7 +666,7 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
         float m = -INFINITY, s = 0.f;
         for (int c = 0; c < nch; ++c, ++seq) {
             const int st = seq % kStages;
-            mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort);
+            if (c > 0) mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort);
             const int e0 = c * kChunk;
             uint4 raw[kVecPerThread];
             float cm = -INFINITY;

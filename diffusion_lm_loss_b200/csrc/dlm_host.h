@@ -79,6 +79,8 @@ struct WsHeader {
     int32_t n_scored_a;   // scored diffusion rows
     int32_t n_scored_b;   // scored encoder rows
     uint32_t ticket;      // completion counter of the unit reduction (zeroed by the plan)
+    uint32_t next_s;      // CE row tickets: next scored / unscored list entry (zeroed by the plan)
+    uint32_t next_u;
 };
 static_assert(sizeof(WsHeader) <= kWsAlign, "header");
 
