@@ -10,8 +10,8 @@
 // Three launches per call, all on the caller's stream:
 //   1. k_plan     one CTA: classifies every logits row (scored or not, its
 //                 target, unit and weight), counts N, and writes a row list
-//                 with the scored rows first -- so the CE kernel can deal the
-//                 expensive rows out evenly.
+//                 with the scored rows first; the CE kernel's CTAs take the
+//                 list's rows by ticket.
 //   2. k_ce_*     the hot kernel, HBM-bound: every scored row must be read
 //                 (V*2 bytes) and every row's gradient written (V*2 bytes).
 //                 Fast path (k_ce_stream): per SM one or two CTAs of a TMA
@@ -26,7 +26,8 @@
 //                 passes; L2 holds it instead.
 //                 General path (k_ce_generic): any V / ld / alignment, one CTA
 //                 per row, two passes over the row with plain loads.
-//   3. k_reduce   one CTA: per-unit sums and the total, fixed order, double.
+//   3. k_reduce   one CTA per unit: per-unit sums and the total, fixed order,
+//                 double.
 #include <mutex>
 
 #include "dlm_device.cuh"
@@ -155,8 +156,68 @@ __device__ __forceinline__ void warp_prefix(const int* s_cnt, int warp, int lane
 // found from a warp ballot plus a prefix over the warps -- 16-byte list
 // stores that coalesce.  The list holds the scored rows in row order, then
 // all other rows in row order.
+constexpr int kPlanBatch = 4;   // rows per thread whose loads are in flight together
+
+// Classification of the kPlanBatch rows q0, q0 + T, ... of one thread in two
+// phases: every address first, then every load (flag, target id, pads, p)
+// with nothing waiting on another, then the decisions -- one memory round
+// trip for the batch instead of one per row.  Same result as classify().
+__device__ __forceinline__ void classify_batch(const PlanParams& P, int64_t q0, int64_t R, int (&tg)[kPlanBatch],
+                                               int (&u)[kPlanBatch], float (&pu)[kPlanBatch], bool& any_bad,
+                                               int& na, int& nb, int& nonpad) {
+    int64_t jj[kPlanBatch];
+    bool ok[kPlanBatch], ina[kPlanBatch], valid[kPlanBatch];
+    #pragma unroll
+    for (int k = 0; k < kPlanBatch; ++k) {
+        const int64_t q = q0 + int64_t(k) * kPlanThreads;
+        valid[k] = q < R;
+        ina[k] = q < P.a.n_tokens;
+        const LayoutDev& L = ina[k] ? P.a : P.b;
+        const int64_t i = !valid[k] ? 0 : (ina[k] ? q : q - P.a.n_tokens);
+        int64_t end = 0;
+        u[k] = 0;
+        if (valid[k]) unit_pos(L, i, u[k], end);
+        const int64_t j = (ina[k] && P.align == DLM_ALIGNED) ? i : i + 1;
+        ok[k] = valid[k] && j < end && j < L.n_tokens;
+        jj[k] = ok[k] ? j : 0;
+    }
+    const bool absorbing = P.mode == DLM_ABSORBING;
+    uint8_t cf[kPlanBatch], pd[kPlanBatch], pq[kPlanBatch];
+    int y[kPlanBatch];
+    #pragma unroll
+    for (int k = 0; k < kPlanBatch; ++k) {
+        const int64_t q = q0 + int64_t(k) * kPlanThreads;
+        const LayoutDev& L = ina[k] ? P.a : P.b;
+        const bool need_c = ok[k] && ina[k] && absorbing;
+        cf[k] = need_c ? P.corrupted[jj[k]] : uint8_t(1);
+        pd[k] = (ok[k] && L.pad) ? L.pad[jj[k]] : uint8_t(0);
+        y[k] = ok[k] ? (ina[k] ? P.clean_a[jj[k]] : P.ids_b[jj[k]]) : -1;
+        pu[k] = (valid[k] && ina[k] && absorbing) ? __ldg(P.p + u[k]) : 0.f;
+        pq[k] = (valid[k] && ina[k] && P.a.pad) ? P.a.pad[q] : uint8_t(0);
+    }
+    #pragma unroll
+    for (int k = 0; k < kPlanBatch; ++k) {
+        tg[k] = -1;
+        if (valid[k] && ina[k]) nonpad += !pq[k];
+        if (!ok[k] || pd[k] || !cf[k]) continue;
+        if (y[k] < 0 || y[k] >= P.vocab) { any_bad = true; continue; }
+        tg[k] = y[k];
+        if (ina[k]) ++na; else ++nb;
+    }
+}
+
+// One CTA.  Thread t takes rows t, t + T, t + 2T, ... (T = kPlanThreads), so
+// a warp always works on 32 consecutive rows: its loads are coalesced, and in
+// pass 2 its scored rows (and its other rows) land in consecutive list slots,
+// found from a warp ballot plus a prefix over the warps -- 16-byte list
+// stores that coalesce.  The list holds the scored rows in row order, then
+// all other rows in row order.  Up to kPlanCacheRows rows, pass 1 keeps each
+// row's classification and every warp's counts in shared memory and pass 2
+// needs no global load and no barrier; beyond that, pass 2 classifies again,
+// T rows at a time.
 __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
-    __shared__ int s_cnt[2][kPlanWarps];
+    constexpr int kTiles = kPlanCacheRows / kPlanThreads;
+    __shared__ int s_cnt[2][kTiles][kPlanWarps];   // per T-row tile and warp: scored / other rows
     __shared__ int s_sum[3][kPlanWarps];
     __shared__ uint32_t s_status;
     pdl_launch_dependents();   // the CE kernel may start its prologue now
@@ -168,19 +229,35 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
 
     const int64_t R = P.a.n_tokens + P.b.n_tokens;
     const bool cached = R <= kPlanCacheRows;
-    extern __shared__ int2 s_rows[];   // {target, unit} per row when cached
+    extern __shared__ int2 s_rows[];   // cached: {target, unit} per row, then p of the row's unit
+    float* s_p = reinterpret_cast<float*>(s_rows + (cached ? R : 0));
 
-    // pass 1: classify (kept in shared memory when R is small enough) and count
+    // pass 1: classify and count
     int na = 0, nb = 0, nonpad = 0;
     bool any_bad = false;
-    for (int64_t q = tid; q < R; q += kPlanThreads) {
-        int tg, u;
-        bool bad;
-        classify(P, q, tg, u, bad);
-        any_bad |= bad;
-        if (tg >= 0) { if (q < P.a.n_tokens) ++na; else ++nb; }
-        if (q < P.a.n_tokens) nonpad += !(P.a.pad && P.a.pad[q]);
-        if (cached) s_rows[q] = make_int2(tg, u);
+    // the bound is the same for every thread (the ballots below need whole warps)
+    for (int64_t base = 0; base < R; base += int64_t(kPlanThreads) * kPlanBatch) {
+        const int64_t q0 = base + tid;
+        int tg[kPlanBatch], u[kPlanBatch];
+        float pu[kPlanBatch];
+        classify_batch(P, q0, R, tg, u, pu, any_bad, na, nb, nonpad);
+        if (cached) {
+            #pragma unroll
+            for (int k = 0; k < kPlanBatch; ++k) {
+                const int64_t q = q0 + int64_t(k) * kPlanThreads;
+                const unsigned bs = __ballot_sync(0xffffffffu, q < R && tg[k] >= 0);
+                const unsigned bv = __ballot_sync(0xffffffffu, q < R);
+                const int t = int((q - tid) / kPlanThreads);
+                if (q - tid < R && lane == 0) {
+                    s_cnt[0][t][warp] = __popc(bs);
+                    s_cnt[1][t][warp] = __popc(bv & ~bs);
+                }
+                if (q < R) {
+                    s_rows[q] = make_int2(tg[k], u[k]);
+                    s_p[q] = pu[k];
+                }
+            }
+        }
     }
     if (any_bad) atomicOr(&s_status, DLM_DEV_BAD_TOKEN_ID);
     {
@@ -200,47 +277,60 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
     const int n_scored = n_a + n_b;
     const float w_canvas = n_a > 0 ? 1.0f / float(n_a) : 0.0f;
     const float w_enc = n_b > 0 ? P.lam / float(n_b) : 0.0f;
+    auto weight = [&](int64_t q, int u, float pu) {
+        if (q >= P.a.n_tokens) return w_enc;
+        return P.mode == DLM_ABSORBING ? 1.0f / (pu * float(N)) : w_canvas;
+    };
 
     // pass 2: weights and the row list, T rows at a time in row order
     int64_t base_s = 0, base_u = n_scored;   // next scored / unscored slot
     const unsigned below = (1u << lane) - 1u;
-    for (int64_t t0 = 0; t0 < R; t0 += kPlanThreads) {
-        const int64_t q = t0 + tid;
-        const bool in = q < R;
-        int tg = -1, u = 0;
-        if (in) {
-            if (cached) {
-                const int2 c = s_rows[q];
-                tg = c.x;
-                u = c.y;
-            } else {
-                bool bad;
-                classify(P, q, tg, u, bad);
+    if (cached) {
+        for (int t = 0; int64_t(t) * kPlanThreads < R; ++t) {
+            const int64_t q = int64_t(t) * kPlanThreads + tid;
+            const bool in = q < R;
+            const int2 c = in ? s_rows[q] : make_int2(-1, 0);
+            const unsigned bs = __ballot_sync(0xffffffffu, in && c.x >= 0);
+            const unsigned bu = __ballot_sync(0xffffffffu, in && c.x < 0);
+            int ps, ts, pu, tu;
+            warp_prefix(s_cnt[0][t], warp, lane, ps, ts);
+            warp_prefix(s_cnt[1][t], warp, lane, pu, tu);
+            if (in) {
+                if (c.x >= 0)
+                    P.list[base_s + ps + __popc(bs & below)] =
+                        make_int4(int(q), c.x, __float_as_int(weight(q, c.y, s_p[q])), c.y);
+                else
+                    P.list[base_u + pu + __popc(bu & below)] = make_int4(int(q), -1, 0, c.y);
             }
+            base_s += ts;
+            base_u += tu;
         }
-        const unsigned bs = __ballot_sync(0xffffffffu, in && tg >= 0);
-        const unsigned bu = __ballot_sync(0xffffffffu, in && tg < 0);
-        if (lane == 0) { s_cnt[0][warp] = __popc(bs); s_cnt[1][warp] = __popc(bu); }
-        __syncthreads();
-        int ps, ts, pu, tu;
-        warp_prefix(s_cnt[0], warp, lane, ps, ts);
-        warp_prefix(s_cnt[1], warp, lane, pu, tu);
-        __syncthreads();   // s_cnt is rewritten for the next rows
-        if (in) {
-            if (tg >= 0) {
-                float w;
-                if (q < P.a.n_tokens) {
-                    w = P.mode == DLM_ABSORBING ? 1.0f / (__ldg(P.p + u) * float(N)) : w_canvas;
+    } else {
+        for (int64_t t0 = 0; t0 < R; t0 += kPlanThreads) {
+            const int64_t q = t0 + tid;
+            const bool in = q < R;
+            int tg = -1, u = 0;
+            bool bad;
+            if (in) classify(P, q, tg, u, bad);
+            const unsigned bs = __ballot_sync(0xffffffffu, in && tg >= 0);
+            const unsigned bu = __ballot_sync(0xffffffffu, in && tg < 0);
+            if (lane == 0) { s_cnt[0][0][warp] = __popc(bs); s_cnt[1][0][warp] = __popc(bu); }
+            __syncthreads();
+            int ps, ts, pu, tu;
+            warp_prefix(s_cnt[0][0], warp, lane, ps, ts);
+            warp_prefix(s_cnt[1][0], warp, lane, pu, tu);
+            __syncthreads();   // s_cnt is rewritten for the next rows
+            if (in) {
+                if (tg >= 0) {
+                    const float pv = (q < P.a.n_tokens && P.mode == DLM_ABSORBING) ? __ldg(P.p + u) : 0.f;
+                    P.list[base_s + ps + __popc(bs & below)] = make_int4(int(q), tg, __float_as_int(weight(q, u, pv)), u);
                 } else {
-                    w = w_enc;
+                    P.list[base_u + pu + __popc(bu & below)] = make_int4(int(q), -1, 0, u);
                 }
-                P.list[base_s + ps + __popc(bs & below)] = make_int4(int(q), tg, __float_as_int(w), u);
-            } else {
-                P.list[base_u + pu + __popc(bu & below)] = make_int4(int(q), -1, 0, u);
             }
+            base_s += ts;
+            base_u += tu;
         }
-        base_s += ts;
-        base_u += tu;
     }
     __syncthreads();
     if (tid == 0) {
@@ -263,15 +353,7 @@ struct CeParams {
     const int4* list;
     const WsHeader* hdr;
     uint32_t* status;
-    // self_plan = 1: no row-plan kernel ran; each CTA of k_ce_stream builds its
-    // own share of the plan (dense layout, no pads, absorbing, no encoder)
-    int self_plan;
-    WsHeader* hdr_w;
-    const uint8_t* corrupted;
-    const int32_t* clean;
-    const float* p;
-    int seq_len;
-    int align;
+    WsHeader* hdr_w;         // the same header, written: the row tickets
     const uint16_t* xa; uint16_t* da; int64_t lda; int64_t rows_a;
     const uint16_t* xb; uint16_t* db; int64_t ldb;
     int vocab;
@@ -341,11 +423,6 @@ struct StreamShape {
 };
 
 constexpr int kRowQ = 16;          // row entries in flight between producer and consumers (> stages / 2)
-constexpr int kMaxMine = 256;       // rows of each kind one CTA may take when it plans for itself
-// Below this many rows the one-CTA plan kernel (overlapped with the CE
-// kernel's launch) is cheaper than every CTA planning in its prologue;
-// measured: 4,096 rows +2.3% with self-planning, 16,384 rows -1.3%.
-constexpr int64_t kSelfPlanMinRows = 8192;
 
 template <int WARPS, int STAGES>
 struct __align__(128) StreamSmem {
@@ -359,90 +436,7 @@ struct __align__(128) StreamSmem {
     int4 rowq[kRowQ];           // list entries of the rows the producer has started
     int4 cur[2];                // the consumers' current row entry
     int abort;
-    // self-planned share of the row list
-    int4 mine_s[kMaxMine];      // scored rows {row, target, weight bits, unit}
-    int mine_u[kMaxMine];       // unscored rows
-    int scan[32];
-    int total;
-    uint32_t bad;
 };
-
-// Self-plan flags of 16 consecutive rows q0..q0+15 (dense layout, no pads,
-// absorbing): bit i set when row q0+i is scored -- its target token j (q or
-// q+1 of the same sequence) is corrupted and holds a valid id.  `bad` gets
-// bits for corrupted targets with ids outside [0, V).  The targets are
-// returned in y[].
-__device__ __forceinline__ uint32_t self_plan_flags(const CeParams& P, int R, int q0, int (&y)[16],
-                                                    bool& bad) {
-    const int sh = P.align == DLM_SHIFTED ? 1 : 0;
-    uint8_t c[16];
-    if (q0 + 16 + sh <= R) {
-        const uint4 cv = *reinterpret_cast<const uint4*>(P.corrupted + q0);
-        const uint4 i0 = *reinterpret_cast<const uint4*>(P.clean + q0);
-        const uint4 i1 = *reinterpret_cast<const uint4*>(P.clean + q0 + 4);
-        const uint4 i2 = *reinterpret_cast<const uint4*>(P.clean + q0 + 8);
-        const uint4 i3 = *reinterpret_cast<const uint4*>(P.clean + q0 + 12);
-        const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
-        int ids[17] = {int(i0.x), int(i0.y), int(i0.z), int(i0.w), int(i1.x), int(i1.y), int(i1.z), int(i1.w),
-                       int(i2.x), int(i2.y), int(i2.z), int(i2.w), int(i3.x), int(i3.y), int(i3.z), int(i3.w), 0};
-        uint8_t cc[17];
-        #pragma unroll
-        for (int i = 0; i < 16; ++i) cc[i] = uint8_t(cw[i >> 2] >> (8 * (i & 3)));
-        cc[16] = 0;
-        if (sh) { cc[16] = P.corrupted[q0 + 16]; ids[16] = P.clean[q0 + 16]; }
-        #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            c[i] = sh ? cc[i + 1] : cc[i];
-            y[i] = sh ? ids[i + 1] : ids[i];
-        }
-    } else {
-        #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int j = q0 + i + sh;
-            c[i] = j < R ? P.corrupted[j] : 0;
-            y[i] = j < R ? P.clean[j] : 0;
-        }
-    }
-    uint32_t f = 0;
-    #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int q = q0 + i;
-        const bool same_unit = !sh || ((q + 1) % P.seq_len != 0);
-        if (q < R && same_unit && c[i]) {
-            if (y[i] >= 0 && y[i] < P.vocab) f |= 1u << i;
-            else bad = true;
-        }
-    }
-    return f;
-}
-
-// Exclusive scan of one int per thread over the CTA (up to 32 warps); the
-// CTA total is returned in `total`.  Uses sm_scan[32].
-__device__ __forceinline__ int cta_exclusive_scan(int v, int* sm_scan, int nwarps, int& total) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
-    #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += t;
-    }
-    if (lane == 31) sm_scan[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < nwarps ? sm_scan[lane] : 0;
-        #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int t = __shfl_up_sync(0xffffffffu, w, o);
-            if (lane >= o) w += t;
-        }
-        if (lane < nwarps) sm_scan[lane] = w;
-    }
-    __syncthreads();
-    total = sm_scan[nwarps - 1];
-    const int r = (warp ? sm_scan[warp - 1] : 0) + x - v;
-    __syncthreads();
-    return r;
-}
 
 template <int WARPS, int STAGES, int CTAS>
 __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_ce_stream(const CeParams P) {
@@ -457,7 +451,6 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int V = P.vocab;
     const int nch = (V + kChunk - 1) / kChunk;
-    const int G = gridDim.x;
     volatile int* abort = &S.abort;
 
     for (int i = tid; i < kZeroBytes / 16; i += kStreamThreads) S.zero[i] = make_uint4(0, 0, 0, 0);
@@ -467,89 +460,23 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
             mbar_init(smem_addr(&S.empty[i]), kConsumerWarps);
         }
         S.abort = 0;
-        S.bad = 0u;
         fence_mbar_init_cluster();
     }
     fence_proxy_async_smem();   // zero block visible to the bulk-copy engine
     __syncthreads();
-    pdl_wait();                 // the previous kernel (row plan, or corruption) is complete
+    pdl_wait();                 // the row plan is complete
     pdl_launch_dependents();    // the reduction may start its prologue
 
-    int n_scored, n_rows;
-    if (P.self_plan) {
-        // This CTA's share of the row plan, built from the corruption flags:
-        // sweep A counts the scored rows, sweep B ranks them (row order) and
-        // keeps ranks == blockIdx.x (mod G), and the unscored rows whose place
-        // in the continued deal falls to this CTA.
-        const int R = int(P.rows_a);
-        const int span = 16 * kStreamThreads;
-        const int nwarps = kStreamThreads / 32;
-        int y[16];
-        bool bad = false;
-        int cnt = 0;
-        for (int t0 = 0; t0 < R; t0 += span) {
-            const int q0 = t0 + tid * 16;
-            cnt += __popc(self_plan_flags(P, R, q0, y, bad));
-        }
-        int tot;
-        cta_exclusive_scan(cnt, S.scan, nwarps, tot);
-        n_scored = tot;
-        n_rows = R;
-        const int b = blockIdx.x;
-        const int first_u0 = n_scored + ((b - n_scored) % G + G) % G;
-        int base = 0;
-        for (int t0 = 0; t0 < R; t0 += span) {
-            const int q0 = t0 + tid * 16;
-            const uint32_t f = self_plan_flags(P, R, q0, y, bad);
-            int tile_tot;
-            const int before = base + cta_exclusive_scan(__popc(f), S.scan, nwarps, tile_tot);
-            #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int q = q0 + i;
-                if (q >= R) break;
-                const int rank = before + __popc(f & ((1u << i) - 1u));
-                if (f >> i & 1u) {
-                    if (rank % G == b) {
-                        const int u = q / P.seq_len;
-                        const float w = 1.0f / (__ldg(P.p + u) * float(R));
-                        S.mine_s[rank / G] = make_int4(q, y[i], __float_as_int(w), u);
-                    }
-                } else {
-                    const int vi = n_scored + (q - rank);   // place in the continued deal
-                    if (vi >= first_u0 && (vi - first_u0) % G == 0) S.mine_u[(vi - first_u0) / G] = q;
-                }
-            }
-            base += tile_tot;
-        }
-        if (bad) atomicOr(&S.bad, 1u);
-        __syncthreads();
-        if (b == 0 && tid == 0) {
-            P.hdr_w->status = S.bad ? DLM_DEV_BAD_TOKEN_ID : 0u;
-            P.hdr_w->n_scored = n_scored;
-            P.hdr_w->n_rows = n_rows;
-            P.hdr_w->n_nonpad = R;
-            P.hdr_w->n_scored_a = n_scored;
-            P.hdr_w->n_scored_b = 0;
-            P.hdr_w->ticket = 0u;
-        }
-    } else {
-        n_scored = P.hdr->n_scored;
-        n_rows = P.hdr->n_rows;
-    }
-    const int my_scored = blockIdx.x < n_scored ? (n_scored - blockIdx.x + G - 1) / G : 0;
-    // The list (scored rows first) is dealt round-robin as one sequence: CTA b
-    // takes entries b, b+G, ...  The scored ones come first; its unscored
-    // entries continue the same deal, so a CTA that got one scored row fewer
-    // gets the extra unscored row instead.
-    const int first_u = n_scored + ((int(blockIdx.x) - n_scored) % G + G) % G;   // first entry >= n_scored of this CTA
-    const int my_unscored = first_u < n_rows ? (n_rows - first_u + G - 1) / G : 0;
+    const int n_scored = P.hdr->n_scored;
+    const int n_rows = P.hdr->n_rows;
 
     if (warp == kConsumerWarps) {
         // ------------------------------ producer ------------------------------
         // Rows come from the plan's list through two tickets in the workspace
         // header (scored rows, unscored rows; zeroed by the plan kernel), so a
         // CTA that streams faster simply takes more rows and all CTAs finish
-        // together; a self-planned CTA takes its own share.  Unscored rows are
+        // together (a fixed deal left the last CTAs finishing ~70 us after the
+        // first on a 0.3 ms call, with HBM idling behind them).  Unscored rows are
         // interleaved with the scored ones in the global ratio so the zero
         // stream overlaps the consumers' work.  Each scored row's list entry
         // is published in S.rowq before its first chunk's arrival, and an
@@ -557,23 +484,15 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
         if (lane == 0) {
             const uint64_t pol_keep = policy_evict_last();
             const uint64_t pol_drop = policy_evict_first();
-            const bool dyn = !P.self_plan;
             const int n_uns = n_rows - n_scored;
-            const int64_t z_num = dyn ? n_uns : my_unscored, z_den = dyn ? n_scored : my_scored;
             uint32_t* const tick_s = &P.hdr_w->next_s;
             uint32_t* const tick_u = &P.hdr_w->next_u;
             int seq = 0, k = 0, zdone = 0;
             bool zleft = true, ok = true;
             auto zero_next = [&]() {   // zero-fill one more unscored row, if any is left
-                int q;
-                if (dyn) {
-                    const int j = int(atomicAdd(tick_u, 1u));
-                    if (j >= n_uns) { zleft = false; return; }
-                    q = P.list[n_scored + j].x;
-                } else {
-                    if (zdone >= my_unscored) { zleft = false; return; }
-                    q = S.mine_u[zdone];
-                }
+                const int j = int(atomicAdd(tick_u, 1u));
+                if (j >= n_uns) { zleft = false; return; }
+                const int q = P.list[n_scored + j].x;
                 const uint16_t* xr;
                 uint16_t* dr;
                 row_ptrs(P, q, xr, dr);
@@ -586,17 +505,10 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
                 P.row_loss[q] = 0.f;
                 ++zdone;
             };
-            int i = dyn ? int(atomicAdd(tick_s, 1u)) : 0;
-            while (ok) {
-                int4 e;
-                if (dyn) {
-                    if (i >= n_scored) break;
-                    e = P.list[i];
-                    i = int(atomicAdd(tick_s, 1u));   // the next row's ticket, in flight meanwhile
-                } else {
-                    if (k >= my_scored) break;
-                    e = S.mine_s[k];
-                }
+            int i = int(atomicAdd(tick_s, 1u));
+            while (ok && i < n_scored) {
+                const int4 e = P.list[i];
+                i = int(atomicAdd(tick_s, 1u));   // the next row's ticket, in flight meanwhile
                 S.rowq[k % kRowQ] = e;
                 const uint16_t* xr;
                 uint16_t* dr;
@@ -614,7 +526,7 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
                     }
                 }
                 ++k;
-                const int64_t want = z_den ? int64_t(k) * z_num / z_den : 0;
+                const int64_t want = int64_t(k) * n_uns / n_scored;
                 while (ok && zleft && zdone < want) zero_next();
             }
             while (ok && zleft) zero_next();
@@ -912,6 +824,11 @@ __global__ void __launch_bounds__(kRedThreads) k_reduce(ReduceParams R) {
             if (R.unit_loss) R.unit_loss[u] = float(t);
         }
     }
+    if (gridDim.x == 1) {
+        // at most one unit: its sum is the total (no hand-off between CTAs)
+        if (tid == 0) R.loss[0] = U > 0 ? float(R.unit_acc[0]) : 0.f;
+        return;
+    }
     // last CTA: the total
     if (tid == 0) {
         __threadfence();
@@ -993,7 +910,7 @@ dlm_status_t launch_plan(const dlm_layout_t* a, const int32_t* clean, const uint
     pp.hdr = hdr;
     pp.list = list;
     const int64_t R = (a ? a->n_tokens : 0) + (b ? b->n_tokens : 0);
-    const size_t smem = R <= kPlanCacheRows ? size_t(R) * sizeof(int2) : 0;
+    const size_t smem = R <= kPlanCacheRows ? size_t(R) * (sizeof(int2) + sizeof(float)) : 0;
     static std::mutex mu;
     static bool attr[64] = {};
     int dev = 0;
@@ -1002,7 +919,7 @@ dlm_status_t launch_plan(const dlm_layout_t* a, const int32_t* clean, const uint
         std::lock_guard<std::mutex> g(mu);
         if (dev >= 0 && dev < 64 && !attr[dev]) {
             cudaError_t e = cudaFuncSetAttribute(k_plan, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 int(kPlanCacheRows * sizeof(int2)));
+                                                 int(kPlanCacheRows * (sizeof(int2) + sizeof(float))));
             if (e != cudaSuccess) return cuda_status(e, "k_plan smem attribute");
             attr[dev] = true;
         }
@@ -1090,23 +1007,11 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
     if (has_enc) fast = fast && (enc_ld % 8 == 0) && aligned16(enc_logits) && aligned16(enc_dlogits);
     const bool two_per_sm = double(sms) * 2.0 * 2.0 * double(vocab) <= kL2RowBudget;
     if (fast) fast = two_per_sm ? stream_kernel_ready<8, 6, 2>(dev) : stream_kernel_ready<16, 12, 1>(dev);
-    const int64_t G = fast ? (R < int64_t(sms) * (two_per_sm ? 2 : 1) ? R : int64_t(sms) * (two_per_sm ? 2 : 1)) : 0;
-    // the CTAs plan for themselves (no row-plan kernel) on the common layout:
-    // dense sequences, no pads, absorbing noise, no encoder term
-#ifndef DLM_CE_SELF_PLAN
-#define DLM_CE_SELF_PLAN 1
-#endif
-    const bool self_plan = DLM_CE_SELF_PLAN && fast && !layout->cu_seqlens && !layout->pad_mask && mode == DLM_ABSORBING && !has_enc &&
-                           layout->seq_len > 0 && aligned16(clean_ids) && aligned16(corrupted) &&
-                           R <= G * int64_t(kMaxMine) && R >= kSelfPlanMinRows;
-
 
     // ---- 1. plan ----
-    if (!self_plan) {
-        if ((st = launch_plan(layout, clean_ids, corrupted, p, mode, align, lb, enc_ids, enc_ar_weight, vocab,
-                              hdr, list, s)) != DLM_OK)
-            return st;
-    }
+    if ((st = launch_plan(layout, clean_ids, corrupted, p, mode, align, lb, enc_ids, enc_ar_weight, vocab,
+                          hdr, list, s)) != DLM_OK)
+        return st;
 
     // ---- 2. CE ----
     if (R > 0) {
@@ -1119,13 +1024,7 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
         cp.vocab = vocab;
         cp.grad_scale = grad_scale;
         cp.row_loss = row_loss;
-        cp.self_plan = self_plan ? 1 : 0;
         cp.hdr_w = hdr;
-        cp.corrupted = corrupted;
-        cp.clean = clean_ids;
-        cp.p = p;
-        cp.seq_len = layout->seq_len;
-        cp.align = align;
 
         bool launched = false;
         if (fast) {

@@ -108,6 +108,17 @@ def test_llada_like_full_size():
                       grad_rows=_sample_rows(4096, 4096, seed=seed))
 
 
+@pytest.mark.parametrize("align", [oracle.ALIGNED, oracle.SHIFTED])
+def test_rows_beyond_the_plan_cache(align):
+    """20,000 rows: more rows than the plan keeps in shared memory, so the
+    list is built by the plan's second, re-classifying pass."""
+    spec = di.WORKLOADS["abs_b1_l4096_v126464"].scaled(vocab=4096, mask_id=4095, ids_high=4000, n_units=5,
+                                                       seq_len=4000, spike=0.0, align=align)
+    case = di.make_case(spec, "cuda")
+    run_absorbing(spec, case.logits, case.clean, n_units=5, seq_len=4000, seed=7,
+                  grad_rows=_sample_rows(20000, 4000, seed=7))
+
+
 def test_dream_like_shifted_mid_size_elementwise():
     spec = di.WORKLOADS["shift_b8_l2048_v152064"].scaled(n_units=3, seq_len=100)
     case = di.make_case(spec, "cuda")
