@@ -114,17 +114,18 @@ __device__ __forceinline__ void classify(const PlanParams& P, int64_t q, int& ta
     target = y;
 }
 
-#ifndef DLM_PLAN_THREADS
-#define DLM_PLAN_THREADS 1024
-#endif
-constexpr int kPlanThreads = DLM_PLAN_THREADS;
+// The plan runs as one cluster of kPlanCluster CTAs (one per SM), each
+// planning a contiguous slice of the rows: on a single SM the per-row
+// instructions alone took ~9 us for 4,096 rows.
+constexpr int kPlanCluster = 8;
+constexpr int kPlanThreads = 512;
 constexpr int kPlanWarps = kPlanThreads / 32;
 
-__device__ __forceinline__ bool layout_bad(const LayoutDev& L) {
-    // every thread checks a strided part of cu_seqlens
+// cu_seqlens consistency, split over all threads of the cluster
+__device__ __forceinline__ bool layout_bad(const LayoutDev& L, int first, int stride) {
     if (!L.cu) return false;
     bool bad = false;
-    for (int i = threadIdx.x; i <= L.n_units; i += blockDim.x) {
+    for (int i = first; i <= L.n_units; i += stride) {
         const int32_t c = L.cu[i];
         if (i == 0 && c != 0) bad = true;
         if (i == L.n_units && int64_t(c) != L.n_tokens) bad = true;
@@ -133,7 +134,7 @@ __device__ __forceinline__ bool layout_bad(const LayoutDev& L) {
     return bad;
 }
 
-constexpr int kPlanCacheRows = 16384;   // rows whose classification is kept in shared memory
+constexpr int kPlanCacheRows = 16384;   // rows per CTA whose classification stays in shared memory
 
 // Exclusive prefix over the warps of the CTA of one count per warp, and the
 // CTA total, from s_cnt[warp]; every lane of every warp gets the values for
@@ -150,19 +151,13 @@ __device__ __forceinline__ void warp_prefix(const int* s_cnt, int warp, int lane
     total = __shfl_sync(0xffffffffu, x, 31);
 }
 
-// One CTA.  Thread t takes rows t, t + T, t + 2T, ... (T = kPlanThreads), so
-// a warp always works on 32 consecutive rows: its loads are coalesced, and in
-// pass 2 its scored rows (and its other rows) land in consecutive list slots,
-// found from a warp ballot plus a prefix over the warps -- 16-byte list
-// stores that coalesce.  The list holds the scored rows in row order, then
-// all other rows in row order.
 constexpr int kPlanBatch = 4;   // rows per thread whose loads are in flight together
 
 // Classification of the kPlanBatch rows q0, q0 + T, ... of one thread in two
 // phases: every address first, then every load (flag, target id, pads, p)
 // with nothing waiting on another, then the decisions -- one memory round
 // trip for the batch instead of one per row.  Same result as classify().
-__device__ __forceinline__ void classify_batch(const PlanParams& P, int64_t q0, int64_t R, int (&tg)[kPlanBatch],
+__device__ __forceinline__ void classify_batch(const PlanParams& P, int64_t q0, int64_t hi, int (&tg)[kPlanBatch],
                                                int (&u)[kPlanBatch], float (&pu)[kPlanBatch], bool& any_bad,
                                                int& na, int& nb, int& nonpad) {
     int64_t jj[kPlanBatch];
@@ -170,7 +165,7 @@ __device__ __forceinline__ void classify_batch(const PlanParams& P, int64_t q0, 
     #pragma unroll
     for (int k = 0; k < kPlanBatch; ++k) {
         const int64_t q = q0 + int64_t(k) * kPlanThreads;
-        valid[k] = q < R;
+        valid[k] = q < hi;
         ina[k] = q < P.a.n_tokens;
         const LayoutDev& L = ina[k] ? P.a : P.b;
         const int64_t i = !valid[k] ? 0 : (ina[k] ? q : q - P.a.n_tokens);
@@ -206,55 +201,73 @@ __device__ __forceinline__ void classify_batch(const PlanParams& P, int64_t q0, 
     }
 }
 
-// One CTA.  Thread t takes rows t, t + T, t + 2T, ... (T = kPlanThreads), so
-// a warp always works on 32 consecutive rows: its loads are coalesced, and in
-// pass 2 its scored rows (and its other rows) land in consecutive list slots,
-// found from a warp ballot plus a prefix over the warps -- 16-byte list
-// stores that coalesce.  The list holds the scored rows in row order, then
-// all other rows in row order.  Up to kPlanCacheRows rows, pass 1 keeps each
-// row's classification and every warp's counts in shared memory and pass 2
-// needs no global load and no barrier; beyond that, pass 2 classifies again,
-// T rows at a time.
+// Load a 32-bit value from the shared memory of another CTA of the cluster.
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr_cluster) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr_cluster) : "memory");
+    return v;
+}
+
+// One cluster; CTA c plans rows [lo, hi) of an even split.  In its slice
+// thread t takes rows lo + t, lo + t + T, ... (T = kPlanThreads), so a warp
+// always works on 32 consecutive rows: its loads are coalesced, and in pass 2
+// its scored rows (and its other rows) land in consecutive list slots, found
+// from a warp ballot plus a prefix over the warps -- 16-byte list stores
+// that coalesce.  The CTAs exchange their slices' counts through distributed
+// shared memory, so each knows N, the totals and where its slice's rows go:
+// the list holds the scored rows in row order, then all other rows in row
+// order.  Up to kPlanCacheRows rows per CTA, pass 1 keeps each row's
+// classification and every warp's counts in shared memory and pass 2 needs
+// no global load and no barrier; beyond that, pass 2 classifies again, T rows
+// at a time.
 __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
     constexpr int kTiles = kPlanCacheRows / kPlanThreads;
     __shared__ int s_cnt[2][kTiles][kPlanWarps];   // per T-row tile and warp: scored / other rows
     __shared__ int s_sum[3][kPlanWarps];
     __shared__ uint32_t s_status;
+    __shared__ int s_pub[6];    // this slice: scored, other, scored diffusion, scored encoder, non-pad, status
+    __shared__ int s_glob[6];   // scored / other rows of the slices before this one; n_a, n_b, N, status
     pdl_launch_dependents();   // the CE kernel may start its prologue now
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c = int(cluster_ctarank()), C = int(cluster_dims_x());
     if (tid == 0) s_status = 0;
     pdl_wait();                // inputs written by earlier kernels are visible
     __syncthreads();
-    if (layout_bad(P.a) || layout_bad(P.b)) atomicOr(&s_status, DLM_DEV_BAD_LAYOUT);
+    if (layout_bad(P.a, c * kPlanThreads + tid, C * kPlanThreads) ||
+        layout_bad(P.b, c * kPlanThreads + tid, C * kPlanThreads))
+        atomicOr(&s_status, DLM_DEV_BAD_LAYOUT);
 
     const int64_t R = P.a.n_tokens + P.b.n_tokens;
-    const bool cached = R <= kPlanCacheRows;
-    extern __shared__ int2 s_rows[];   // cached: {target, unit} per row, then p of the row's unit
-    float* s_p = reinterpret_cast<float*>(s_rows + (cached ? R : 0));
+    const int64_t per = ((R + C - 1) / C + 31) / 32 * 32;
+    const int64_t lo = min(R, int64_t(c) * per), hi = min(R, lo + per);
+    const int64_t Rc = hi - lo;
+    const bool cached = Rc <= kPlanCacheRows;
+    extern __shared__ int2 s_rows[];   // cached: {target, unit} per row of the slice, then p of the row's unit
+    float* s_p = reinterpret_cast<float*>(s_rows + (cached ? Rc : 0));
 
-    // pass 1: classify and count
+    // pass 1: classify and count (the bound is the same for every thread:
+    // the ballots below need whole warps)
     int na = 0, nb = 0, nonpad = 0;
     bool any_bad = false;
-    // the bound is the same for every thread (the ballots below need whole warps)
-    for (int64_t base = 0; base < R; base += int64_t(kPlanThreads) * kPlanBatch) {
-        const int64_t q0 = base + tid;
+    for (int64_t base = 0; base < Rc; base += int64_t(kPlanThreads) * kPlanBatch) {
+        const int64_t q0 = lo + base + tid;
         int tg[kPlanBatch], u[kPlanBatch];
         float pu[kPlanBatch];
-        classify_batch(P, q0, R, tg, u, pu, any_bad, na, nb, nonpad);
+        classify_batch(P, q0, hi, tg, u, pu, any_bad, na, nb, nonpad);
         if (cached) {
             #pragma unroll
             for (int k = 0; k < kPlanBatch; ++k) {
-                const int64_t q = q0 + int64_t(k) * kPlanThreads;
-                const unsigned bs = __ballot_sync(0xffffffffu, q < R && tg[k] >= 0);
-                const unsigned bv = __ballot_sync(0xffffffffu, q < R);
-                const int t = int((q - tid) / kPlanThreads);
-                if (q - tid < R && lane == 0) {
+                const int64_t r = base + tid + int64_t(k) * kPlanThreads;   // row within the slice
+                const unsigned bs = __ballot_sync(0xffffffffu, r < Rc && tg[k] >= 0);
+                const unsigned bv = __ballot_sync(0xffffffffu, r < Rc);
+                const int t = int((r - tid) / kPlanThreads);
+                if (r - tid < Rc && lane == 0) {
                     s_cnt[0][t][warp] = __popc(bs);
                     s_cnt[1][t][warp] = __popc(bv & ~bs);
                 }
-                if (q < R) {
-                    s_rows[q] = make_int2(tg[k], u[k]);
-                    s_p[q] = pu[k];
+                if (r < Rc) {
+                    s_rows[r] = make_int2(tg[k], u[k]);
+                    s_p[r] = pu[k];
                 }
             }
         }
@@ -271,44 +284,75 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
         if (lane == 0) { s_sum[0][warp] = v0; s_sum[1][warp] = v1; s_sum[2][warp] = v2; }
     }
     __syncthreads();
-    int n_a = 0, n_b = 0, N = 0;
-    #pragma unroll
-    for (int w = 0; w < kPlanWarps; ++w) { n_a += s_sum[0][w]; n_b += s_sum[1][w]; N += s_sum[2][w]; }
+    if (tid == 0) {
+        int la = 0, lb = 0, lnp = 0;
+        for (int w = 0; w < kPlanWarps; ++w) { la += s_sum[0][w]; lb += s_sum[1][w]; lnp += s_sum[2][w]; }
+        s_pub[0] = la + lb;
+        s_pub[1] = int(Rc) - (la + lb);
+        s_pub[2] = la;
+        s_pub[3] = lb;
+        s_pub[4] = lnp;
+        s_pub[5] = int(s_status);
+    }
+    __syncwarp();
+    cluster_sync_all();   // every slice's counts are published
+    if (warp == 0) {
+        int v[6];
+        #pragma unroll
+        for (int j = 0; j < 6; ++j)
+            v[j] = lane < C ? ld_cluster_s32(mapa_shared(smem_addr(&s_pub[j]), uint32_t(lane))) : 0;
+        #pragma unroll
+        for (int j = 0; j < 5; ++j) {
+            // sums over the slices before this CTA's (scored, other) or over all of them
+            int x = (j >= 2 || lane < c) ? v[j] : 0;
+            #pragma unroll
+            for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+            if (lane == 0) s_glob[j] = x;
+        }
+        int st = v[5];
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) st |= __shfl_xor_sync(0xffffffffu, st, o);
+        if (lane == 0) s_glob[5] = st;
+    }
+    __syncwarp();
+    cluster_sync_all();   // all remote reads are done (no CTA leaves before), s_glob is visible
+    const int n_a = s_glob[2], n_b = s_glob[3], N = s_glob[4];
     const int n_scored = n_a + n_b;
     const float w_canvas = n_a > 0 ? 1.0f / float(n_a) : 0.0f;
     const float w_enc = n_b > 0 ? P.lam / float(n_b) : 0.0f;
-    auto weight = [&](int64_t q, int u, float pu) {
+    auto weight = [&](int64_t q, float pu) {
         if (q >= P.a.n_tokens) return w_enc;
         return P.mode == DLM_ABSORBING ? 1.0f / (pu * float(N)) : w_canvas;
     };
 
-    // pass 2: weights and the row list, T rows at a time in row order
-    int64_t base_s = 0, base_u = n_scored;   // next scored / unscored slot
+    // pass 2: weights and this slice's list entries, T rows at a time in row order
+    int64_t base_s = s_glob[0], base_u = int64_t(n_scored) + s_glob[1];   // next scored / other slot
     const unsigned below = (1u << lane) - 1u;
     if (cached) {
-        for (int t = 0; int64_t(t) * kPlanThreads < R; ++t) {
-            const int64_t q = int64_t(t) * kPlanThreads + tid;
-            const bool in = q < R;
-            const int2 c = in ? s_rows[q] : make_int2(-1, 0);
-            const unsigned bs = __ballot_sync(0xffffffffu, in && c.x >= 0);
-            const unsigned bu = __ballot_sync(0xffffffffu, in && c.x < 0);
+        for (int t = 0; int64_t(t) * kPlanThreads < Rc; ++t) {
+            const int64_t r = int64_t(t) * kPlanThreads + tid;
+            const int64_t q = lo + r;
+            const bool in = r < Rc;
+            const int2 cl = in ? s_rows[r] : make_int2(-1, 0);
+            const unsigned bs = __ballot_sync(0xffffffffu, in && cl.x >= 0);
+            const unsigned bu = __ballot_sync(0xffffffffu, in && cl.x < 0);
             int ps, ts, pu, tu;
             warp_prefix(s_cnt[0][t], warp, lane, ps, ts);
             warp_prefix(s_cnt[1][t], warp, lane, pu, tu);
             if (in) {
-                if (c.x >= 0)
+                if (cl.x >= 0)
                     P.list[base_s + ps + __popc(bs & below)] =
-                        make_int4(int(q), c.x, __float_as_int(weight(q, c.y, s_p[q])), c.y);
+                        make_int4(int(q), cl.x, __float_as_int(weight(q, s_p[r])), cl.y);
                 else
-                    P.list[base_u + pu + __popc(bu & below)] = make_int4(int(q), -1, 0, c.y);
+                    P.list[base_u + pu + __popc(bu & below)] = make_int4(int(q), -1, 0, cl.y);
             }
             base_s += ts;
             base_u += tu;
         }
     } else {
-        for (int64_t t0 = 0; t0 < R; t0 += kPlanThreads) {
-            const int64_t q = t0 + tid;
-            const bool in = q < R;
+        for (int64_t t0 = 0; t0 < Rc; t0 += kPlanThreads) {
+            const int64_t q = lo + t0 + tid;
+            const bool in = q < hi;
             int tg = -1, u = 0;
             bool bad;
             if (in) classify(P, q, tg, u, bad);
@@ -323,7 +367,7 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
             if (in) {
                 if (tg >= 0) {
                     const float pv = (q < P.a.n_tokens && P.mode == DLM_ABSORBING) ? __ldg(P.p + u) : 0.f;
-                    P.list[base_s + ps + __popc(bs & below)] = make_int4(int(q), tg, __float_as_int(weight(q, u, pv)), u);
+                    P.list[base_s + ps + __popc(bs & below)] = make_int4(int(q), tg, __float_as_int(weight(q, pv)), u);
                 } else {
                     P.list[base_u + pu + __popc(bu & below)] = make_int4(int(q), -1, 0, u);
                 }
@@ -332,9 +376,8 @@ __global__ void __launch_bounds__(kPlanThreads, 1) k_plan(PlanParams P) {
             base_u += tu;
         }
     }
-    __syncthreads();
-    if (tid == 0) {
-        P.hdr->status = s_status;
+    if (c == 0 && tid == 0) {
+        P.hdr->status = uint32_t(s_glob[5]);
         P.hdr->n_scored = n_scored;
         P.hdr->n_rows = int(R);
         P.hdr->n_nonpad = N;
@@ -910,7 +953,8 @@ dlm_status_t launch_plan(const dlm_layout_t* a, const int32_t* clean, const uint
     pp.hdr = hdr;
     pp.list = list;
     const int64_t R = (a ? a->n_tokens : 0) + (b ? b->n_tokens : 0);
-    const size_t smem = R <= kPlanCacheRows ? size_t(R) * (sizeof(int2) + sizeof(float)) : 0;
+    const int64_t per = ((R + kPlanCluster - 1) / kPlanCluster + 31) / 32 * 32;   // rows per CTA (as the kernel splits)
+    const size_t smem = per <= kPlanCacheRows ? size_t(per) * (sizeof(int2) + sizeof(float)) : 0;
     static std::mutex mu;
     static bool attr[64] = {};
     int dev = 0;
@@ -924,7 +968,25 @@ dlm_status_t launch_plan(const dlm_layout_t* a, const int32_t* clean, const uint
             attr[dev] = true;
         }
     }
-    return launch_pdl(k_plan, dim3(1), dim3(kPlanThreads), smem, s, "k_plan launch", pp);
+    // one cluster of kPlanCluster CTAs, launched with programmatic stream
+    // serialization like the other kernels of the call
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kPlanCluster);
+    cfg.blockDim = dim3(kPlanThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = kPlanCluster;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, k_plan, pp);
+    if (e != cudaSuccess) cudaGetLastError();
+    return cuda_status(e, "k_plan launch");
 }
 
 dlm_status_t launch_reduce(const dlm_layout_t* a, const dlm_layout_t* b, const float* row_loss,

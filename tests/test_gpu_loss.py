@@ -108,15 +108,16 @@ def test_llada_like_full_size():
                       grad_rows=_sample_rows(4096, 4096, seed=seed))
 
 
-@pytest.mark.parametrize("align", [oracle.ALIGNED, oracle.SHIFTED])
-def test_rows_beyond_the_plan_cache(align):
-    """20,000 rows: more rows than the plan keeps in shared memory, so the
-    list is built by the plan's second, re-classifying pass."""
-    spec = di.WORKLOADS["abs_b1_l4096_v126464"].scaled(vocab=4096, mask_id=4095, ids_high=4000, n_units=5,
+@pytest.mark.parametrize("units,align", [(5, oracle.ALIGNED), (5, oracle.SHIFTED), (33, oracle.ALIGNED)])
+def test_many_rows_plan_slices(units, align):
+    """Sequences of 4,000 rows split over the plan's CTAs: 20,000 rows (every
+    CTA keeps its slice in shared memory) and 132,000 rows (more than the
+    eight CTAs keep, so the list comes from the re-classifying pass)."""
+    spec = di.WORKLOADS["abs_b1_l4096_v126464"].scaled(vocab=4096, mask_id=4095, ids_high=4000, n_units=units,
                                                        seq_len=4000, spike=0.0, align=align)
     case = di.make_case(spec, "cuda")
-    run_absorbing(spec, case.logits, case.clean, n_units=5, seq_len=4000, seed=7,
-                  grad_rows=_sample_rows(20000, 4000, seed=7))
+    run_absorbing(spec, case.logits, case.clean, n_units=units, seq_len=4000, seed=7,
+                  grad_rows=_sample_rows(units * 4000, 4000, seed=7))
 
 
 def test_dream_like_shifted_mid_size_elementwise():
