@@ -92,8 +92,14 @@ WORKLOADS = {
         h_std=1.0, w_std=0.02, data_seed=5,
         description="packed documents (lengths geometric, mean 296, 16..4096) through a fused "
                     "lm_head, T=16384 D=4096 V=126464"),
-    # a smaller case of the same kernels, sized for detailed profiling (W is
-    # still larger than L2)
+    # smaller cases of the same kernels, sized for detailed profiling (the
+    # inputs are still larger than L2)
+    "unif_b1_p256_c512_v262144": Spec(
+        "unif_b1_p256_c512_v262144", "loss", UNIFORM, ALIGNED, vocab=262144, mask_id=-1,
+        ids_high=262143, n_units=1, seq_len=512, prefix=256, std=3.0, enc_ar_weight=1.0,
+        data_seed=6,
+        description="DiffusionGemma-like uniform-token noise, B=1, prefix 256 + canvas 512, "
+                    "V=262144 (every row scored; 0.67 GB of logits)"),
     "lin_t4096_d4096_v32768": Spec(
         "lin_t4096_d4096_v32768", "linear", ABSORBING, ALIGNED, vocab=32768,
         mask_id=32767, ids_high=32000, n_tokens_packed=4096, d_model=4096,
