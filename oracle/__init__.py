@@ -46,6 +46,10 @@ from . import build as _build
 
 ABSORBING, UNIFORM = 0, 1
 ALIGNED, SHIFTED = 0, 1
+# uniform-noise objective options ([Gemma] "Rhine objectives", page
+# "Native diffusion language-model training", Objective and recurrence options)
+NO_TIME_WEIGHT, INV_ONE_MINUS_T = 0, 1
+TOKEN_MEAN, EXAMPLE_MEAN = 0, 1
 
 _lib = None
 
@@ -166,13 +170,23 @@ class RowPlan:
 
 
 def plan_diffusion(layout: Layout, clean: np.ndarray, corrupted: Optional[np.ndarray],
-                   p: Optional[np.ndarray], mode: int, align: int) -> RowPlan:
+                   p: Optional[np.ndarray], mode: int, align: int,
+                   time_weighting: int = NO_TIME_WEIGHT, weight_clip: float = 0.0,
+                   reduction: int = TOKEN_MEAN) -> RowPlan:
     """Diffusion term.  Row i scores token j = i (aligned) or j = i+1 of the
     same unit (shifted; [Axolotl] model table: Dream's logit i predicts token
     i+1).  The target must be a non-pad token; absorbing noise additionally
     requires it to be corrupted ([LLaDA]: CE on masked tokens).
       absorbing: weight = 1 / (p_unit * N), N = non-pad tokens in the call.
-      uniform:   weight = 1 / (number of scored canvas rows)  (mean, [Gemma]).
+      uniform:   weight = f_unit / (number of scored canvas rows)  (mean, [Gemma]),
+                 or, with reduction EXAMPLE_MEAN, f_unit / (B' * n_unit): the
+                 mean over each example's scored rows, then over the B'
+                 examples that have any ([Axolotl] Objective options:
+                 objective_reduction example_mean).
+                 f_unit = 1, or with time weighting INV_ONE_MINUS_T
+                 min(1 / (1 - t_unit), clip) (no cap when clip <= 0), t = p for
+                 uniform noise ([Axolotl]: Rhine objectives, rhine_weight_clip
+                 caps the 1 / (1 - t) weights).
     """
     n = layout.n_tokens
     unit = layout.unit_of_token()
@@ -195,9 +209,21 @@ def plan_diffusion(layout: Layout, clean: np.ndarray, corrupted: Optional[np.nda
         if N > 0:
             weight[ok] = 1.0 / (p[unit[ok]].astype(np.float64) * N)
     else:
-        cnt = int(ok.sum())
-        if cnt > 0:
-            weight[ok] = 1.0 / cnt
+        f = np.ones(n, np.float64)
+        if time_weighting == INV_ONE_MINUS_T:
+            fu = 1.0 / (1.0 - p.astype(np.float64))
+            if weight_clip > 0:
+                fu = np.minimum(fu, float(weight_clip))
+            f = fu[unit]
+        if reduction == TOKEN_MEAN:
+            cnt = int(ok.sum())
+            if cnt > 0:
+                weight[ok] = f[ok] / cnt
+        else:
+            n_u = np.bincount(unit[ok], minlength=layout.n_units)
+            b_eff = int((n_u > 0).sum())
+            if b_eff > 0:
+                weight[ok] = f[ok] / (b_eff * n_u[unit[ok]])
     return RowPlan(target, unit, weight)
 
 
@@ -327,9 +353,13 @@ def loss_absorbing(layout: Layout, logits: np.ndarray, vocab: int, clean: np.nda
 
 def loss_uniform(canvas: Layout, logits: np.ndarray, canvas_clean: np.ndarray,
                  encoder: Layout, enc_logits: np.ndarray, enc_clean: np.ndarray,
-                 vocab: int, lam: float, align: int = ALIGNED):
-    """[Gemma] total = canvas CE (mean) + lam * encoder AR CE (mean)."""
-    pc = plan_diffusion(canvas, canvas_clean, None, None, UNIFORM, align)
+                 vocab: int, lam: float, align: int = ALIGNED, p: Optional[np.ndarray] = None,
+                 time_weighting: int = NO_TIME_WEIGHT, weight_clip: float = 0.0,
+                 reduction: int = TOKEN_MEAN):
+    """[Gemma] total = canvas CE (mean; optionally time-weighted and/or the
+    mean of per-example means, see plan_diffusion) + lam * encoder AR CE
+    (mean over next-token pairs)."""
+    pc = plan_diffusion(canvas, canvas_clean, None, p, UNIFORM, align, time_weighting, weight_clip, reduction)
     pe = plan_encoder(encoder, enc_clean, lam)
     tc = term(logits, vocab, pc)
     te = term(enc_logits, vocab, pe)

@@ -272,6 +272,85 @@ def test_encoder_term_is_plain_causal_ce():
 
 
 # --------------------------------------------------------------------------
+# uniform noise: 1/(1-t) time weighting with a cap, per-example mean
+# --------------------------------------------------------------------------
+def _canvas_case(seed, B=3, C=6, V=37, pads=None):
+    rng = np.random.default_rng(seed)
+    pad = None
+    if pads is not None:
+        pad = np.zeros(B * C, np.uint8)
+        for b, n in enumerate(pads):
+            pad[b * C + n:(b + 1) * C] = 1
+    canvas = oracle.Layout(B, C, None, pad)
+    clean = rng.integers(0, V, B * C).astype(np.int32)
+    x = rng.standard_normal((B * C, V)) * 2
+    t = np.array([0.2, 0.55, 0.9][:B], np.float32)
+    return canvas, clean, x, t, V
+
+
+def _canvas_loss(canvas, clean, x, t, V, tw, clip, red):
+    plan = oracle.plan_diffusion(canvas, clean, None, t, oracle.UNIFORM, oracle.ALIGNED, tw, clip, red)
+    tr = oracle.term(x, V, plan)
+    return oracle.reduce_units(canvas.n_units, tr)[0], tr
+
+
+def test_rhine_cap_one_is_the_plain_mean():
+    """1/(1-t) >= 1, so a cap of 1 leaves every weight at 1: the plain token
+    mean exactly (a cap applied the wrong way would not)."""
+    case = _canvas_case(21)
+    plain, _ = _canvas_loss(*case, oracle.NO_TIME_WEIGHT, 0.0, oracle.TOKEN_MEAN)
+    capped, _ = _canvas_loss(*case, oracle.INV_ONE_MINUS_T, 1.0, oracle.TOKEN_MEAN)
+    assert abs(capped - plain) < 1e-12
+    canvas, clean, x, t, V = case
+    assert abs(plain - torch_ce(x, clean).mean()) < 1e-12
+
+
+def test_rhine_single_example_scales_by_inverse_one_minus_t():
+    canvas, clean, x, t, V = _canvas_case(22, B=1)
+    plain, _ = _canvas_loss(canvas, clean, x, t, V, oracle.NO_TIME_WEIGHT, 0.0, oracle.TOKEN_MEAN)
+    for red in (oracle.TOKEN_MEAN, oracle.EXAMPLE_MEAN):
+        w, _ = _canvas_loss(canvas, clean, x, t, V, oracle.INV_ONE_MINUS_T, 0.0, red)
+        assert abs(w - plain / (1.0 - float(t[0]))) < 1e-12 * abs(w)
+    # a cap below 1/(1-t) = 1.25 takes over
+    w, _ = _canvas_loss(canvas, clean, x, t, V, oracle.INV_ONE_MINUS_T, 1.1, oracle.TOKEN_MEAN)
+    assert abs(w - plain * 1.1) < 1e-12 * abs(w)
+
+
+def test_example_mean_equal_lengths_is_token_mean_and_unequal_is_not():
+    case = _canvas_case(23)
+    tok, _ = _canvas_loss(*case, oracle.NO_TIME_WEIGHT, 0.0, oracle.TOKEN_MEAN)
+    ex, _ = _canvas_loss(*case, oracle.NO_TIME_WEIGHT, 0.0, oracle.EXAMPLE_MEAN)
+    assert abs(tok - ex) < 1e-12
+    # examples of 6, 2 and 4 canvas tokens: the mean of the three per-example
+    # means, each a textbook CE mean over that example's rows
+    canvas, clean, x, t, V = _canvas_case(23, pads=(6, 2, 4))
+    ex, tr = _canvas_loss(canvas, clean, x, t, V, oracle.NO_TIME_WEIGHT, 0.0, oracle.EXAMPLE_MEAN)
+    ce = torch_ce(x, clean).reshape(3, 6)
+    want = (ce[0, :6].mean() + ce[1, :2].mean() + ce[2, :4].mean()) / 3
+    assert abs(ex - want) < 1e-12
+    tok, _ = _canvas_loss(canvas, clean, x, t, V, oracle.NO_TIME_WEIGHT, 0.0, oracle.TOKEN_MEAN)
+    assert abs(tok - (ce[0, :6].sum() + ce[1, :2].sum() + ce[2, :4].sum()) / 12) < 1e-12
+    assert abs(tok - ex) > 1e-3
+
+
+def test_rhine_example_mean_on_zero_logits_closed_form():
+    """All-zero logits: every CE is ln V, so the loss is ln V times the mean
+    over examples of min(1/(1-t), cap)."""
+    canvas, clean, x, t, V = _canvas_case(24, pads=(6, 3, 1))
+    x = np.zeros_like(x)
+    loss, _ = _canvas_loss(canvas, clean, x, t, V, oracle.INV_ONE_MINUS_T, 4.0, oracle.EXAMPLE_MEAN)
+    f = [min(1.0 / (1.0 - float(tt)), 4.0) for tt in t]     # 1.25, 2.22.., 10 -> 4
+    assert abs(loss - math.log(V) * sum(f) / 3) < 1e-12
+
+
+def test_example_mean_skips_examples_without_scored_rows():
+    canvas, clean, x, t, V = _canvas_case(25, pads=(6, 0, 3))
+    ex, _ = _canvas_loss(canvas, clean, x, t, V, oracle.NO_TIME_WEIGHT, 0.0, oracle.EXAMPLE_MEAN)
+    ce = torch_ce(x, clean).reshape(3, 6)
+    assert abs(ex - (ce[0].mean() + ce[2, :3].mean()) / 2) < 1e-12
+
+
+# --------------------------------------------------------------------------
 # packed documents
 # --------------------------------------------------------------------------
 def test_packing_invariance_of_unit_sums():
