@@ -28,6 +28,8 @@ LIB_PATH = os.path.join(HERE, "libdlm.so")
 
 ABSORBING, UNIFORM = 0, 1
 ALIGNED, SHIFTED = 0, 1
+TIME_WEIGHT_NONE, TIME_WEIGHT_INV_ONE_MINUS_T = 0, 1
+REDUCE_TOKEN_MEAN, REDUCE_EXAMPLE_MEAN = 0, 1
 
 DEV_BAD_TOKEN_ID = 0x1
 DEV_BAD_LAYOUT = 0x2
@@ -38,7 +40,7 @@ STATUS = {0: "DLM_OK", 1: "DLM_ERR_INVALID_ARGUMENT", 2: "DLM_ERR_UNSUPPORTED",
 
 # every symbol include/dlm.h declares
 EXPORTS = ("dlm_status_string", "dlm_last_cuda_error", "dlm_version", "dlm_sample_t", "dlm_corrupt",
-           "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_loss_fwd_bwd_static",
+           "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_loss_fwd_bwd_ex", "dlm_loss_fwd_bwd_static",
            "dlm_linear_loss_workspace_size",
            "dlm_linear_loss_fwd_bwd", "dlm_get_device_status", "dlm_selftest_bounded_wait")
 
@@ -47,6 +49,15 @@ class DlmError(RuntimeError):
     def __init__(self, code: int, where: str, detail: str = ""):
         super().__init__(f"{where}: {STATUS.get(code, code)}" + (f" [{detail}]" if detail else ""))
         self.code = code
+
+
+class LossOptions(ctypes.Structure):
+    """dlm_loss_options_t: uniform-noise objective options."""
+    _fields_ = [("struct_size", ctypes.c_uint32), ("time_weighting", ctypes.c_int32),
+                ("weight_clip", ctypes.c_float), ("reduction", ctypes.c_int32)]
+
+    def __init__(self, time_weighting=TIME_WEIGHT_NONE, weight_clip=0.0, reduction=REDUCE_TOKEN_MEAN):
+        super().__init__(ctypes.sizeof(LossOptions), time_weighting, weight_clip, reduction)
 
 
 class Layout(ctypes.Structure):
@@ -105,6 +116,9 @@ def lib():
     L.dlm_loss_fwd_bwd.restype = ctypes.c_int
     L.dlm_loss_fwd_bwd.argtypes = [lp, vp, i64, i32, vp, vp, vp, i32, i32, lp, vp, i64, vp, f32,
                                    f32, vp, vp, vp, vp, vp, sz, vp]
+    L.dlm_loss_fwd_bwd_ex.restype = ctypes.c_int
+    L.dlm_loss_fwd_bwd_ex.argtypes = [lp, vp, i64, i32, vp, vp, vp, i32, i32, lp, vp, i64, vp, f32,
+                                      f32, ctypes.POINTER(LossOptions), vp, vp, vp, vp, vp, sz, vp]
     L.dlm_loss_fwd_bwd_static.restype = ctypes.c_int
     L.dlm_loss_fwd_bwd_static.argtypes = [lp, vp, i64, i32, vp, vp, vp, i32, i32, lp, vp, i64, vp, f32,
                                           f32, vp, vp, vp, vp, vp]
@@ -194,7 +208,8 @@ def loss_fwd_bwd(layout: Layout, logits: torch.Tensor, vocab: int, clean_ids: to
                  mode: int = ABSORBING, align: int = ALIGNED,
                  enc_layout: Optional[Layout] = None, enc_logits: Optional[torch.Tensor] = None,
                  enc_ids: Optional[torch.Tensor] = None, enc_ar_weight: float = 1.0,
-                 grad_scale: float = 1.0, out: Optional[LossOut] = None) -> LossOut:
+                 grad_scale: float = 1.0, out: Optional[LossOut] = None,
+                 options: Optional[LossOptions] = None) -> LossOut:
     """Weighted CE forward + backward (see dlm_loss_fwd_bwd).  logits: bf16
     [rows, ld] (2-D, row stride ld >= vocab).  Reuses the buffers of `out`
     when given (no allocation)."""
@@ -217,12 +232,20 @@ def loss_fwd_bwd(layout: Layout, logits: torch.Tensor, vocab: int, clean_ids: to
                       torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
                       torch.empty_like(logits),
                       torch.empty_like(enc_logits) if enc_logits is not None else None, ws)
-    _ok(lib().dlm_loss_fwd_bwd(
-        ctypes.byref(layout), _ptr(logits), ld, vocab, _ptr(clean_ids), _ptr(corrupted), _ptr(p),
-        mode, align, ctypes.byref(enc_layout) if enc_layout is not None else None,
-        _ptr(enc_logits), enc_ld, _ptr(enc_ids), enc_ar_weight, grad_scale, _ptr(out.loss),
-        _ptr(out.unit_loss), _ptr(out.dlogits), _ptr(out.enc_dlogits), _ptr(out.workspace),
-        out.workspace.numel(), _stream()), "dlm_loss_fwd_bwd")
+    if options is None:
+        _ok(lib().dlm_loss_fwd_bwd(
+            ctypes.byref(layout), _ptr(logits), ld, vocab, _ptr(clean_ids), _ptr(corrupted), _ptr(p),
+            mode, align, ctypes.byref(enc_layout) if enc_layout is not None else None,
+            _ptr(enc_logits), enc_ld, _ptr(enc_ids), enc_ar_weight, grad_scale, _ptr(out.loss),
+            _ptr(out.unit_loss), _ptr(out.dlogits), _ptr(out.enc_dlogits), _ptr(out.workspace),
+            out.workspace.numel(), _stream()), "dlm_loss_fwd_bwd")
+    else:
+        _ok(lib().dlm_loss_fwd_bwd_ex(
+            ctypes.byref(layout), _ptr(logits), ld, vocab, _ptr(clean_ids), _ptr(corrupted), _ptr(p),
+            mode, align, ctypes.byref(enc_layout) if enc_layout is not None else None,
+            _ptr(enc_logits), enc_ld, _ptr(enc_ids), enc_ar_weight, grad_scale, ctypes.byref(options),
+            _ptr(out.loss), _ptr(out.unit_loss), _ptr(out.dlogits), _ptr(out.enc_dlogits),
+            _ptr(out.workspace), out.workspace.numel(), _stream()), "dlm_loss_fwd_bwd_ex")
     return out
 
 

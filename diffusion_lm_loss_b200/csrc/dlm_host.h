@@ -84,13 +84,23 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) <= kWsAlign, "header");
 
-// Row plan (one CTA): classifies every row of `a` (and of the encoder
-// layout `b`, rows after a's), writes list[] = {row, target, weight bits,
-// unit} with the scored rows first in row order, and fills *hdr.
+// Objective options of the uniform-noise canvas term (see
+// dlm_loss_fwd_bwd_ex); unit_cnt: [n_units] int32 scratch for the
+// per-example mean.
+struct ObjOpts {
+    int time_weighting = DLM_TIME_WEIGHT_NONE;
+    float weight_clip = 0.f;
+    int reduction = DLM_REDUCE_TOKEN_MEAN;
+    int32_t* unit_cnt = nullptr;
+};
+
+// Row plan (one cluster of CTAs): classifies every row of `a` (and of the
+// encoder layout `b`, rows after a's), writes list[] = {row, target, weight
+// bits, unit} with the scored rows first in row order, and fills *hdr.
 dlm_status_t launch_plan(const dlm_layout_t* a, const int32_t* clean, const uint8_t* corrupted,
                          const float* p, int mode, int align, const dlm_layout_t* b,
                          const int32_t* ids_b, float lam, int vocab, WsHeader* hdr, int4* list,
-                         cudaStream_t s);
+                         cudaStream_t s, const ObjOpts& opts = ObjOpts());
 
 // Per-unit sums of row_loss over a's rows (and b's rows, indexed after a's)
 // and their total, in a fixed order.  Uses hdr->ticket (zeroed by the plan).

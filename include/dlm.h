@@ -10,7 +10,8 @@
  *   dlm_corrupt              seeded corruption of the clean ids
  *   dlm_loss_fwd_bwd         inverse-time weighted CE over the vocabulary at
  *                            the corrupted positions, forward + backward, from
- *                            materialised bf16 logits
+ *                            materialised bf16 logits (dlm_loss_fwd_bwd_ex:
+ *                            with the uniform-noise objective options)
  *   dlm_linear_loss_fwd_bwd  the same loss from hidden states and a linear
  *                            output head, logits never materialised
  *
@@ -195,6 +196,47 @@ DLM_API dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t *layout, const uint16_t
                               float grad_scale, float *loss, float *unit_loss,
                               uint16_t *dlogits, uint16_t *enc_dlogits,
                               void *workspace, size_t workspace_bytes, dlm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * dlm_loss_fwd_bwd_ex -- dlm_loss_fwd_bwd with objective options for uniform
+ * noise ("Native diffusion language-model training", Objective and
+ * recurrence options: DiffusionGemma's Rhine objectives use time weighting
+ * inv_one_minus_t with objective_reduction example_mean; rhine_weight_clip
+ * caps the 1 / (1 - t) weights).
+ *
+ * For mode == DLM_UNIFORM the weight of a scored canvas row of unit u becomes
+ *   w = f_u / (number of scored canvas rows)           DLM_REDUCE_TOKEN_MEAN
+ *   w = f_u / (B' * n_u)                               DLM_REDUCE_EXAMPLE_MEAN
+ * with n_u the scored canvas rows of unit u, B' the units that have any, and
+ *   f_u = 1                                            DLM_TIME_WEIGHT_NONE
+ *   f_u = min(1 / (1 - t_u), weight_clip)              DLM_TIME_WEIGHT_INV_ONE_MINUS_T
+ * (no cap when weight_clip <= 0; t_u = p[u], the uniform-noise time from
+ * dlm_sample_t, which p must then hold).  The encoder AR term is unchanged.
+ * options == NULL, or both fields at their defaults, is dlm_loss_fwd_bwd.
+ * Non-default options with absorbing noise, or time weighting without p,
+ * return DLM_ERR_INVALID_ARGUMENT; so does options->struct_size <
+ * sizeof(dlm_loss_options_t).
+ * ---------------------------------------------------------------------- */
+#define DLM_TIME_WEIGHT_NONE 0
+#define DLM_TIME_WEIGHT_INV_ONE_MINUS_T 1
+#define DLM_REDUCE_TOKEN_MEAN 0
+#define DLM_REDUCE_EXAMPLE_MEAN 1
+
+typedef struct {
+    uint32_t struct_size;      /* sizeof(dlm_loss_options_t) */
+    int32_t time_weighting;    /* DLM_TIME_WEIGHT_* */
+    float weight_clip;         /* cap of 1 / (1 - t); <= 0: none */
+    int32_t reduction;         /* DLM_REDUCE_* */
+} dlm_loss_options_t;
+
+DLM_API dlm_status_t dlm_loss_fwd_bwd_ex(const dlm_layout_t *layout, const uint16_t *logits, int64_t ld,
+                                 int32_t vocab, const int32_t *clean_ids, const uint8_t *corrupted,
+                                 const float *p, int32_t mode, int32_t align,
+                                 const dlm_layout_t *enc_layout, const uint16_t *enc_logits,
+                                 int64_t enc_ld, const int32_t *enc_ids, float enc_ar_weight,
+                                 float grad_scale, const dlm_loss_options_t *options, float *loss,
+                                 float *unit_loss, uint16_t *dlogits, uint16_t *enc_dlogits,
+                                 void *workspace, size_t workspace_bytes, dlm_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * dlm_loss_fwd_bwd_static -- dlm_loss_fwd_bwd without a caller workspace.

@@ -74,6 +74,23 @@ def test_host_side_rejections(L):
     assert L.dlm_loss_fwd_bwd(*a) == 3                                    # workspace too small
     a = list(args); a[19] = 100
     assert L.dlm_loss_fwd_bwd(*a) == 1                                    # misaligned workspace
+    # objective options: only for uniform noise, known values, a full struct,
+    # time weighting needs p
+    def ex(opts, mode=1, p=16):
+        a = list(args)
+        a[6] = p
+        a[7] = mode
+        a.insert(15, ctypes.byref(opts) if opts is not None else None)
+        return L.dlm_loss_fwd_bwd_ex(*a)
+    assert ex(dlm.LossOptions(dlm.TIME_WEIGHT_INV_ONE_MINUS_T, 2.0), mode=0) == 1   # absorbing
+    assert ex(dlm.LossOptions(reduction=dlm.REDUCE_EXAMPLE_MEAN), mode=0) == 1
+    assert ex(dlm.LossOptions(time_weighting=7)) == 1
+    assert ex(dlm.LossOptions(reduction=5)) == 1
+    short = dlm.LossOptions(dlm.TIME_WEIGHT_INV_ONE_MINUS_T)
+    short.struct_size = 8
+    assert ex(short) == 1
+    assert ex(dlm.LossOptions(dlm.TIME_WEIGHT_INV_ONE_MINUS_T), p=None) == 1          # no p
+    assert ex(dlm.LossOptions(weight_clip=float("nan"))) == 1
     # bounded-wait self-test: no status word, zero or over-long limit
     assert L.dlm_selftest_bounded_wait(10, None, None) == 1
     assert L.dlm_selftest_bounded_wait(0, 16, None) == 1

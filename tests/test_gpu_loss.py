@@ -279,32 +279,39 @@ def test_bitwise_reproducible():
 # uniform noise + encoder AR term
 # --------------------------------------------------------------------------
 def run_uniform(spec, case, *, seed=0, grad_rows=None, enc_grad_rows=None, lam=None,
-                align=oracle.ALIGNED, grad_scale=1.0):
+                align=oracle.ALIGNED, grad_scale=1.0, opts=None, canvas_pad=None):
+    """opts: (time weighting, cap, reduction) for dlm_loss_fwd_bwd_ex;
+    canvas_pad: uint8 [B*C] pad mask of the canvas (examples of unequal
+    length)."""
     dev = torch.device("cuda")
     B, C, P, V = spec.n_units, spec.seq_len, spec.prefix, spec.vocab
     lam = spec.enc_ar_weight if lam is None else lam
-    lay = dlm.make_layout(B, C)
+    pad_d = torch.from_numpy(canvas_pad).to(dev) if canvas_pad is not None else None
+    lay = dlm.make_layout(B, C, None, pad_d)
     enc_lay = dlm.make_layout(B, P + C)
     clean = case.clean.to(dev)
     enc_clean = case.enc_clean.to(dev)
     t, p = dlm.sample_t(seed, B, oracle.UNIFORM, spec.eps)
     noisy, corr = dlm.corrupt(lay, clean, p, oracle.UNIFORM, -1, V, seed)
+    options = dlm.LossOptions(*opts) if opts is not None else None
     out = dlm.loss_fwd_bwd(lay, case.logits.to(dev), V, clean, corr, p, oracle.UNIFORM, align,
                            enc_layout=enc_lay, enc_logits=case.enc_logits.to(dev),
-                           enc_ids=enc_clean, enc_ar_weight=lam, grad_scale=grad_scale)
+                           enc_ids=enc_clean, enc_ar_weight=lam, grad_scale=grad_scale, options=options)
     torch.cuda.synchronize()
     assert out.device_status() == 0
     # oracle
     _, p_o = oracle.sample_t(seed, B, oracle.UNIFORM, spec.eps)
     assert np.array_equal(p.cpu().numpy().view(np.uint32), p_o.view(np.uint32))
-    lay_o = oracle.Layout(B, C, None, None)
+    lay_o = oracle.Layout(B, C, None, canvas_pad)
     noisy_o, corr_o = oracle.corrupt(lay_o, case.clean.cpu().numpy(), p_o, oracle.UNIFORM, -1, V, seed)
     assert np.array_equal(corr.cpu().numpy(), corr_o)
     assert np.array_equal(noisy.cpu().numpy(), noisy_o)
     xc, xe = _bits(case.logits), _bits(case.enc_logits)
+    tw, clip, red = opts if opts is not None else (oracle.NO_TIME_WEIGHT, 0.0, oracle.TOKEN_MEAN)
     loss_o, unit_o, tc, te = oracle.loss_uniform(lay_o, xc, case.clean.cpu().numpy(),
                                                  oracle.Layout(B, P + C, None, None), xe,
-                                                 case.enc_clean.cpu().numpy(), V, lam, align)
+                                                 case.enc_clean.cpu().numpy(), V, lam, align, p_o,
+                                                 tw, clip, red)
     assert_loss_close(float(out.loss.item()), loss_o)
     assert_units_close(out.unit_loss.cpu().numpy()[:B], unit_o, loss_o)
     rows = np.arange(B * C) if grad_rows is None else np.asarray(grad_rows)
@@ -322,6 +329,32 @@ def test_gemma_like_uniform_mid_size_elementwise():
     run_uniform(spec, case, seed=0)
     run_uniform(spec, case, seed=1, lam=0.0)
     run_uniform(spec, case, seed=2, lam=0.3, align=oracle.SHIFTED, grad_scale=2.0)
+
+
+def _canvas_pad(B, C, lengths):
+    pad = np.zeros(B * C, np.uint8)
+    for b, n in enumerate(lengths):
+        pad[b * C + n:(b + 1) * C] = 1
+    return pad
+
+
+@pytest.mark.parametrize("opts", [(oracle.INV_ONE_MINUS_T, 3.0, oracle.EXAMPLE_MEAN),
+                                  (oracle.INV_ONE_MINUS_T, 0.0, oracle.TOKEN_MEAN),
+                                  (oracle.NO_TIME_WEIGHT, 0.0, oracle.EXAMPLE_MEAN)])
+def test_gemma_like_rhine_objective_options(opts):
+    """1/(1-t) time weighting with and without a cap, and the mean of
+    per-example canvas means, on examples of 32, 20 and 7 canvas tokens."""
+    spec = di.WORKLOADS["unif_b4_p512_c1024_v262144"].scaled(n_units=3, prefix=8, seq_len=32)
+    case = di.make_case(spec, "cuda")
+    run_uniform(spec, case, seed=4, opts=opts, canvas_pad=_canvas_pad(3, 32, (32, 20, 7)))
+
+
+def test_example_mean_skips_an_example_without_canvas_rows_general_path():
+    spec = di.WORKLOADS["unif_b4_p512_c1024_v262144"].scaled(n_units=3, prefix=4, seq_len=16, vocab=1000,
+                                                             ids_high=999)
+    case = di.make_case(spec, "cuda")
+    run_uniform(spec, case, seed=5, opts=(oracle.INV_ONE_MINUS_T, 2.0, oracle.EXAMPLE_MEAN),
+                canvas_pad=_canvas_pad(3, 16, (16, 0, 5)), lam=0.5)
 
 
 def test_gemma_like_uniform_small_vocab_general_path():
