@@ -192,6 +192,13 @@ def run_ours(args):
     lay = dlm.make_layout(B, spec.seq_len)
     enc_lay = dlm.make_layout(B, spec.prefix + spec.seq_len) if uniform else None
     out = None
+    # uniform noise, --objective rhine: DiffusionGemma's Rhine objectives --
+    # 1/(1-t) time weighting capped at 10 (the pages give no default cap) and
+    # the per-example mean
+    if args.objective == "rhine" and not uniform:
+        raise SystemExit("--objective rhine applies to uniform-noise workloads")
+    options = (dlm.LossOptions(dlm.TIME_WEIGHT_INV_ONE_MINUS_T, 10.0, dlm.REDUCE_EXAMPLE_MEAN)
+               if args.objective == "rhine" else None)
 
     def step(seed, logits, clean, enc_logits=None, enc_clean=None, ev=None):
         nonlocal out
@@ -201,7 +208,7 @@ def run_ours(args):
             ev[0].record()
         out = dlm.loss_fwd_bwd(lay, logits, V, clean, corr, p, mode, align,
                                enc_layout=enc_lay, enc_logits=enc_logits, enc_ids=enc_clean,
-                               enc_ar_weight=spec.enc_ar_weight, out=out)
+                               enc_ar_weight=spec.enc_ar_weight, out=out, options=options)
         if ev is not None:
             ev[1].record()
         return corr
@@ -332,7 +339,9 @@ def run_ours(args):
         "config": {"workload": spec.key, "description": spec.description, "global_batch": B * world,
                    "seq_len": spec.seq_len, "vocab": V, "parallelism": f"replicas{world}",
                    "l2": "inputs larger than L2 (logits %.2f GB per replica)" % (case.logits.numel() * 2 / 1e9),
-                   "scored_tokens": scored_all, "seeds": "t/corruption seed 1000+step"},
+                   "scored_tokens": scored_all, "seeds": "t/corruption seed 1000+step",
+                   "objective": ("rhine: 1/(1-t) capped at 10, per-example mean" if options is not None
+                                 else "plain")},
         "roofline": roof, "cpu_baseline": cpu, "clocks": clk, "e2e": e2e,
         "gpu_launches": 5 * K,
     }
@@ -536,6 +545,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--objective", choices=["plain", "rhine"], default="plain",
+                    help="uniform-noise workloads: plain canvas mean, or the Rhine objective options")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -508,9 +508,9 @@ struct StreamShape {
     static constexpr int kConsumers = WARPS * 32;
     static constexpr int kThreads = kConsumers + 32;
     static constexpr int kStages = STAGES;
-    // bf16 elements per ring stage: 16 KB, or 24 KB for the 24-warp shape
-    // (a whole number of 16-byte vectors per consumer thread)
-    static constexpr int kChunkE = WARPS == 24 ? 12288 : kChunk;
+    // bf16 elements per ring stage: 16 KB, or two 16-byte vectors per
+    // consumer thread for the wide shapes (24 warps: 24 KB)
+    static constexpr int kChunkE = WARPS >= 24 ? WARPS * 512 : kChunk;
     static constexpr int kVec = kChunkE / 8 / kConsumers;   // 16-byte vectors per thread per chunk
     static_assert(kVec * 8 * kConsumers == kChunkE, "chunk split");
 };
@@ -1127,7 +1127,8 @@ static dlm_status_t loss_fwd_bwd(const dlm_layout_t* layout, const uint16_t* log
     const bool two_per_sm = double(sms) * 2.0 * 2.0 * double(vocab) <= kL2RowBudget;
     // one CTA per SM: 24 consumer warps, 24 KB chunks, 8 stages (measured
     // against 16 warps with 16 KB chunks and 12 stages: 3-5% faster on the
-    // V = 152k-262k workloads, where the consumers are latency-bound)
+    // V = 152k-262k workloads, where the consumers are latency-bound; 28
+    // warps with 28 KB chunks and 7 stages: 1-2% slower again)
 #ifndef DLM_CE_WIDE_WARPS
 #define DLM_CE_WIDE_WARPS 24
 #endif
