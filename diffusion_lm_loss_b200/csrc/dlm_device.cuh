@@ -192,15 +192,6 @@ __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, u
     }
 }
 
-// Bulk copy global -> this CTA's shared memory, completion on `bar`
-// (tx bytes).  dst, src 16-byte aligned; bytes a multiple of 16.  No
-// multicast.
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
-}
-
 __device__ __forceinline__ uint32_t cluster_ctarank() {
     uint32_t r;
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
@@ -230,15 +221,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
-}
-
-// 16-byte store into a peer CTA's shared memory that completes tx bytes on
-// the peer's mbarrier.
-__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, float a, float b, float c, float d,
-                                            uint32_t remote_bar) {
-    asm volatile(
-        "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
-        :: "r"(remote_addr), "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar) : "memory");
 }
 
 // Programmatic dependent launch: a kernel launched with the programmatic
