@@ -432,9 +432,11 @@ def run_linear(args, spec, dev, rank, world):
            "dtype": "bf16", "data": "synthetic",
            "config": {"workload": spec.key, "description": spec.description, "tokens": T, "d_model": D,
                       "vocab": V, "documents": case.n_units, "parallelism": f"replicas{world}",
-                      "scored_tokens": scored_all, "l2": "inputs larger than L2 (W 1.04 GB)"},
+                      "scored_tokens": scored_all, "l2": "inputs larger than L2 (W %.2f GB)" % (V * D * 2 / 1e9)},
            "roofline": roof, "cpu_baseline": None, "clocks": clk, "e2e": None,
-           "gpu_launches": None}
+           # per step: time draw, corruption, plan, gather, forward GEMM, lse,
+           # dZ + dH + dW per 16,384-column vocabulary chunk, scatter, reduce
+           "gpu_launches": K * (6 + 3 * ((V + 16383) // 16384) + 2)}
     print(json.dumps(res), flush=True)
 
 
