@@ -8,7 +8,7 @@
 // Finetuning notes (canvas CE + weight * encoder causal AR CE).
 //
 // Three launches per call, all on the caller's stream:
-//   1. k_plan     one CTA: classifies every logits row (scored or not, its
+//   1. k_plan     one cluster of 8 CTAs: classifies every logits row (scored or not, its
 //                 target, unit and weight), counts N, and writes a row list
 //                 with the scored rows first; the CE kernel's CTAs take the
 //                 list's rows by ticket.

@@ -8,19 +8,22 @@
 //
 // With H_M = the M masked rows of H (gathered), W the [V, D] head:
 //   forward   Z = H_M W^T, tile by tile; the epilogue reads each 128x256
-//             accumulator tile out of tensor memory and keeps only per-row
+//             accumulator half-tile out of tensor memory and keeps only per-row
 //             (max, sum exp) partials and the target logit -> lse per row.
 //   backward  per vocabulary chunk of kVc columns (a bounded buffer, never a
 //             [M, V] tensor): Z_c recomputed, dZ_c = w (softmax - onehot) in
 //             bf16; dH_M += dZ_c W_c; dW_c = dZ_c^T H_M.
 // Executed flops 8 M D V (the recompute adds 2 M D V to the 6 M D V the
-// method needs); every GEMM is the same warp-specialized persistent kernel:
-//   warp 0   TMA producer (one thread), 4-stage ring of 128x64 A + 256x64 B
-//   warp 1   MMA issuer (one thread), 128x256x16 bf16 MMAs, two 256-column
-//            accumulators in tensor memory (epilogue of tile i overlaps the
-//            main loop of tile i+1)
-//   warps 2-5  epilogue: tensor memory -> registers -> (partials | dZ |
-//            dH accumulate | dW store)
+// method needs); every GEMM is the same warp-specialized persistent kernel,
+// launched as clusters of two CTAs (one per SM) that share each MMA:
+//   warp 0   TMA producer (one thread per CTA): this CTA's 128 A rows and
+//            its half of the 256 B rows per K step, a 6-stage ring
+//   warp 1   MMA issuer (one thread, even CTA only): 256x256x16 bf16
+//            cta_group::2 MMAs; the accumulator's rows are split 128/128
+//            over the two CTAs' tensor memory, two 256-column buffers each
+//            (the epilogue of tile i overlaps the main loop of tile i+1)
+//   warps 2-5  epilogue, in both CTAs: tensor memory -> registers ->
+//            (partials | dZ | dH accumulate | dW store)
 // Tile raster: the forward and dZ GEMMs walk M fastest (H_M, the small
 // operand, stays in L2 while W streams once); the dH and dW GEMMs walk N
 // fastest so the dZ chunk (the large operand) streams once per wave.
