@@ -70,7 +70,7 @@ extern "C" const char* dlm_status_string(dlm_status_t status) {
     }
 }
 
-extern "C" int dlm_version(void) { return 100; }   // 0.1.0
+extern "C" int dlm_version(void) { return 200; }   // 0.2.0: + dlm_loss_fwd_bwd_ex
 
 extern "C" const char* dlm_last_cuda_error(void) { return dlm::g_last_error; }
 
