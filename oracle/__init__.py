@@ -384,12 +384,14 @@ def linear_logits(H_rows: np.ndarray, W: np.ndarray, chunk: int = 16384) -> np.n
 
 def linear_loss(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
                 corrupted: np.ndarray, p: np.ndarray, grad_scale: float = 1.0,
-                want_grads: bool = True):
-    """[Axolotl] CCE path, aligned absorbing only.  Rows of H at masked
-    positions form Z = H_M W^T in double; CE and weights as for the unfused
-    loss; dZ = grad_scale * w * (softmax - onehot); dH_M = dZ W, dW = dZ^T H_M,
-    other rows of dH exactly zero."""
-    plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, ALIGNED)
+                want_grads: bool = True, align: int = ALIGNED):
+    """[Axolotl] CCE path, absorbing noise.  The rows of H that score a
+    target (aligned: row i scores token i, as CCE does on the page; shifted:
+    row i scores token i+1 of the same unit, the unfused loss's Dream
+    reading carried over) form Z = H_M W^T in double; CE and weights as for
+    the unfused loss; dZ = grad_scale * w * (softmax - onehot); dH_M = dZ W,
+    dW = dZ^T H_M, other rows of dH exactly zero."""
+    plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, align)
     rows = np.nonzero(plan.target >= 0)[0]
     V, D = W.shape
     Z = linear_logits(H[rows], W)
@@ -418,10 +420,10 @@ def linear_loss(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
 
 def linear_rows(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
                 corrupted: np.ndarray, p: np.ndarray, sample_rows: np.ndarray,
-                grad_scale: float = 1.0):
+                grad_scale: float = 1.0, align: int = ALIGNED):
     """Full-size spot check: for a few scored rows only, their CE, weight*ce
     and their row of dH (which needs only that row's own softmax)."""
-    plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, ALIGNED)
+    plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, align)
     sample_rows = np.asarray(sample_rows, np.int64)
     assert (plan.target[sample_rows] >= 0).all()
     V, D = W.shape

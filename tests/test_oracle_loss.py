@@ -389,7 +389,8 @@ def test_packing_invariance_of_unit_sums():
 # --------------------------------------------------------------------------
 # fused lm_head
 # --------------------------------------------------------------------------
-def test_linear_equals_unfused_on_materialised_logits():
+@pytest.mark.parametrize("align", [oracle.ALIGNED, oracle.SHIFTED])
+def test_linear_equals_unfused_on_materialised_logits(align):
     rng = np.random.default_rng(12)
     T, D, V = 64, 64, 1000
     lens = [10, 30, 24]
@@ -400,9 +401,9 @@ def test_linear_equals_unfused_on_materialised_logits():
     clean = rng.integers(0, V - 1, T).astype(np.int32)
     _, p = oracle.sample_t(1, 3, oracle.ABSORBING, 1e-3)
     _, corr = oracle.corrupt(lay, clean, p, oracle.ABSORBING, V - 1, V, 2)
-    out = oracle.linear_loss(lay, H, W, clean, corr, p, grad_scale=2.0)
+    out = oracle.linear_loss(lay, H, W, clean, corr, p, grad_scale=2.0, align=align)
     Z = oracle.bf16_to_f64(H) @ oracle.bf16_to_f64(W).T
-    loss, tr = _absorbing_loss_f64(Z, lay, clean, corr, p, oracle.ALIGNED)
+    loss, tr = _absorbing_loss_f64(Z, lay, clean, corr, p, align)
     assert abs(out["loss"] - loss) < 1e-12 * max(1, loss)
     dZ = oracle.term_grad(Z, V, tr, np.arange(T), grad_scale=2.0)
     assert np.allclose(out["dH"], dZ @ oracle.bf16_to_f64(W), rtol=1e-10, atol=1e-14)
