@@ -361,6 +361,7 @@ def run_linear(args, spec, dev, rank, world):
     T, D, V = case.n_tokens, spec.d_model, spec.vocab
     lay = dlm.make_layout(case.n_units, 0, case.cu_seqlens, None, n_tokens=T)
     out = None
+    align = dlm.SHIFTED if args.align == "shifted" else dlm.ALIGNED
 
     def step(seed, ev=None):
         nonlocal out
@@ -368,7 +369,7 @@ def run_linear(args, spec, dev, rank, world):
         _, corr = dlm.corrupt(lay, case.clean, p, spec.mode, spec.mask_id, V, seed)
         if ev is not None:
             ev[0].record()
-        out = dlm.linear_loss_fwd_bwd(lay, case.hidden, case.weight, case.clean, corr, p, out=out)
+        out = dlm.linear_loss_fwd_bwd(lay, case.hidden, case.weight, case.clean, corr, p, out=out, align=align)
         if ev is not None:
             ev[1].record()
         return corr
@@ -405,6 +406,11 @@ def run_linear(args, spec, dev, rank, world):
         t, p = dlm.sample_t(1000 + i, case.n_units, spec.mode, spec.eps)
         _, corr = dlm.corrupt(lay, case.clean, p, spec.mode, spec.mask_id, V, 1000 + i)
         scored += int(corr.sum().item())
+        if align == dlm.SHIFTED:
+            # a document's first token is never a target when rows score the next token
+            cu = case.cu_seqlens.to(torch.int64)
+            first = cu[:-1][cu[1:] > cu[:-1]]
+            scored -= int(corr[first].sum().item())
     ms, call_ms, scored_all = reduce_over_ranks(ms, call_ms, scored, dev)
     value = scored_all / (ms / 1e3)
     M = scored_all / world / K
@@ -430,7 +436,8 @@ def run_linear(args, spec, dev, rank, world):
     res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": spec.key, "description": spec.description, "tokens": T, "d_model": D,
+           "config": {"workload": spec.key, "description": spec.description, "align": args.align,
+                      "tokens": T, "d_model": D,
                       "vocab": V, "documents": case.n_units, "parallelism": f"replicas{world}",
                       "scored_tokens": scored_all, "l2": "inputs larger than L2 (W %.2f GB)" % (V * D * 2 / 1e9)},
            "roofline": roof, "cpu_baseline": None, "clocks": clk, "e2e": None,
@@ -547,6 +554,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--align", choices=["aligned", "shifted"], default="aligned",
+                    help="fused-head workloads: targets aligned (row i scores token i) or shifted (token i+1)")
     ap.add_argument("--objective", choices=["plain", "rhine"], default="plain",
                     help="uniform-noise workloads: plain canvas mean, or the Rhine objective options")
     args = ap.parse_args()

@@ -42,7 +42,7 @@ STATUS = {0: "DLM_OK", 1: "DLM_ERR_INVALID_ARGUMENT", 2: "DLM_ERR_UNSUPPORTED",
 EXPORTS = ("dlm_status_string", "dlm_last_cuda_error", "dlm_version", "dlm_sample_t", "dlm_corrupt",
            "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_loss_fwd_bwd_ex", "dlm_loss_fwd_bwd_static",
            "dlm_linear_loss_workspace_size",
-           "dlm_linear_loss_fwd_bwd", "dlm_get_device_status", "dlm_selftest_bounded_wait")
+           "dlm_linear_loss_fwd_bwd", "dlm_linear_loss_fwd_bwd_ex", "dlm_get_device_status", "dlm_selftest_bounded_wait")
 
 
 class DlmError(RuntimeError):
@@ -127,6 +127,9 @@ def lib():
     L.dlm_linear_loss_fwd_bwd.restype = ctypes.c_int
     L.dlm_linear_loss_fwd_bwd.argtypes = [lp, vp, vp, i32, i32, vp, vp, vp, f32, vp, vp, vp, vp,
                                           vp, sz, vp]
+    L.dlm_linear_loss_fwd_bwd_ex.restype = ctypes.c_int
+    L.dlm_linear_loss_fwd_bwd_ex.argtypes = [lp, vp, vp, i32, i32, vp, vp, vp, i32, f32, vp, vp, vp, vp,
+                                             vp, sz, vp]
     L.dlm_selftest_bounded_wait.restype = ctypes.c_int
     L.dlm_selftest_bounded_wait.argtypes = [u64, vp, vp]
     L.dlm_get_device_status.restype = ctypes.c_int
@@ -268,8 +271,9 @@ def linear_loss_workspace_size(layout: Layout, d_model: int, vocab: int) -> int:
 def linear_loss_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: torch.Tensor,
                         clean_ids: torch.Tensor, corrupted: torch.Tensor, p: torch.Tensor,
                         grad_scale: float = 1.0, want_d_weight: bool = True,
-                        out: Optional[LinearOut] = None) -> LinearOut:
-    """Fused lm_head + absorbing aligned loss (see dlm_linear_loss_fwd_bwd)."""
+                        out: Optional[LinearOut] = None, align: int = ALIGNED) -> LinearOut:
+    """Fused lm_head + absorbing loss (see dlm_linear_loss_fwd_bwd; align =
+    SHIFTED goes through dlm_linear_loss_fwd_bwd_ex)."""
     _check(hidden, torch.bfloat16, "hidden")
     _check(weight, torch.bfloat16, "weight")
     if not (hidden.is_contiguous() and weight.is_contiguous()):
@@ -285,11 +289,18 @@ def linear_loss_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: torch.Tens
                         torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
                         torch.empty_like(hidden),
                         torch.empty_like(weight) if want_d_weight else None, ws)
-    _ok(lib().dlm_linear_loss_fwd_bwd(
-        ctypes.byref(layout), _ptr(hidden), _ptr(weight), D, V, _ptr(clean_ids), _ptr(corrupted),
-        _ptr(p), grad_scale, _ptr(out.loss), _ptr(out.unit_loss), _ptr(out.d_hidden),
-        _ptr(out.d_weight), _ptr(out.workspace), out.workspace.numel(), _stream()),
-        "dlm_linear_loss_fwd_bwd")
+    if align == ALIGNED:
+        _ok(lib().dlm_linear_loss_fwd_bwd(
+            ctypes.byref(layout), _ptr(hidden), _ptr(weight), D, V, _ptr(clean_ids), _ptr(corrupted),
+            _ptr(p), grad_scale, _ptr(out.loss), _ptr(out.unit_loss), _ptr(out.d_hidden),
+            _ptr(out.d_weight), _ptr(out.workspace), out.workspace.numel(), _stream()),
+            "dlm_linear_loss_fwd_bwd")
+    else:
+        _ok(lib().dlm_linear_loss_fwd_bwd_ex(
+            ctypes.byref(layout), _ptr(hidden), _ptr(weight), D, V, _ptr(clean_ids), _ptr(corrupted),
+            _ptr(p), align, grad_scale, _ptr(out.loss), _ptr(out.unit_loss), _ptr(out.d_hidden),
+            _ptr(out.d_weight), _ptr(out.workspace), out.workspace.numel(), _stream()),
+            "dlm_linear_loss_fwd_bwd_ex")
     return out
 
 

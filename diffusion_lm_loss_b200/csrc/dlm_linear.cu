@@ -641,13 +641,14 @@ extern "C" size_t dlm_linear_loss_workspace_size(const dlm_layout_t* layout, int
     return lin_ws(layout->n_tokens, layout->n_units, d_model, vocab).total;
 }
 
-extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16_t* hidden,
-                                                const uint16_t* weight, int32_t d_model, int32_t vocab,
-                                                const int32_t* clean_ids, const uint8_t* corrupted,
-                                                const float* p, float grad_scale, float* loss,
-                                                float* unit_loss, uint16_t* d_hidden, uint16_t* d_weight,
-                                                void* workspace, size_t workspace_bytes, dlm_stream_t stream) {
+static dlm_status_t linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16_t* hidden,
+                                        const uint16_t* weight, int32_t d_model, int32_t vocab,
+                                        const int32_t* clean_ids, const uint8_t* corrupted, const float* p,
+                                        int32_t align, float grad_scale, float* loss, float* unit_loss,
+                                        uint16_t* d_hidden, uint16_t* d_weight, void* workspace,
+                                        size_t workspace_bytes, dlm_stream_t stream) {
     if (!layout_ok(layout)) return DLM_ERR_INVALID_ARGUMENT;
+    if (align != DLM_ALIGNED && align != DLM_SHIFTED) return DLM_ERR_INVALID_ARGUMENT;
     if (d_model <= 0 || d_model % 64 != 0 || vocab <= 0 || vocab % 8 != 0) return DLM_ERR_INVALID_ARGUMENT;
     if (!loss || !workspace) return DLM_ERR_INVALID_ARGUMENT;
     const int64_t T = layout->n_tokens;
@@ -674,8 +675,9 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, cons
     uint16_t* dz = reinterpret_cast<uint16_t*>(ws + W.dz);
     float* dh = reinterpret_cast<float*>(ws + W.dh);
 
-    // 1. which rows are scored, their targets and weights (absorbing, aligned)
-    if ((st = launch_plan(layout, clean_ids, corrupted, p, DLM_ABSORBING, DLM_ALIGNED, nullptr, nullptr, 0.f,
+    // 1. which rows are scored, their targets and weights (absorbing; row i
+    //    scores token i, or token i+1 of the same unit when shifted)
+    if ((st = launch_plan(layout, clean_ids, corrupted, p, DLM_ABSORBING, align, nullptr, nullptr, 0.f,
                           vocab, hdr, list, s)) != DLM_OK)
         return st;
     if (T == 0) {
@@ -755,4 +757,27 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, cons
     k_scatter_dh<<<sms * 4, 256, 0, s>>>(hdr, list, dh, d_model, d_hidden);
     if ((st = last_launch_status("k_scatter_dh launch")) != DLM_OK) return st;
     return launch_reduce(layout, nullptr, row_loss, unit_acc, unit_loss, loss, hdr, s);
+}
+
+extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16_t* hidden,
+                                                const uint16_t* weight, int32_t d_model, int32_t vocab,
+                                                const int32_t* clean_ids, const uint8_t* corrupted,
+                                                const float* p, float grad_scale, float* loss,
+                                                float* unit_loss, uint16_t* d_hidden, uint16_t* d_weight,
+                                                void* workspace, size_t workspace_bytes, dlm_stream_t stream) {
+    return linear_loss_fwd_bwd(layout, hidden, weight, d_model, vocab, clean_ids, corrupted, p, DLM_ALIGNED,
+                               grad_scale, loss, unit_loss, d_hidden, d_weight, workspace, workspace_bytes,
+                               stream);
+}
+
+extern "C" dlm_status_t dlm_linear_loss_fwd_bwd_ex(const dlm_layout_t* layout, const uint16_t* hidden,
+                                                   const uint16_t* weight, int32_t d_model, int32_t vocab,
+                                                   const int32_t* clean_ids, const uint8_t* corrupted,
+                                                   const float* p, int32_t align, float grad_scale,
+                                                   float* loss, float* unit_loss, uint16_t* d_hidden,
+                                                   uint16_t* d_weight, void* workspace, size_t workspace_bytes,
+                                                   dlm_stream_t stream) {
+    return linear_loss_fwd_bwd(layout, hidden, weight, d_model, vocab, clean_ids, corrupted, p, align,
+                               grad_scale, loss, unit_loss, d_hidden, d_weight, workspace, workspace_bytes,
+                               stream);
 }

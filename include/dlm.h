@@ -14,6 +14,8 @@
  *                            with the uniform-noise objective options)
  *   dlm_linear_loss_fwd_bwd  the same loss from hidden states and a linear
  *                            output head, logits never materialised
+ *                            (dlm_linear_loss_fwd_bwd_ex: aligned or shifted
+ *                            targets)
  *
  * The method (page title, section):
  *   "LLaDA-8B-MDLM-LoRA", Training table, row "Objective": t ~ U(0,1) per
@@ -294,6 +296,21 @@ DLM_API dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t *layout, const u
                                      float *unit_loss, uint16_t *d_hidden, uint16_t *d_weight,
                                      void *workspace, size_t workspace_bytes,
                                      dlm_stream_t stream);
+
+/* dlm_linear_loss_fwd_bwd_ex -- the same with the alignment as an argument:
+ * DLM_ALIGNED as above, or DLM_SHIFTED (row i, i.e. hidden state i, scores
+ * token i + 1 of the same unit; a unit's last row is unscored -- the rows
+ * and weights of dlm_loss_fwd_bwd with DLM_SHIFTED).  The page describes
+ * Cut Cross Entropy for aligned targets only; the shifted form carries the
+ * unfused loss's Dream alignment over.  Any other align returns
+ * DLM_ERR_INVALID_ARGUMENT. */
+DLM_API dlm_status_t dlm_linear_loss_fwd_bwd_ex(const dlm_layout_t *layout, const uint16_t *hidden,
+                                        const uint16_t *weight, int32_t d_model, int32_t vocab,
+                                        const int32_t *clean_ids, const uint8_t *corrupted,
+                                        const float *p, int32_t align, float grad_scale,
+                                        float *loss, float *unit_loss, uint16_t *d_hidden,
+                                        uint16_t *d_weight, void *workspace, size_t workspace_bytes,
+                                        dlm_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * dlm_get_device_status -- copy the device status word of a loss workspace

@@ -36,7 +36,7 @@ def rel_fro(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
-def run_linear(spec, case, seed=0, grad_scale=1.0, want_dw=True):
+def run_linear(spec, case, seed=0, grad_scale=1.0, want_dw=True, align=oracle.ALIGNED):
     dev = torch.device("cuda")
     T = case.n_tokens
     lay = dlm.make_layout(case.n_units, case.seq_len, case.cu_seqlens.to(dev) if case.cu_seqlens is not None else None,
@@ -45,7 +45,7 @@ def run_linear(spec, case, seed=0, grad_scale=1.0, want_dw=True):
     t, p = dlm.sample_t(seed, case.n_units, oracle.ABSORBING, spec.eps)
     _, corr = dlm.corrupt(lay, clean, p, oracle.ABSORBING, spec.mask_id, spec.vocab, seed)
     out = dlm.linear_loss_fwd_bwd(lay, case.hidden.to(dev), case.weight.to(dev), clean, corr, p,
-                                  grad_scale=grad_scale, want_d_weight=want_dw)
+                                  grad_scale=grad_scale, want_d_weight=want_dw, align=align)
     torch.cuda.synchronize()
     assert out.device_status() == 0
     cu = case.cu_seqlens.cpu().numpy() if case.cu_seqlens is not None else None
@@ -55,6 +55,29 @@ def run_linear(spec, case, seed=0, grad_scale=1.0, want_dw=True):
                                spec.vocab, seed)
     assert np.array_equal(corr.cpu().numpy(), corr_o)
     return out, lay_o, p_o, corr_o
+
+
+@pytest.mark.parametrize("T,D,V,seed", [(64, 64, 1000, 4), (700, 128, 4104, 5), (2048, 256, 20000, 6)])
+def test_linear_shifted_elementwise(T, D, V, seed):
+    """Shifted targets through the fused head: hidden state i scores token
+    i+1 of its document (the unfused loss's Dream alignment)."""
+    spec = di.WORKLOADS["lin_t16384_d4096_v126464"].scaled(n_tokens_packed=T, d_model=D, vocab=V,
+                                                           ids_high=V - 2, mask_id=V - 1, doc_mean=50.0)
+    case = di.make_case(spec, "cuda")
+    out, lay_o, p_o, corr_o = run_linear(spec, case, seed=seed, grad_scale=0.75, align=oracle.SHIFTED)
+    H = di.bf16_bits(case.hidden)
+    W = di.bf16_bits(case.weight)
+    ref = oracle.linear_loss(lay_o, H, W, case.clean.cpu().numpy(), corr_o, p_o, grad_scale=0.75,
+                             align=oracle.SHIFTED)
+    assert_loss_close(float(out.loss.item()), ref["loss"])
+    assert_units_close(out.unit_loss.cpu().numpy()[:case.n_units], ref["unit_loss"], ref["loss"])
+    dH = out.d_hidden.double().cpu().numpy()
+    dW = out.d_weight.double().cpu().numpy()
+    assert rel_fro(dH, ref["dH"]) < GRAD_REL_FRO
+    assert rel_fro(dW, ref["dW"]) < GRAD_REL_FRO
+    unscored = np.ones(T, bool)
+    unscored[ref["rows"]] = False
+    assert (dH[unscored] == 0).all()
 
 
 @pytest.mark.parametrize("T,D,V,seed", [(64, 64, 1000, 0), (512, 256, 4096, 1), (300, 128, 2056, 2),
