@@ -54,10 +54,13 @@ class DlmError(RuntimeError):
 class LossOptions(ctypes.Structure):
     """dlm_loss_options_t: uniform-noise objective options."""
     _fields_ = [("struct_size", ctypes.c_uint32), ("time_weighting", ctypes.c_int32),
-                ("weight_clip", ctypes.c_float), ("reduction", ctypes.c_int32)]
+                ("weight_clip", ctypes.c_float), ("reduction", ctypes.c_int32),
+                ("keep_unscored_rows", ctypes.c_int32)]
 
-    def __init__(self, time_weighting=TIME_WEIGHT_NONE, weight_clip=0.0, reduction=REDUCE_TOKEN_MEAN):
-        super().__init__(ctypes.sizeof(LossOptions), time_weighting, weight_clip, reduction)
+    def __init__(self, time_weighting=TIME_WEIGHT_NONE, weight_clip=0.0, reduction=REDUCE_TOKEN_MEAN,
+                 keep_unscored_rows=0):
+        super().__init__(ctypes.sizeof(LossOptions), time_weighting, weight_clip, reduction,
+                         keep_unscored_rows)
 
 
 class Layout(ctypes.Structure):
@@ -231,10 +234,12 @@ def loss_fwd_bwd(layout: Layout, logits: torch.Tensor, vocab: int, clean_ids: to
     dev = logits.device
     if out is None:
         ws = torch.empty(loss_workspace_size(layout, enc_layout), dtype=torch.uint8, device=dev)
+        # rows the call leaves untouched must start as zeros
+        grad_buf = torch.zeros_like if (options is not None and options.keep_unscored_rows) else torch.empty_like
         out = LossOut(torch.empty(1, dtype=torch.float32, device=dev),
                       torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
-                      torch.empty_like(logits),
-                      torch.empty_like(enc_logits) if enc_logits is not None else None, ws)
+                      grad_buf(logits),
+                      grad_buf(enc_logits) if enc_logits is not None else None, ws)
     if options is None:
         _ok(lib().dlm_loss_fwd_bwd(
             ctypes.byref(layout), _ptr(logits), ld, vocab, _ptr(clean_ids), _ptr(corrupted), _ptr(p),

@@ -444,6 +444,7 @@ struct CeParams {
     const WsHeader* hdr;
     uint32_t* status;
     WsHeader* hdr_w;         // the same header, written: the row tickets
+    int keep_unscored;       // 1: unscored rows of the gradient are not written
     const uint16_t* xa; uint16_t* da; int64_t lda; int64_t rows_a;
     const uint16_t* xb; uint16_t* db; int64_t ldb;
     int vocab;
@@ -587,15 +588,17 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
                 const int j = int(atomicAdd(tick_u, 1u));
                 if (j >= n_uns) { zleft = false; return; }
                 const int q = P.list[n_scored + j].x;
-                const uint16_t* xr;
-                uint16_t* dr;
-                row_ptrs(P, q, xr, dr);
-                const uint32_t bytes = uint32_t(V) * 2u;
-                for (uint32_t off = 0; off < bytes; off += kZeroBytes) {
-                    const uint32_t n = bytes - off < uint32_t(kZeroBytes) ? bytes - off : uint32_t(kZeroBytes);
-                    bulk_s2g_hint(reinterpret_cast<uint8_t*>(dr) + off, smem_addr(S.zero), n, pol_drop);
+                if (!P.keep_unscored) {
+                    const uint16_t* xr;
+                    uint16_t* dr;
+                    row_ptrs(P, q, xr, dr);
+                    const uint32_t bytes = uint32_t(V) * 2u;
+                    for (uint32_t off = 0; off < bytes; off += kZeroBytes) {
+                        const uint32_t n = bytes - off < uint32_t(kZeroBytes) ? bytes - off : uint32_t(kZeroBytes);
+                        bulk_s2g_hint(reinterpret_cast<uint8_t*>(dr) + off, smem_addr(S.zero), n, pol_drop);
+                    }
+                    bulk_commit_group();
                 }
-                bulk_commit_group();
                 P.row_loss[q] = 0.f;
                 ++zdone;
             };
@@ -809,7 +812,8 @@ __global__ void __launch_bounds__(kGenThreads) k_ce_generic(const CeParams P) {
         uint16_t* d;
         row_ptrs(P, q, x, d);
         if (y < 0) {
-            for (int v = tid; v < V; v += kGenThreads) d[v] = 0;
+            if (!P.keep_unscored)
+                for (int v = tid; v < V; v += kGenThreads) d[v] = 0;
             if (tid == 0) P.row_loss[q] = 0.f;
             continue;
         }
@@ -1156,6 +1160,7 @@ static dlm_status_t loss_fwd_bwd(const dlm_layout_t* layout, const uint16_t* log
         cp.grad_scale = grad_scale;
         cp.row_loss = row_loss;
         cp.hdr_w = hdr;
+        cp.keep_unscored = opts.keep_unscored_rows;
 
         bool launched = false;
         if (fast) {
@@ -1198,7 +1203,8 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd_ex(const dlm_layout_t* layout, const ui
                                             void* workspace, size_t workspace_bytes, dlm_stream_t stream) {
     ObjOpts o;
     if (options) {
-        if (options->struct_size < sizeof(dlm_loss_options_t)) return DLM_ERR_INVALID_ARGUMENT;
+        // 16 bytes: the struct before keep_unscored_rows was added
+        if (options->struct_size < 16) return DLM_ERR_INVALID_ARGUMENT;
         if (options->time_weighting != DLM_TIME_WEIGHT_NONE &&
             options->time_weighting != DLM_TIME_WEIGHT_INV_ONE_MINUS_T)
             return DLM_ERR_INVALID_ARGUMENT;
@@ -1211,6 +1217,11 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd_ex(const dlm_layout_t* layout, const ui
         o.time_weighting = options->time_weighting;
         o.weight_clip = options->weight_clip;
         o.reduction = options->reduction;
+        if (options->struct_size >= offsetof(dlm_loss_options_t, keep_unscored_rows) + sizeof(int32_t)) {
+            if (options->keep_unscored_rows != 0 && options->keep_unscored_rows != 1)
+                return DLM_ERR_INVALID_ARGUMENT;
+            o.keep_unscored_rows = options->keep_unscored_rows;
+        }
     }
     return loss_fwd_bwd(layout, logits, ld, vocab, clean_ids, corrupted, p, mode, align, enc_layout, enc_logits,
                         enc_ld, enc_ids, enc_ar_weight, grad_scale, o, loss, unit_loss, dlogits, enc_dlogits,

@@ -92,6 +92,7 @@ struct ObjOpts {
     float weight_clip = 0.f;
     int reduction = DLM_REDUCE_TOKEN_MEAN;
     int32_t* unit_cnt = nullptr;
+    int keep_unscored_rows = 0;   // unscored dlogits rows are not written
 };
 
 // Row plan (one cluster of CTAs): classifies every row of `a` (and of the

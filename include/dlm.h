@@ -214,10 +214,10 @@ DLM_API dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t *layout, const uint16_t
  *   f_u = min(1 / (1 - t_u), weight_clip)              DLM_TIME_WEIGHT_INV_ONE_MINUS_T
  * (no cap when weight_clip <= 0; t_u = p[u], the uniform-noise time from
  * dlm_sample_t, which p must then hold).  The encoder AR term is unchanged.
- * options == NULL, or both fields at their defaults, is dlm_loss_fwd_bwd.
- * Non-default options with absorbing noise, or time weighting without p,
- * return DLM_ERR_INVALID_ARGUMENT; so does options->struct_size <
- * sizeof(dlm_loss_options_t).
+ * options == NULL, or every field at its default, is dlm_loss_fwd_bwd.
+ * Non-default time weighting or reduction with absorbing noise, or time
+ * weighting without p, return DLM_ERR_INVALID_ARGUMENT; so does
+ * options->struct_size < 16.
  * ---------------------------------------------------------------------- */
 #define DLM_TIME_WEIGHT_NONE 0
 #define DLM_TIME_WEIGHT_INV_ONE_MINUS_T 1
@@ -229,6 +229,11 @@ typedef struct {
     int32_t time_weighting;    /* DLM_TIME_WEIGHT_* */
     float weight_clip;         /* cap of 1 / (1 - t); <= 0: none */
     int32_t reduction;         /* DLM_REDUCE_* */
+    int32_t keep_unscored_rows;/* 1: rows of dlogits / enc_dlogits that are not
+                                  scored are left as they are instead of being
+                                  zeroed (for a caller that keeps them zero);
+                                  any noise mode.  Read only when struct_size
+                                  covers it (older 16-byte structs: 0). */
 } dlm_loss_options_t;
 
 DLM_API dlm_status_t dlm_loss_fwd_bwd_ex(const dlm_layout_t *layout, const uint16_t *logits, int64_t ld,

@@ -91,6 +91,10 @@ def test_host_side_rejections(L):
     assert ex(short) == 1
     assert ex(dlm.LossOptions(dlm.TIME_WEIGHT_INV_ONE_MINUS_T), p=None) == 1          # no p
     assert ex(dlm.LossOptions(weight_clip=float("nan"))) == 1
+    assert ex(dlm.LossOptions(keep_unscored_rows=2)) == 1
+    old16 = dlm.LossOptions(keep_unscored_rows=2)    # a 16-byte struct: the field is not read
+    old16.struct_size = 16
+    assert ex(old16) != 1
     # fused head: alignment must be aligned or shifted
     lin = dlm.Layout(1, 64, 64, None, None)
     assert L.dlm_linear_loss_fwd_bwd_ex(ctypes.byref(lin), 16, 16, 64, 1024, 16, 16, 16, 7, 1.0, 16, None,

@@ -233,6 +233,39 @@ def test_empty_input():
     assert out.unit_loss.cpu().tolist() == [0.0, 0.0]
 
 
+@pytest.mark.parametrize("V", [126464, 1000])
+def test_keep_unscored_rows_leaves_them_untouched(V):
+    """keep_unscored_rows: scored rows as usual, every other row of dlogits
+    keeps what the caller put there (fast kernel and general kernel)."""
+    spec = di.WORKLOADS["abs_b1_l4096_v126464"].scaled(vocab=V, mask_id=V - 1, ids_high=V - 2, seq_len=96,
+                                                       spike=0.0)
+    case = di.make_case(spec, "cuda")
+    dev = torch.device("cuda")
+    lay = dlm.make_layout(1, 96)
+    t, p = dlm.sample_t(6, 1)
+    _, corr = dlm.corrupt(lay, case.clean, p, oracle.ABSORBING, spec.mask_id, V, 6)
+    opts = dlm.LossOptions(keep_unscored_rows=1)
+    sentinel = 0x3F80                                        # bf16 1.0
+    out = dlm.loss_fwd_bwd(lay, case.logits, V, case.clean, corr, p, options=opts)
+    out.dlogits.view(torch.int16).fill_(sentinel)
+    out = dlm.loss_fwd_bwd(lay, case.logits, V, case.clean, corr, p, options=opts, out=out)
+    torch.cuda.synchronize()
+    assert out.device_status() == 0
+    lay_o = oracle.Layout(1, 96, None, None)
+    _, p_o = oracle.sample_t(6, 1, oracle.ABSORBING, 1e-3)
+    _, corr_o = oracle.corrupt(lay_o, case.clean.cpu().numpy(), p_o, oracle.ABSORBING, spec.mask_id, V, 6)
+    x = di.bf16_bits(case.logits)
+    loss_o, unit_o, tr = oracle.loss_absorbing(lay_o, x, V, case.clean.cpu().numpy(), corr_o, p_o, oracle.ALIGNED)
+    assert_loss_close(float(out.loss.item()), loss_o)
+    scored = tr.rows
+    assert 0 < scored.size < 96
+    assert_grad_close(gpu_bf16_to_f64(out.dlogits[torch.from_numpy(scored).to(dev)]),
+                      oracle.term_grad(x, V, tr, scored, 1.0))
+    unscored = np.setdiff1d(np.arange(96), scored)
+    bits = out.dlogits.view(torch.int16)[torch.from_numpy(unscored).to(dev)].cpu().numpy()
+    assert (bits == sentinel).all()
+
+
 def test_bad_target_id_is_flagged_and_row_skipped():
     spec = di.WORKLOADS["abs_b1_l4096_v126464"].scaled(seq_len=64)
     case = di.make_case(spec, "cuda")
