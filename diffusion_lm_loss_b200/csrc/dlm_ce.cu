@@ -1188,6 +1188,7 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd(const dlm_layout_t* layout, const uint1
                                          float grad_scale, float* loss, float* unit_loss,
                                          uint16_t* dlogits, uint16_t* enc_dlogits,
                                          void* workspace, size_t workspace_bytes, dlm_stream_t stream) {
+    DLM_NVTX("dlm_loss_fwd_bwd");
     return loss_fwd_bwd(layout, logits, ld, vocab, clean_ids, corrupted, p, mode, align, enc_layout, enc_logits,
                         enc_ld, enc_ids, enc_ar_weight, grad_scale, ObjOpts(), loss, unit_loss, dlogits,
                         enc_dlogits, workspace, workspace_bytes, stream);
@@ -1201,6 +1202,7 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd_ex(const dlm_layout_t* layout, const ui
                                             float grad_scale, const dlm_loss_options_t* options, float* loss,
                                             float* unit_loss, uint16_t* dlogits, uint16_t* enc_dlogits,
                                             void* workspace, size_t workspace_bytes, dlm_stream_t stream) {
+    DLM_NVTX("dlm_loss_fwd_bwd_ex");
     ObjOpts o;
     if (options) {
         // 16 bytes: the struct before keep_unscored_rows was added

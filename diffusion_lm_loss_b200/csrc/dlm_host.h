@@ -7,9 +7,21 @@
 #include <cuda_runtime.h>
 #include <utility>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/dlm.h"
 
 namespace dlm {
+
+// NVTX range around an entry point, so a profiler's timeline shows each
+// library call by name (header-only NVTX: a no-op unless a tool is attached).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+#define DLM_NVTX(name) ::dlm::NvtxRange dlm_nvtx_range_(name)
 
 constexpr size_t kWsAlign = 256;
 

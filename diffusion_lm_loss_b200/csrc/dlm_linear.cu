@@ -765,6 +765,7 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, cons
                                                 const float* p, float grad_scale, float* loss,
                                                 float* unit_loss, uint16_t* d_hidden, uint16_t* d_weight,
                                                 void* workspace, size_t workspace_bytes, dlm_stream_t stream) {
+    DLM_NVTX("dlm_linear_loss_fwd_bwd");
     return linear_loss_fwd_bwd(layout, hidden, weight, d_model, vocab, clean_ids, corrupted, p, DLM_ALIGNED,
                                grad_scale, loss, unit_loss, d_hidden, d_weight, workspace, workspace_bytes,
                                stream);
@@ -777,6 +778,7 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd_ex(const dlm_layout_t* layout, c
                                                    float* loss, float* unit_loss, uint16_t* d_hidden,
                                                    uint16_t* d_weight, void* workspace, size_t workspace_bytes,
                                                    dlm_stream_t stream) {
+    DLM_NVTX("dlm_linear_loss_fwd_bwd_ex");
     return linear_loss_fwd_bwd(layout, hidden, weight, d_model, vocab, clean_ids, corrupted, p, align,
                                grad_scale, loss, unit_loss, d_hidden, d_weight, workspace, workspace_bytes,
                                stream);

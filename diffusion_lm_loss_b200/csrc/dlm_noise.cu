@@ -78,6 +78,7 @@ using namespace dlm;
 
 extern "C" dlm_status_t dlm_sample_t(uint64_t seed, int32_t n_units, int32_t mode, float eps,
                                      float* t, float* p, dlm_stream_t stream) {
+    DLM_NVTX("dlm_sample_t");
     if (n_units < 0 || n_units >= (1 << 24)) return DLM_ERR_INVALID_ARGUMENT;
     if (mode != DLM_ABSORBING && mode != DLM_UNIFORM) return DLM_ERR_INVALID_ARGUMENT;
     if (!(eps >= 0.0f && eps < 1.0f)) return DLM_ERR_INVALID_ARGUMENT;
@@ -94,6 +95,7 @@ extern "C" dlm_status_t dlm_corrupt(const dlm_layout_t* layout, const int32_t* c
                                     const float* p, int32_t mode, int32_t mask_id, int32_t vocab,
                                     uint64_t seed, int32_t* noisy_ids, uint8_t* corrupted,
                                     uint32_t* dev_status, dlm_stream_t stream) {
+    DLM_NVTX("dlm_corrupt");
     if (!layout_ok(layout)) return DLM_ERR_INVALID_ARGUMENT;
     if (mode != DLM_ABSORBING && mode != DLM_UNIFORM) return DLM_ERR_INVALID_ARGUMENT;
     if (mode == DLM_UNIFORM && vocab <= 0) return DLM_ERR_INVALID_ARGUMENT;

@@ -60,6 +60,7 @@ extern "C" dlm_status_t dlm_loss_fwd_bwd_static(const dlm_layout_t* layout, cons
                                                 float enc_ar_weight, float grad_scale, float* loss,
                                                 float* unit_loss, uint16_t* dlogits, uint16_t* enc_dlogits,
                                                 dlm_stream_t stream) {
+    DLM_NVTX("dlm_loss_fwd_bwd_static");
     if (!dlm::layout_ok(layout)) return DLM_ERR_INVALID_ARGUMENT;
     if (enc_logits && !dlm::layout_ok(enc_layout)) return DLM_ERR_INVALID_ARGUMENT;
     const size_t need = dlm_loss_workspace_size(layout, enc_logits ? enc_layout : nullptr);

@@ -266,6 +266,44 @@ def test_keep_unscored_rows_leaves_them_untouched(V):
     assert (bits == sentinel).all()
 
 
+@pytest.mark.parametrize("V,align", [(126464, oracle.ALIGNED), (152064, oracle.SHIFTED), (1000, oracle.ALIGNED)])
+def test_every_gradient_element_is_written(V, align):
+    """Outputs poisoned with NaN before the call: afterwards no element of
+    dlogits may still hold the poison (scored rows get the gradient, all
+    others zeros)."""
+    spec = di.WORKLOADS["abs_b1_l4096_v126464"].scaled(vocab=V, mask_id=V - 1, ids_high=V - 2, n_units=3,
+                                                       seq_len=70, spike=0.0, align=align)
+    case = di.make_case(spec, "cuda")
+    lay = dlm.make_layout(3, 70)
+    t, p = dlm.sample_t(9, 3)
+    _, corr = dlm.corrupt(lay, case.clean, p, oracle.ABSORBING, spec.mask_id, V, 9)
+    out = dlm.loss_fwd_bwd(lay, case.logits, V, case.clean, corr, p, oracle.ABSORBING, align)
+    out.dlogits.fill_(float("nan"))
+    out = dlm.loss_fwd_bwd(lay, case.logits, V, case.clean, corr, p, oracle.ABSORBING, align, out=out)
+    torch.cuda.synchronize()
+    assert out.device_status() == 0
+    assert not bool(torch.isnan(out.dlogits).any())
+
+
+def test_every_gradient_element_is_written_uniform():
+    spec = di.WORKLOADS["unif_b4_p512_c1024_v262144"].scaled(n_units=2, prefix=8, seq_len=24)
+    case = di.make_case(spec, "cuda")
+    B, C, P, V = 2, 24, 8, spec.vocab
+    lay = dlm.make_layout(B, C)
+    enc_lay = dlm.make_layout(B, P + C)
+    t, p = dlm.sample_t(2, B, oracle.UNIFORM, spec.eps)
+    _, corr = dlm.corrupt(lay, case.clean, p, oracle.UNIFORM, -1, V, 2)
+    kw = dict(enc_layout=enc_lay, enc_logits=case.enc_logits, enc_ids=case.enc_clean, enc_ar_weight=1.0)
+    out = dlm.loss_fwd_bwd(lay, case.logits, V, case.clean, corr, p, oracle.UNIFORM, oracle.ALIGNED, **kw)
+    out.dlogits.fill_(float("nan"))
+    out.enc_dlogits.fill_(float("nan"))
+    out = dlm.loss_fwd_bwd(lay, case.logits, V, case.clean, corr, p, oracle.UNIFORM, oracle.ALIGNED, out=out,
+                           **kw)
+    torch.cuda.synchronize()
+    assert not bool(torch.isnan(out.dlogits).any())
+    assert not bool(torch.isnan(out.enc_dlogits).any())
+
+
 def test_bad_target_id_is_flagged_and_row_skipped():
     spec = di.WORKLOADS["abs_b1_l4096_v126464"].scaled(seq_len=64)
     case = di.make_case(spec, "cuda")
