@@ -74,6 +74,9 @@ class Layout(ctypes.Structure):
 
 def make_layout(n_units: int, seq_len: int = 0, cu_seqlens: Optional[torch.Tensor] = None,
                 pad_mask: Optional[torch.Tensor] = None, n_tokens: Optional[int] = None) -> Layout:
+    """A dlm_layout_t over device tensors.  The layout holds references to
+    cu_seqlens and pad_mask, whose device pointers it carries, so they stay
+    allocated as long as the layout is in use."""
     if cu_seqlens is not None:
         _check(cu_seqlens, torch.int32, "cu_seqlens")
         if n_tokens is None:
@@ -86,7 +89,9 @@ def make_layout(n_units: int, seq_len: int = 0, cu_seqlens: Optional[torch.Tenso
     if pad_mask is not None:
         _check(pad_mask, torch.uint8, "pad_mask")
         pm = pad_mask.data_ptr()
-    return Layout(n_units, seq_len, n_tokens, cu, pm)
+    lay = Layout(n_units, seq_len, n_tokens, cu, pm)
+    lay._tensors = (cu_seqlens, pad_mask)
+    return lay
 
 
 _lib = None

@@ -80,6 +80,34 @@ def test_linear_shifted_elementwise(T, D, V, seed):
     assert (dH[unscored] == 0).all()
 
 
+def test_linear_pads_negative_scale_no_dw():
+    """Padded tokens (never scored, not counted in N), a negative gradient
+    scale, and d_weight skipped."""
+    T, D, V = 640, 128, 4096
+    spec = di.WORKLOADS["lin_t16384_d4096_v126464"].scaled(n_tokens_packed=T, d_model=D, vocab=V,
+                                                           ids_high=V - 2, mask_id=V - 1, doc_mean=60.0)
+    case = di.make_case(spec, "cuda")
+    dev = torch.device("cuda")
+    rng = np.random.default_rng(8)
+    pad = (rng.random(T) < 0.15).astype(np.uint8)
+    lay = dlm.make_layout(case.n_units, 0, case.cu_seqlens, torch.from_numpy(pad).to(dev), n_tokens=T)
+    t, p = dlm.sample_t(8, case.n_units)
+    _, corr = dlm.corrupt(lay, case.clean, p, oracle.ABSORBING, spec.mask_id, V, 8)
+    out = dlm.linear_loss_fwd_bwd(lay, case.hidden, case.weight, case.clean, corr, p, grad_scale=-0.5,
+                                  want_d_weight=False)
+    torch.cuda.synchronize()
+    assert out.device_status() == 0 and out.d_weight is None
+    lay_o = oracle.Layout(case.n_units, 0, case.cu_seqlens.cpu().numpy(), pad)
+    _, p_o = oracle.sample_t(8, case.n_units, oracle.ABSORBING, spec.eps)
+    _, corr_o = oracle.corrupt(lay_o, case.clean.cpu().numpy(), p_o, oracle.ABSORBING, spec.mask_id, V, 8)
+    assert np.array_equal(corr.cpu().numpy(), corr_o)
+    assert not corr_o[pad == 1].any()
+    ref = oracle.linear_loss(lay_o, di.bf16_bits(case.hidden), di.bf16_bits(case.weight),
+                             case.clean.cpu().numpy(), corr_o, p_o, grad_scale=-0.5)
+    assert_loss_close(float(out.loss.item()), ref["loss"])
+    assert rel_fro(out.d_hidden.double().cpu().numpy(), ref["dH"]) < GRAD_REL_FRO
+
+
 @pytest.mark.parametrize("T,D,V,seed", [(64, 64, 1000, 0), (512, 256, 4096, 1), (300, 128, 2056, 2),
                                         (2048, 512, 40000, 3)])
 def test_linear_elementwise(T, D, V, seed):
