@@ -483,19 +483,30 @@ def oracle_step(spec, case_cpu, seed, rows_sample):
     clean = case_cpu.clean.view(B, spec.seq_len)[:, :L].reshape(-1).numpy()
     x = di.bf16_bits(case_cpu.logits.view(B, spec.seq_len, -1)[:, :L].reshape(B * L, -1))
     _, p = oracle.sample_t(seed, B, spec.mode, spec.eps)
+    _, corr = oracle.corrupt(lay, clean, p, spec.mode, spec.mask_id, spec.vocab, seed)
     if spec.mode == oracle.ABSORBING:
-        _, corr = oracle.corrupt(lay, clean, p, spec.mode, spec.mask_id, spec.vocab, seed)
         loss, unit, tr = oracle.loss_absorbing(lay, x, spec.vocab, clean, corr, p, spec.align)
         oracle.term_grad(x, spec.vocab, tr, np.arange(B * L), 1.0)
         return int(tr.rows.shape[0])
-    raise SystemExit("reference arm: uniform workloads not wired")
+    # uniform noise: the canvas term plus the encoder AR term over the first
+    # rows of each (prefix + canvas) sequence
+    S = spec.prefix + spec.seq_len
+    Le = min(S, rows_sample)
+    enc = oracle.Layout(B, Le, None, None)
+    eclean = case_cpu.enc_clean.view(B, S)[:, :Le].reshape(-1).numpy()
+    xe = di.bf16_bits(case_cpu.enc_logits.view(B, S, -1)[:, :Le].reshape(B * Le, -1))
+    loss, unit, tc, te = oracle.loss_uniform(lay, x, clean, enc, xe, eclean, spec.vocab,
+                                             spec.enc_ar_weight, spec.align)
+    oracle.term_grad(x, spec.vocab, tc, np.arange(B * L), 1.0)
+    oracle.term_grad(xe, spec.vocab, te, np.arange(B * Le), 1.0)
+    return int(tc.rows.shape[0] + te.rows.shape[0])
 
 
 def _calibrated_rows(spec, per_step_s, cap=1024):
     """Rows per sequence such that one oracle step takes about per_step_s."""
     import dlm_inputs as di
 
-    probe = spec.scaled(seq_len=min(spec.seq_len, 16))
+    probe = spec.scaled(seq_len=min(spec.seq_len, 16), prefix=min(spec.prefix, 16))
     case = di.make_case(probe, "cpu")
     oracle_step(probe, case, 0, probe.seq_len)          # first call builds / loads the oracle
     t0 = time.perf_counter()
@@ -513,7 +524,7 @@ def cpu_baseline(spec, budget_s=15.0, steps=3):
     import dlm_inputs as di
 
     rows = _calibrated_rows(spec, budget_s / steps)
-    sub = spec.scaled(seq_len=rows)
+    sub = spec.scaled(seq_len=rows, prefix=min(spec.prefix, rows))
     case = di.make_case(sub, "cpu")
     t0 = time.perf_counter()
     scored = 0
@@ -537,7 +548,7 @@ def run_reference(args):
 
     spec = di.WORKLOADS[args.workload]
     rows = _calibrated_rows(spec, 100.0 / (args.steps + args.warmup))
-    sub = spec.scaled(seq_len=rows)
+    sub = spec.scaled(seq_len=rows, prefix=min(spec.prefix, rows))
     case = di.make_case(sub, "cpu")
     for i in range(args.warmup):
         oracle_step(sub, case, 10 + i, rows)
