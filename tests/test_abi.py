@@ -113,6 +113,33 @@ def test_workspace_size_grows_with_rows(L):
     assert sa > 4096 * 16 and sb > sa and sa % 256 == 0
 
 
+def test_header_is_plain_c_and_links(L, tmp_path):
+    """include/dlm.h compiles as pedantic C99 and as C++, and a C program
+    links against the library and calls it (no GPU call: the version)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_dlm.c"
+    src.write_text(
+        '#include "dlm.h"\n'
+        'int main(void) {\n'
+        '    dlm_loss_options_t o = {sizeof(o), DLM_TIME_WEIGHT_NONE, 0.f, DLM_REDUCE_TOKEN_MEAN, 0};\n'
+        '    dlm_layout_t l = {1, 4, 4, 0, 0};\n'
+        '    (void)o; (void)l;\n'
+        '    return dlm_version() == %d ? 0 : 1;\n'
+        '}\n' % L.dlm_version())
+    inc = os.path.join(ROOT, "include")
+    libdir = os.path.dirname(dlm.LIB_PATH)
+    exe = tmp_path / "use_dlm"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc, str(src),
+                    "-L", libdir, "-ldlm", "-Wl,-rpath," + libdir, "-o", str(exe)], check=True)
+    subprocess.run(["g++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-I", inc, "-x", "c++", "-fsyntax-only",
+                    str(src)], check=True)
+    assert subprocess.run([str(exe)]).returncode == 0
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises((ValueError, TypeError)):
