@@ -486,15 +486,15 @@ __device__ __forceinline__ void row_ptrs(const CeParams& P, int q, const uint16_
 }
 
 // Fast path.  Each CTA = one TMA producer warp + WARPS consumer warps; it
-// takes every G-th scored row of the list (G = grid size) and streams it
-// twice through a ring of kStages shared-memory chunks of kChunk elements:
+// takes scored rows of the list by ticket and streams each twice through a
+// ring of kStages shared-memory chunks:
 //   pass 1: bulk loads from HBM with an L2 evict_last policy; per-thread
 //           online (max, sum exp) -> one block combine -> lse of the row;
 //   pass 2: the same chunks again (L2 hits), loaded evict_first; the
 //           gradient g*w*(exp(x - lse) - [v == y]) goes out as 128-bit
 //           stores with an L2 evict_first policy.
-// The producer warp also zero-fills this CTA's share of the unscored rows
-// with bulk shared->global copies from a zeroed shared block, interleaved with
+// The producer warp also zero-fills unscored rows (taken by ticket too) with
+// bulk shared->global copies from a zeroed shared block, interleaved with
 // the scored rows so the zero stream overlaps the consumers' work.
 constexpr int kChunk = 8192;        // bf16 elements per ring stage (16 KB)
 constexpr int kZeroBytes = 4096;    // zero block the producer copies over unscored rows
