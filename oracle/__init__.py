@@ -437,3 +437,76 @@ def linear_rows(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
     for v0 in range(0, V, 16384):
         dH += dZ[:, v0:v0 + 16384] @ bf16_to_f64(W[v0:v0 + 16384])
     return dict(ce=ce, lse=lse, weighted=plan.weight[sample_rows] * ce, dH=dH, plan=plan)
+
+
+def _linear_term(plan: RowPlan, H: np.ndarray, W: np.ndarray, grad_scale: float, want_grads: bool):
+    """One term of a fused-head loss: the scored rows of H (by `plan`) form
+    Z = H_M W^T in double; returns (rows, lse, ce, row_loss, dH, dW), dH over
+    all rows of H (zeros on unscored rows), dW = dZ^T H_M ([V, D])."""
+    rows = np.nonzero(plan.target >= 0)[0]
+    V, D = W.shape
+    Z = linear_logits(H[rows], W)
+    local = np.arange(rows.shape[0], dtype=np.int64)
+    lse, ce = ce_rows(Z, V, local, plan.target[rows])
+    row_loss = np.zeros(plan.target.shape[0], np.float64)
+    row_loss[rows] = plan.weight[rows] * ce
+    dH = dW = None
+    if want_grads:
+        dZ = grad_rows(Z, V, local, plan.target[rows], grad_scale * plan.weight[rows], lse)
+        del Z
+        Hd = bf16_to_f64(H[rows])
+        dH = np.zeros((H.shape[0], D), np.float64)
+        dW = np.zeros((V, D), np.float64)
+        for v0 in range(0, V, 16384):
+            Wd = bf16_to_f64(W[v0:v0 + 16384])
+            dH[rows] += dZ[:, v0:v0 + 16384] @ Wd
+            dW[v0:v0 + 16384] = dZ[:, v0:v0 + 16384].T @ Hd
+    return rows, lse, ce, row_loss, dH, dW
+
+
+def linear_loss_uniform(canvas: Layout, H: np.ndarray, W: np.ndarray, canvas_clean: np.ndarray,
+                        encoder: Optional[Layout], He: Optional[np.ndarray],
+                        enc_clean: Optional[np.ndarray], lam: float, align: int = ALIGNED,
+                        grad_scale: float = 1.0, want_grads: bool = True):
+    """[Gemma] uniform-noise objective through a plain linear head, without a
+    logits tensor ([Axolotl] Cut Cross Entropy carried to uniform noise):
+    canvas term = mean CE of every non-pad canvas target (row i scores token
+    i, or token i+1 of the same unit when shifted) on Z = H W^T; encoder term
+    = lam * mean next-token CE over the clean full sequence on Ze = He W^T.
+    dH, dHe = dZ W, dZe W (zeros on unscored rows); dW = dZ^T H_M + dZe^T He_M,
+    one shared head.  H, He, W: uint16 bf16 bits [T, D], [Te, D], [V, D]."""
+    pc = plan_diffusion(canvas, canvas_clean, None, None, UNIFORM, align)
+    tc = _linear_term(pc, H, W, grad_scale, want_grads)
+    terms = [(pc, tc)]
+    if encoder is not None:
+        pe = plan_encoder(encoder, enc_clean, lam)
+        terms.append((pe, _linear_term(pe, He, W, grad_scale, want_grads)))
+    unit_loss = np.zeros(canvas.n_units, np.float64)
+    for plan, t in terms:
+        np.add.at(unit_loss, plan.unit, t[3])
+    out = dict(loss=float(unit_loss.sum()), unit_loss=unit_loss, rows=tc[0], ce=tc[2], plan=pc)
+    if encoder is not None:
+        out.update(enc_rows=terms[1][1][0], enc_ce=terms[1][1][2], enc_plan=terms[1][0])
+    if want_grads:
+        out.update(dH=tc[4], dW=tc[5] + (terms[1][1][5] if encoder is not None else 0.0))
+        if encoder is not None:
+            out.update(dHe=terms[1][1][4])
+    return out
+
+
+def linear_rows_plan(plan: RowPlan, H: np.ndarray, W: np.ndarray, sample_rows: np.ndarray,
+                     grad_scale: float = 1.0):
+    """Full-size spot check for any row plan (uniform canvas, encoder AR):
+    for a few scored rows, their CE, weight*ce and their row of dH."""
+    sample_rows = np.asarray(sample_rows, np.int64)
+    assert (plan.target[sample_rows] >= 0).all()
+    V, D = W.shape
+    Z = linear_logits(H[sample_rows], W)
+    local = np.arange(sample_rows.shape[0], dtype=np.int64)
+    tgt = plan.target[sample_rows]
+    lse, ce = ce_rows(Z, V, local, tgt)
+    dZ = grad_rows(Z, V, local, tgt, grad_scale * plan.weight[sample_rows], lse)
+    dH = np.zeros((sample_rows.shape[0], D), np.float64)
+    for v0 in range(0, V, 16384):
+        dH += dZ[:, v0:v0 + 16384] @ bf16_to_f64(W[v0:v0 + 16384])
+    return dict(ce=ce, lse=lse, weighted=plan.weight[sample_rows] * ce, dH=dH)

@@ -467,3 +467,118 @@ def test_linear_rows_spot_check_matches_full():
     pos = np.searchsorted(full["rows"], rows)
     assert np.allclose(spot["ce"], full["ce"][pos], rtol=1e-14)
     assert np.allclose(spot["dH"], full["dH"][rows], rtol=1e-12, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# fused lm_head, uniform noise (canvas term + encoder AR term, one head)
+# --------------------------------------------------------------------------
+def _uniform_linear_case(seed, D=64, V=1000):
+    rng = np.random.default_rng(seed)
+    lens = [10, 30, 24]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    canvas = oracle.Layout(3, 0, cu, None)
+    Le = 40                                   # encoder: dense [3, 40] with trailing pads
+    pad = np.zeros(3 * Le, np.uint8)
+    for u, n in enumerate((40, 33, 2)):
+        pad[u * Le + n:(u + 1) * Le] = 1
+    enc = oracle.Layout(3, Le, None, pad)
+    H = bf16_bits_of(rng.standard_normal((64, D)).astype(np.float32))
+    He = bf16_bits_of(rng.standard_normal((3 * Le, D)).astype(np.float32))
+    W = bf16_bits_of((rng.standard_normal((V, D)) * 0.05).astype(np.float32))
+    clean = rng.integers(0, V, 64).astype(np.int32)
+    eclean = rng.integers(0, V, 3 * Le).astype(np.int32)
+    return canvas, enc, H, He, W, clean, eclean
+
+
+@pytest.mark.parametrize("align", [oracle.ALIGNED, oracle.SHIFTED])
+def test_linear_uniform_equals_unfused_on_materialised_logits(align):
+    """The fused uniform loss equals the unfused two-term loss on Z = H W^T
+    and Ze = He W^T (double), with dH = dZ W, dHe = dZe W and dW the sum of
+    both terms' dZ^T H."""
+    canvas, enc, H, He, W, clean, eclean = _uniform_linear_case(21)
+    V = W.shape[0]
+    lam, g = 0.7, 1.5
+    out = oracle.linear_loss_uniform(canvas, H, W, clean, enc, He, eclean, lam, align, grad_scale=g)
+    Hd, Hed, Wd = oracle.bf16_to_f64(H), oracle.bf16_to_f64(He), oracle.bf16_to_f64(W)
+    Z, Ze = Hd @ Wd.T, Hed @ Wd.T
+    loss, unit, tc, te = oracle.loss_uniform(canvas, Z, clean, enc, Ze, eclean, V, lam, align)
+    assert abs(out["loss"] - loss) < 1e-12 * max(1.0, loss)
+    assert np.allclose(out["unit_loss"], unit, rtol=1e-12, atol=1e-15)
+    dZ = oracle.term_grad(Z, V, tc, np.arange(64), g)
+    dZe = oracle.term_grad(Ze, V, te, np.arange(120), g)
+    assert np.allclose(out["dH"], dZ @ Wd, rtol=1e-10, atol=1e-14)
+    assert np.allclose(out["dHe"], dZe @ Wd, rtol=1e-10, atol=1e-14)
+    assert np.allclose(out["dW"], dZ.T @ Hd + dZe.T @ Hed, rtol=1e-10, atol=1e-14)
+    # rows with no target: the last row of each unit when shifted (canvas),
+    # the last non-pad token of each unit and every pad row (encoder)
+    n_c = 64 - (3 if align == oracle.SHIFTED else 0)
+    assert out["rows"].shape[0] == n_c and out["enc_rows"].shape[0] == 39 + 32 + 1
+    unscored = np.ones(120, bool); unscored[out["enc_rows"]] = False
+    assert (out["dHe"][unscored] == 0).all()
+
+
+def test_linear_uniform_finite_differences():
+    """d loss / d(H, He, W) of the two-term loss against central differences
+    (a transposed operand or a dropped encoder share of dW fails)."""
+    rng = np.random.default_rng(22)
+    D, V = 3, 5
+    canvas = oracle.Layout(1, 4, None, None)
+    enc = oracle.Layout(1, 5, None, None)
+    Hf = rng.standard_normal((4, D))
+    Hef = rng.standard_normal((5, D))
+    Wf = rng.standard_normal((V, D)) * 0.5
+    clean = rng.integers(0, V, 4).astype(np.int32)
+    eclean = rng.integers(0, V, 5).astype(np.int32)
+    lam = 0.3
+
+    def loss_of(Hm, Hem, Wm):
+        return oracle.loss_uniform(canvas, Hm @ Wm.T, clean, enc, Hem @ Wm.T, eclean, V, lam)
+
+    loss, _, tc, te = loss_of(Hf, Hef, Wf)
+    dZ = oracle.term_grad(Hf @ Wf.T, V, tc, np.arange(4), 1.0)
+    dZe = oracle.term_grad(Hef @ Wf.T, V, te, np.arange(5), 1.0)
+    grads = (dZ @ Wf, dZe @ Wf, dZ.T @ Hf + dZe.T @ Hef)
+    h = 1e-6
+    args = [Hf, Hef, Wf]
+    for which, G in enumerate(grads):
+        fd = np.zeros_like(args[which])
+        for idx in np.ndindex(*fd.shape):
+            ap = [a.copy() for a in args]; ap[which][idx] += h
+            am = [a.copy() for a in args]; am[which][idx] -= h
+            fd[idx] = (loss_of(*ap)[0] - loss_of(*am)[0]) / (2 * h)
+        assert np.abs(fd - G).max() < 1e-7
+    # the oracle's fused entry on the same inputs rounded to bf16
+    Hb, Heb, Wb = (bf16_bits_of(a.astype(np.float32)) for a in (Hf, Hef, Wf))
+    out = oracle.linear_loss_uniform(canvas, Hb, Wb, clean, enc, Heb, eclean, lam)
+    Hq, Heq, Wq = (oracle.bf16_to_f64(a) for a in (Hb, Heb, Wb))
+    lq, _, tcq, teq = loss_of(Hq, Heq, Wq)
+    dZq = oracle.term_grad(Hq @ Wq.T, V, tcq, np.arange(4), 1.0)
+    dZeq = oracle.term_grad(Heq @ Wq.T, V, teq, np.arange(5), 1.0)
+    assert abs(out["loss"] - lq) < 1e-12
+    assert np.allclose(out["dH"], dZq @ Wq, atol=1e-13)
+    assert np.allclose(out["dHe"], dZeq @ Wq, atol=1e-13)
+    assert np.allclose(out["dW"], dZq.T @ Hq + dZeq.T @ Heq, atol=1e-13)
+
+
+def test_linear_uniform_without_encoder_is_lambda_zero():
+    canvas, enc, H, He, W, clean, eclean = _uniform_linear_case(23, D=32, V=300)
+    a = oracle.linear_loss_uniform(canvas, H, W, clean, None, None, None, 0.0)
+    b = oracle.linear_loss_uniform(canvas, H, W, clean, enc, He, eclean, 0.0)
+    assert a["loss"] == b["loss"]
+    assert np.array_equal(a["dH"], b["dH"]) and np.array_equal(a["dW"], b["dW"])
+    assert (b["dHe"] == 0).all()
+    # every canvas row is scored with weight 1/64 (aligned, no pads)
+    assert a["rows"].shape[0] == 64 and np.allclose(a["plan"].weight, 1 / 64)
+
+
+def test_linear_rows_plan_spot_check_matches_full():
+    canvas, enc, H, He, W, clean, eclean = _uniform_linear_case(24, D=32, V=300)
+    full = oracle.linear_loss_uniform(canvas, H, W, clean, enc, He, eclean, 0.5, oracle.SHIFTED, 0.25)
+    rows = full["enc_rows"][::5]
+    spot = oracle.linear_rows_plan(full["enc_plan"], He, W, rows, 0.25)
+    pos = np.searchsorted(full["enc_rows"], rows)
+    assert np.allclose(spot["ce"], full["enc_ce"][pos], rtol=1e-14)
+    assert np.allclose(spot["dH"], full["dHe"][rows], rtol=1e-12, atol=1e-15)
+    rows = full["rows"][1::4]
+    spot = oracle.linear_rows_plan(full["plan"], H, W, rows, 0.25)
+    assert np.allclose(spot["dH"], full["dH"][rows], rtol=1e-12, atol=1e-15)
