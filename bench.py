@@ -368,7 +368,9 @@ def run_ours(args):
 
 def run_linear(args, spec, dev, rank, world):
     """The fused lm_head workload: time draw, corruption, and the loss from
-    hidden states and the head (dlm_linear_loss_fwd_bwd, dH and dW)."""
+    hidden states and the head (dlm_linear_loss_fwd_bwd, dH and dW; uniform
+    workloads: dlm_linear_loss_uniform_fwd_bwd, canvas and encoder hidden
+    states against one head, dH, dH_enc and dW)."""
     import torch
     import torch.distributed as dist
 
@@ -377,9 +379,16 @@ def run_linear(args, spec, dev, rank, world):
 
     case = di.make_case(spec, dev, seed=spec.data_seed + rank)
     T, D, V = case.n_tokens, spec.d_model, spec.vocab
-    lay = dlm.make_layout(case.n_units, 0, case.cu_seqlens, None, n_tokens=T)
     out = None
     align = dlm.SHIFTED if args.align == "shifted" else dlm.ALIGNED
+    uniform = spec.mode == dlm.UNIFORM
+    if uniform:
+        B, C, P = case.n_units, case.seq_len, spec.prefix
+        lay = dlm.make_layout(B, C)
+        enc = dlm.make_layout(B, P + C)
+        T = B * C + B * (P + C)
+    else:
+        lay = dlm.make_layout(case.n_units, 0, case.cu_seqlens, None, n_tokens=T)
 
     def step(seed, ev=None):
         nonlocal out
@@ -387,7 +396,12 @@ def run_linear(args, spec, dev, rank, world):
         _, corr = dlm.corrupt(lay, case.clean, p, spec.mode, spec.mask_id, V, seed)
         if ev is not None:
             ev[0].record()
-        out = dlm.linear_loss_fwd_bwd(lay, case.hidden, case.weight, case.clean, corr, p, out=out, align=align)
+        if uniform:
+            out = dlm.linear_loss_uniform_fwd_bwd(lay, case.hidden, case.weight, case.clean, enc, case.enc_hidden,
+                                                  case.enc_clean, enc_ar_weight=spec.enc_ar_weight, align=align,
+                                                  out=out)
+        else:
+            out = dlm.linear_loss_fwd_bwd(lay, case.hidden, case.weight, case.clean, corr, p, out=out, align=align)
         if ev is not None:
             ev[1].record()
         return corr
@@ -420,7 +434,7 @@ def run_linear(args, spec, dev, rank, world):
     call_ms = sum(a.elapsed_time(b) for a, b in evs) / K
     clk = clocks.stop() if rank == 0 else None
     scored = 0
-    for i in range(K):
+    for i in range(K if not uniform else 0):
         t, p = dlm.sample_t(1000 + i, case.n_units, spec.mode, spec.eps)
         _, corr = dlm.corrupt(lay, case.clean, p, spec.mode, spec.mask_id, V, 1000 + i)
         scored += int(corr.sum().item())
@@ -429,6 +443,10 @@ def run_linear(args, spec, dev, rank, world):
             cu = case.cu_seqlens.to(torch.int64)
             first = cu[:-1][cu[1:] > cu[:-1]]
             scored -= int(corr[first].sum().item())
+    if uniform:
+        # every canvas target (each unit's first token is none when shifted)
+        # and every encoder next-token pair
+        scored = K * (B * (C - (1 if align == dlm.SHIFTED else 0)) + B * (P + C - 1))
     ms, call_ms, scored_all = reduce_over_ranks(ms, call_ms, scored, dev)
     value = scored_all / (ms / 1e3)
     M = scored_all / world / K
@@ -442,7 +460,8 @@ def run_linear(args, spec, dev, rank, world):
     achieved = flops / (call_ms / 1e3) / 1e12
     roof = {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
             "frac": achieved / sustained, "traffic": None,
-            "kernel": "k_gemm (the whole dlm_linear_loss_fwd_bwd call: 6 GEMMs-worth of algorithmic flops "
+            "kernel": f"k_gemm (the whole {'dlm_linear_loss_uniform_fwd_bwd' if uniform else 'dlm_linear_loss_fwd_bwd'}"
+                      " call: 6 GEMMs-worth of algorithmic flops "
                       "6*M*D*V; executed 8*M*D*V with the backward recompute)",
             "algorithmic_flops_per_call": flops, "launch_ms": call_ms,
             "frac_of_burst_peak": achieved / bf16, "peak_source": f"{kind} bf16 sustained (burst in frac_of_burst_peak)"}
@@ -455,7 +474,7 @@ def run_linear(args, spec, dev, rank, world):
            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "bf16", "data": "synthetic",
            "config": {"workload": spec.key, "description": spec.description, "align": args.align,
-                      "tokens": T, "d_model": D,
+                      "tokens": T, "d_model": D, "encoder_ar_weight": spec.enc_ar_weight if uniform else None,
                       "vocab": V, "documents": case.n_units, "parallelism": f"replicas{world}",
                       "scored_tokens": scored_all, "l2": "inputs larger than L2 (W %.2f GB)" % (V * D * 2 / 1e9)},
            "roofline": roof, "cpu_baseline": None, "clocks": clk, "e2e": None,

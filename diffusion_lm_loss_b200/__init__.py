@@ -42,7 +42,8 @@ STATUS = {0: "DLM_OK", 1: "DLM_ERR_INVALID_ARGUMENT", 2: "DLM_ERR_UNSUPPORTED",
 EXPORTS = ("dlm_status_string", "dlm_last_cuda_error", "dlm_version", "dlm_sample_t", "dlm_corrupt",
            "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_loss_fwd_bwd_ex", "dlm_loss_fwd_bwd_static",
            "dlm_linear_loss_workspace_size",
-           "dlm_linear_loss_fwd_bwd", "dlm_linear_loss_fwd_bwd_ex", "dlm_get_device_status", "dlm_selftest_bounded_wait")
+           "dlm_linear_loss_fwd_bwd", "dlm_linear_loss_fwd_bwd_ex", "dlm_linear_loss_uniform_workspace_size",
+           "dlm_linear_loss_uniform_fwd_bwd", "dlm_get_device_status", "dlm_selftest_bounded_wait")
 
 
 class DlmError(RuntimeError):
@@ -138,6 +139,11 @@ def lib():
     L.dlm_linear_loss_fwd_bwd_ex.restype = ctypes.c_int
     L.dlm_linear_loss_fwd_bwd_ex.argtypes = [lp, vp, vp, i32, i32, vp, vp, vp, i32, f32, vp, vp, vp, vp,
                                              vp, sz, vp]
+    L.dlm_linear_loss_uniform_workspace_size.restype = sz
+    L.dlm_linear_loss_uniform_workspace_size.argtypes = [lp, lp, i32, i32]
+    L.dlm_linear_loss_uniform_fwd_bwd.restype = ctypes.c_int
+    L.dlm_linear_loss_uniform_fwd_bwd.argtypes = [lp, vp, lp, vp, vp, vp, i32, i32, vp, i32, f32, f32,
+                                                  vp, vp, vp, vp, vp, vp, sz, vp]
     L.dlm_selftest_bounded_wait.restype = ctypes.c_int
     L.dlm_selftest_bounded_wait.argtypes = [u64, vp, vp]
     L.dlm_get_device_status.restype = ctypes.c_int
@@ -269,6 +275,7 @@ class LinearOut:
     d_hidden: torch.Tensor
     d_weight: Optional[torch.Tensor]
     workspace: torch.Tensor
+    d_enc_hidden: Optional[torch.Tensor] = None
 
     def device_status(self) -> int:
         return device_status(self.workspace)
@@ -311,6 +318,53 @@ def linear_loss_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: torch.Tens
             _ptr(p), align, grad_scale, _ptr(out.loss), _ptr(out.unit_loss), _ptr(out.d_hidden),
             _ptr(out.d_weight), _ptr(out.workspace), out.workspace.numel(), _stream()),
             "dlm_linear_loss_fwd_bwd_ex")
+    return out
+
+
+def linear_loss_uniform_workspace_size(layout: Layout, enc_layout: Optional[Layout], d_model: int,
+                                       vocab: int) -> int:
+    enc = ctypes.byref(enc_layout) if enc_layout is not None else None
+    return int(lib().dlm_linear_loss_uniform_workspace_size(ctypes.byref(layout), enc, d_model, vocab))
+
+
+def linear_loss_uniform_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: torch.Tensor,
+                                clean_ids: torch.Tensor, enc_layout: Optional[Layout] = None,
+                                enc_hidden: Optional[torch.Tensor] = None,
+                                enc_ids: Optional[torch.Tensor] = None, enc_ar_weight: float = 1.0,
+                                align: int = ALIGNED, grad_scale: float = 1.0, want_d_weight: bool = True,
+                                out: Optional[LinearOut] = None) -> LinearOut:
+    """Fused lm_head + uniform-noise loss with the optional encoder
+    next-token term (see dlm_linear_loss_uniform_fwd_bwd)."""
+    _check(hidden, torch.bfloat16, "hidden")
+    _check(weight, torch.bfloat16, "weight")
+    if not (hidden.is_contiguous() and weight.is_contiguous()):
+        raise ValueError("hidden and weight must be contiguous")
+    T, D = hidden.shape
+    V, D2 = weight.shape
+    if D != D2:
+        raise ValueError("hidden / weight d_model mismatch")
+    if enc_layout is not None:
+        if enc_hidden is None or enc_ids is None:
+            raise ValueError("enc_layout needs enc_hidden and enc_ids")
+        _check(enc_hidden, torch.bfloat16, "enc_hidden")
+        if not enc_hidden.is_contiguous() or enc_hidden.shape[1] != D:
+            raise ValueError("enc_hidden must be contiguous [enc_tokens, d_model]")
+    dev = hidden.device
+    if out is None:
+        ws = torch.empty(linear_loss_uniform_workspace_size(layout, enc_layout, D, V), dtype=torch.uint8,
+                         device=dev)
+        out = LinearOut(torch.empty(1, dtype=torch.float32, device=dev),
+                        torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
+                        torch.empty_like(hidden),
+                        torch.empty_like(weight) if want_d_weight else None, ws,
+                        torch.empty_like(enc_hidden) if enc_layout is not None else None)
+    enc = ctypes.byref(enc_layout) if enc_layout is not None else None
+    _ok(lib().dlm_linear_loss_uniform_fwd_bwd(
+        ctypes.byref(layout), _ptr(hidden), enc, _ptr(enc_hidden), _ptr(enc_ids), _ptr(weight), D, V,
+        _ptr(clean_ids), align, enc_ar_weight, grad_scale, _ptr(out.loss), _ptr(out.unit_loss),
+        _ptr(out.d_hidden), _ptr(out.d_enc_hidden), _ptr(out.d_weight), _ptr(out.workspace),
+        out.workspace.numel(), _stream()),
+        "dlm_linear_loss_uniform_fwd_bwd")
     return out
 
 

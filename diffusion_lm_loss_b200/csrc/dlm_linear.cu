@@ -1,8 +1,13 @@
-// dlm_linear.cu -- the absorbing-mask loss computed from hidden states and a
+// dlm_linear.cu -- the diffusion loss computed from hidden states and a
 // linear output head, logits never written to memory ("Native diffusion
 // language-model training", Adapters, merging and inference: Cut Cross
 // Entropy -- full-vocabulary CE from hidden states, aligned targets, plain
-// linear head).  The head is a dense contraction, so it runs on the 5th-gen
+// linear head).  Absorbing noise (aligned or shifted rows), and uniform noise
+// with its encoder next-token term ("diffusiongemma-26B-A4B-it-ALWAYS-THINK",
+// Finetuning notes): the row plan lists the scored rows of both hidden-state
+// arrays (canvas rows first, then encoder rows) and everything after the
+// gather sees one set of M rows against one head.  The head is a dense
+// contraction, so it runs on the 5th-gen
 // tensor cores: tcgen05.mma from shared memory into tensor-memory
 // accumulators, operands brought in by TMA tile loads (no multicast).
 //
@@ -444,17 +449,20 @@ k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensor
 // ---------------------------------------------------------------------------
 // small kernels around the GEMMs
 // ---------------------------------------------------------------------------
-// H_M[m] = H[list[m].row] for m < M, zero rows up to round_up(M, 256) (the
-// height of a paired tile).
-__global__ void k_gather(const WsHeader* hdr, const int4* list, const uint16_t* __restrict__ H, int D,
-                         uint16_t* __restrict__ HM) {
+// H_M[m] = row list[m].row of the hidden states for m < M, zero rows up to
+// round_up(M, 256) (the height of a paired tile).  Rows [0, Ta) are rows of H,
+// rows from Ta on are rows of He (the encoder's hidden states, uniform noise).
+__global__ void k_gather(const WsHeader* hdr, const int4* list, const uint16_t* __restrict__ H,
+                         const uint16_t* __restrict__ He, int64_t Ta, int D, uint16_t* __restrict__ HM) {
     const int M = hdr->n_scored;
     const int Mp = round_up_dev(M, kRowPad);
     const int vecs = D / 8;
     for (int r = blockIdx.x; r < Mp; r += gridDim.x) {
         uint4* dst = reinterpret_cast<uint4*>(HM + size_t(r) * D);
         if (r < M) {
-            const uint4* src = reinterpret_cast<const uint4*>(H + size_t(__ldg(&list[r].x)) * D);
+            const int64_t q = __ldg(&list[r].x);
+            const uint16_t* row = q < Ta ? H + size_t(q) * D : He + size_t(q - Ta) * D;
+            const uint4* src = reinterpret_cast<const uint4*>(row);
             for (int i = threadIdx.x; i < vecs; i += blockDim.x) dst[i] = __ldg(src + i);
         } else {
             for (int i = threadIdx.x; i < vecs; i += blockDim.x) dst[i] = make_uint4(0, 0, 0, 0);
@@ -505,15 +513,17 @@ __global__ void k_lse(const WsHeader* hdr, const int4* list, const float2* __res
     }
 }
 
-// d_hidden[row] = bf16(dH_M[m]) for the masked rows, 0 for all other rows.
+// d_hidden[row] = bf16(dH_M[m]) for the masked rows, 0 for all other rows
+// (rows from Ta on go to d_enc_hidden[row - Ta]).
 __global__ void k_scatter_dh(const WsHeader* hdr, const int4* list, const float* __restrict__ dh, int D,
-                             uint16_t* __restrict__ d_hidden) {
+                             int64_t Ta, uint16_t* __restrict__ d_hidden, uint16_t* __restrict__ d_enc_hidden) {
     const int M = hdr->n_scored;
     const int R = hdr->n_rows;
     const int vecs = D / 8;
     for (int i = blockIdx.x; i < R; i += gridDim.x) {
-        const int row = list[i].x;
-        uint4* dst = reinterpret_cast<uint4*>(d_hidden + size_t(row) * D);
+        const int64_t row = list[i].x;
+        uint4* dst = reinterpret_cast<uint4*>(row < Ta ? d_hidden + size_t(row) * D
+                                                        : d_enc_hidden + size_t(row - Ta) * D);
         if (i < M) {
             const float4* src = reinterpret_cast<const float4*>(dh + size_t(i) * D);
             for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
@@ -641,23 +651,51 @@ extern "C" size_t dlm_linear_loss_workspace_size(const dlm_layout_t* layout, int
     return lin_ws(layout->n_tokens, layout->n_units, d_model, vocab).total;
 }
 
+extern "C" size_t dlm_linear_loss_uniform_workspace_size(const dlm_layout_t* layout,
+                                                         const dlm_layout_t* enc_layout, int32_t d_model,
+                                                         int32_t vocab) {
+    if (!layout || d_model <= 0 || vocab <= 0) return 0;
+    const int64_t rows = layout->n_tokens + (enc_layout ? enc_layout->n_tokens : 0);
+    return lin_ws(rows, layout->n_units, d_model, vocab).total;
+}
+
+// Both entry families: absorbing noise (corrupted + p select and weight the
+// rows; no encoder) or uniform noise (every canvas target scored, plus the
+// encoder's next-token rows when enc_layout is given).
 static dlm_status_t linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16_t* hidden,
                                         const uint16_t* weight, int32_t d_model, int32_t vocab,
                                         const int32_t* clean_ids, const uint8_t* corrupted, const float* p,
-                                        int32_t align, float grad_scale, float* loss, float* unit_loss,
-                                        uint16_t* d_hidden, uint16_t* d_weight, void* workspace,
-                                        size_t workspace_bytes, dlm_stream_t stream) {
+                                        int32_t mode, int32_t align, const dlm_layout_t* enc_layout,
+                                        const uint16_t* enc_hidden, const int32_t* enc_ids,
+                                        float enc_ar_weight, float grad_scale, float* loss, float* unit_loss,
+                                        uint16_t* d_hidden, uint16_t* d_enc_hidden, uint16_t* d_weight,
+                                        void* workspace, size_t workspace_bytes, dlm_stream_t stream) {
     if (!layout_ok(layout)) return DLM_ERR_INVALID_ARGUMENT;
+    if (mode != DLM_ABSORBING && mode != DLM_UNIFORM) return DLM_ERR_INVALID_ARGUMENT;
     if (align != DLM_ALIGNED && align != DLM_SHIFTED) return DLM_ERR_INVALID_ARGUMENT;
     if (d_model <= 0 || d_model % 64 != 0 || vocab <= 0 || vocab % 8 != 0) return DLM_ERR_INVALID_ARGUMENT;
     if (!loss || !workspace) return DLM_ERR_INVALID_ARGUMENT;
+    const bool has_enc = enc_layout != nullptr;
+    if (has_enc) {
+        if (mode != DLM_UNIFORM) return DLM_ERR_INVALID_ARGUMENT;
+        if (!layout_ok(enc_layout) || enc_layout->n_units != layout->n_units) return DLM_ERR_INVALID_ARGUMENT;
+        if (enc_layout->n_tokens > 0 &&
+            (!enc_hidden || !enc_ids || !d_enc_hidden || !weight ||
+             (!enc_layout->cu_seqlens && enc_layout->seq_len == 0)))
+            return DLM_ERR_INVALID_ARGUMENT;
+        if (!aligned16(enc_hidden) || !aligned16(d_enc_hidden)) return DLM_ERR_INVALID_ARGUMENT;
+    }
     const int64_t T = layout->n_tokens;
-    if (T > 0 && (!hidden || !weight || !clean_ids || !corrupted || !p || !d_hidden)) return DLM_ERR_INVALID_ARGUMENT;
+    const int64_t Te = has_enc ? enc_layout->n_tokens : 0;
+    const int64_t R = T + Te;
+    if (R >= (int64_t(1) << 31)) return DLM_ERR_INVALID_ARGUMENT;
+    if (T > 0 && (!hidden || !weight || !clean_ids || !d_hidden)) return DLM_ERR_INVALID_ARGUMENT;
+    if (T > 0 && mode == DLM_ABSORBING && (!corrupted || !p)) return DLM_ERR_INVALID_ARGUMENT;
     if (T > 0 && !layout->cu_seqlens && layout->seq_len == 0) return DLM_ERR_INVALID_ARGUMENT;
     if (!aligned16(hidden) || !aligned16(weight) || !aligned16(d_hidden) || (d_weight && !aligned16(d_weight)))
         return DLM_ERR_INVALID_ARGUMENT;
     if (reinterpret_cast<uintptr_t>(workspace) % 1024) return DLM_ERR_INVALID_ARGUMENT;
-    const LinWs W = lin_ws(T, layout->n_units, d_model, vocab);
+    const LinWs W = lin_ws(R, layout->n_units, d_model, vocab);
     if (workspace_bytes < W.total) return DLM_ERR_WORKSPACE_TOO_SMALL;
     dlm_status_t st = check_device();
     if (st != DLM_OK) return st;
@@ -675,17 +713,19 @@ static dlm_status_t linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16
     uint16_t* dz = reinterpret_cast<uint16_t*>(ws + W.dz);
     float* dh = reinterpret_cast<float*>(ws + W.dh);
 
-    // 1. which rows are scored, their targets and weights (absorbing; row i
-    //    scores token i, or token i+1 of the same unit when shifted)
-    if ((st = launch_plan(layout, clean_ids, corrupted, p, DLM_ABSORBING, align, nullptr, nullptr, 0.f,
+    // 1. which rows are scored, their targets and weights (row i scores token
+    //    i, or token i+1 of the same unit when shifted; absorbing noise only
+    //    the corrupted ones; encoder rows after the canvas rows)
+    const dlm_layout_t* lb = has_enc ? enc_layout : nullptr;
+    if ((st = launch_plan(layout, clean_ids, corrupted, p, mode, align, lb, enc_ids, enc_ar_weight,
                           vocab, hdr, list, s)) != DLM_OK)
         return st;
-    if (T == 0) {
+    if (R == 0) {
         if (d_weight) {
             cudaError_t e = cudaMemsetAsync(d_weight, 0, size_t(vocab) * d_model * 2, s);
             if (e != cudaSuccess) return cuda_status(e, "cudaMemsetAsync d_weight");
         }
-        return launch_reduce(layout, nullptr, row_loss, unit_acc, unit_loss, loss, hdr, s);
+        return launch_reduce(layout, lb, row_loss, unit_acc, unit_loss, loss, hdr, s);
     }
 
     int dev = 0, sms = 148;
@@ -693,7 +733,7 @@ static dlm_status_t linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
     // 2. gather the masked rows of H (zero padding to a 128-row tile)
-    k_gather<<<sms * 4, 256, 0, s>>>(hdr, list, hidden, d_model, HM);
+    k_gather<<<sms * 4, 256, 0, s>>>(hdr, list, hidden, enc_hidden, T, d_model, HM);
     if ((st = last_launch_status("k_gather launch")) != DLM_OK) return st;
 
     // tensor maps (shapes are host-known upper bounds; the kernels read M)
@@ -754,9 +794,9 @@ static dlm_status_t linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16
     }
 
     // 5. d_hidden (zero rows for unscored tokens) and the reductions
-    k_scatter_dh<<<sms * 4, 256, 0, s>>>(hdr, list, dh, d_model, d_hidden);
+    k_scatter_dh<<<sms * 4, 256, 0, s>>>(hdr, list, dh, d_model, T, d_hidden, d_enc_hidden);
     if ((st = last_launch_status("k_scatter_dh launch")) != DLM_OK) return st;
-    return launch_reduce(layout, nullptr, row_loss, unit_acc, unit_loss, loss, hdr, s);
+    return launch_reduce(layout, lb, row_loss, unit_acc, unit_loss, loss, hdr, s);
 }
 
 extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16_t* hidden,
@@ -766,9 +806,9 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd(const dlm_layout_t* layout, cons
                                                 float* unit_loss, uint16_t* d_hidden, uint16_t* d_weight,
                                                 void* workspace, size_t workspace_bytes, dlm_stream_t stream) {
     DLM_NVTX("dlm_linear_loss_fwd_bwd");
-    return linear_loss_fwd_bwd(layout, hidden, weight, d_model, vocab, clean_ids, corrupted, p, DLM_ALIGNED,
-                               grad_scale, loss, unit_loss, d_hidden, d_weight, workspace, workspace_bytes,
-                               stream);
+    return linear_loss_fwd_bwd(layout, hidden, weight, d_model, vocab, clean_ids, corrupted, p, DLM_ABSORBING,
+                               DLM_ALIGNED, nullptr, nullptr, nullptr, 0.f, grad_scale, loss, unit_loss,
+                               d_hidden, nullptr, d_weight, workspace, workspace_bytes, stream);
 }
 
 extern "C" dlm_status_t dlm_linear_loss_fwd_bwd_ex(const dlm_layout_t* layout, const uint16_t* hidden,
@@ -779,7 +819,22 @@ extern "C" dlm_status_t dlm_linear_loss_fwd_bwd_ex(const dlm_layout_t* layout, c
                                                    uint16_t* d_weight, void* workspace, size_t workspace_bytes,
                                                    dlm_stream_t stream) {
     DLM_NVTX("dlm_linear_loss_fwd_bwd_ex");
-    return linear_loss_fwd_bwd(layout, hidden, weight, d_model, vocab, clean_ids, corrupted, p, align,
-                               grad_scale, loss, unit_loss, d_hidden, d_weight, workspace, workspace_bytes,
-                               stream);
+    return linear_loss_fwd_bwd(layout, hidden, weight, d_model, vocab, clean_ids, corrupted, p, DLM_ABSORBING,
+                               align, nullptr, nullptr, nullptr, 0.f, grad_scale, loss, unit_loss, d_hidden,
+                               nullptr, d_weight, workspace, workspace_bytes, stream);
+}
+
+extern "C" dlm_status_t dlm_linear_loss_uniform_fwd_bwd(const dlm_layout_t* layout, const uint16_t* hidden,
+                                                        const dlm_layout_t* enc_layout, const uint16_t* enc_hidden,
+                                                        const int32_t* enc_ids, const uint16_t* weight,
+                                                        int32_t d_model, int32_t vocab, const int32_t* clean_ids,
+                                                        int32_t align, float enc_ar_weight, float grad_scale,
+                                                        float* loss, float* unit_loss, uint16_t* d_hidden,
+                                                        uint16_t* d_enc_hidden, uint16_t* d_weight,
+                                                        void* workspace, size_t workspace_bytes,
+                                                        dlm_stream_t stream) {
+    DLM_NVTX("dlm_linear_loss_uniform_fwd_bwd");
+    return linear_loss_fwd_bwd(layout, hidden, weight, d_model, vocab, clean_ids, nullptr, nullptr, DLM_UNIFORM,
+                               align, enc_layout, enc_hidden, enc_ids, enc_ar_weight, grad_scale, loss,
+                               unit_loss, d_hidden, d_enc_hidden, d_weight, workspace, workspace_bytes, stream);
 }

@@ -20,7 +20,8 @@ Draw order for a given seed (a fixed recipe, so a seed names one input):
   1. packed-document lengths (packed workloads only; CPU generator);
   2. clean ids;
   3. logits (diffusion / canvas), then encoder logits (uniform workloads),
-     or hidden states then head weights (linear workloads).
+     or hidden states then head weights (linear workloads; uniform linear
+     workloads: canvas hidden states, encoder hidden states, head weights).
 Normal draws are generated in fp32 in row blocks and rounded to bf16.
 "N(0, s)" means standard deviation s.
 """
@@ -100,6 +101,13 @@ WORKLOADS = {
         data_seed=6,
         description="DiffusionGemma-like uniform-token noise, B=1, prefix 256 + canvas 512, "
                     "V=262144 (every row scored; 0.67 GB of logits)"),
+    "lin_unif_b4_p512_c1024_d4096_v262144": Spec(
+        "lin_unif_b4_p512_c1024_d4096_v262144", "linear", UNIFORM, ALIGNED, vocab=262144,
+        mask_id=-1, ids_high=262143, n_units=4, seq_len=1024, prefix=512, d_model=4096,
+        h_std=1.0, w_std=0.02, enc_ar_weight=1.0, data_seed=7,
+        description="DiffusionGemma-like uniform-token noise through a fused lm_head: B=4, "
+                    "prefix 512 + canvas 1024, D=4096, V=262144, canvas and encoder hidden "
+                    "states against one head, encoder AR weight 1"),
     "lin_t4096_d4096_v32768": Spec(
         "lin_t4096_d4096_v32768", "linear", ABSORBING, ALIGNED, vocab=32768,
         mask_id=32767, ids_high=32000, n_tokens_packed=4096, d_model=4096,
@@ -148,8 +156,9 @@ class Case:
     logits: Optional[torch.Tensor] = None       # bf16 [rows, V]
     enc_clean: Optional[torch.Tensor] = None    # int32 [n_units*(prefix+seq_len)]
     enc_logits: Optional[torch.Tensor] = None   # bf16
-    hidden: Optional[torch.Tensor] = None       # bf16 [T, D]
+    hidden: Optional[torch.Tensor] = None       # bf16 [T, D] (canvas rows for uniform)
     weight: Optional[torch.Tensor] = None       # bf16 [V, D]
+    enc_hidden: Optional[torch.Tensor] = None   # bf16 [n_units*(prefix+seq_len), D]
     extra: dict = field(default_factory=dict)
 
     @property
@@ -167,6 +176,18 @@ def make_case(spec: Spec, device="cpu", seed: Optional[int] = None,
     gen.manual_seed(seed)
     cpu_gen = torch.Generator()
     cpu_gen.manual_seed(seed)
+
+    if spec.kind == "linear" and spec.mode == UNIFORM:
+        B, C, P = spec.n_units, spec.seq_len, spec.prefix
+        full = torch.randint(0, spec.ids_high + 1, (B, P + C), generator=gen, device=dev,
+                             dtype=torch.int64).to(torch.int32)
+        canvas = full[:, P:].contiguous().reshape(-1)
+        case = Case(spec, B, C, None, None, canvas, enc_clean=full.reshape(-1).contiguous())
+        if with_tensors:
+            case.hidden = _normal_bf16(B * C, spec.d_model, spec.h_std, gen, dev)
+            case.enc_hidden = _normal_bf16(B * (P + C), spec.d_model, spec.h_std, gen, dev)
+            case.weight = _normal_bf16(spec.vocab, spec.d_model, spec.w_std, gen, dev)
+        return case
 
     if spec.kind == "linear":
         lens = doc_lengths(spec.n_tokens_packed, spec.doc_mean, spec.doc_min, spec.doc_max, cpu_gen)

@@ -15,7 +15,8 @@
  *   dlm_linear_loss_fwd_bwd  the same loss from hidden states and a linear
  *                            output head, logits never materialised
  *                            (dlm_linear_loss_fwd_bwd_ex: aligned or shifted
- *                            targets)
+ *                            targets; dlm_linear_loss_uniform_fwd_bwd: the
+ *                            uniform-noise loss with its encoder term)
  *
  * The method (page title, section):
  *   "LLaDA-8B-MDLM-LoRA", Training table, row "Objective": t ~ U(0,1) per
@@ -316,6 +317,53 @@ DLM_API dlm_status_t dlm_linear_loss_fwd_bwd_ex(const dlm_layout_t *layout, cons
                                         float *loss, float *unit_loss, uint16_t *d_hidden,
                                         uint16_t *d_weight, void *workspace, size_t workspace_bytes,
                                         dlm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * dlm_linear_loss_uniform_fwd_bwd -- the uniform-noise loss of
+ * dlm_loss_fwd_bwd (DLM_UNIFORM) from hidden states and a linear output
+ * head, logits never materialised: the DiffusionGemma objective
+ * ("diffusiongemma-26B-A4B-it-ALWAYS-THINK", Finetuning notes: canvas CE +
+ * encoder_loss_weight * encoder AR CE) through the Cut Cross Entropy form of
+ * "Native diffusion language-model training", Adapters, merging and
+ * inference.  The page describes that form for absorbing noise and aligned
+ * targets only; this call carries the unfused uniform loss over unchanged.
+ *   Canvas term: every non-pad canvas target is scored (row i scores token
+ *     i, or token i + 1 of the same unit with DLM_SHIFTED), w = 1 / (number
+ *     of scored canvas rows), logits = hidden @ weight^T.
+ *   Encoder term (enc_layout != NULL): row i of enc_hidden scores enc_ids[i+1]
+ *     of the same unit (non-pad), w = enc_ar_weight / (number of such rows),
+ *     logits = enc_hidden @ weight^T with the same head.
+ *   hidden [layout.n_tokens, d_model], enc_hidden [enc_layout.n_tokens,
+ *   d_model], weight [vocab, d_model]: bf16 row-major.  clean_ids
+ *   [layout.n_tokens] (the canvas targets), enc_ids [enc_layout.n_tokens].
+ *   No corrupted mask or p: uniform noise scores every canvas position.
+ *   d_hidden, d_enc_hidden: bf16, same shapes as hidden / enc_hidden
+ *   (written; rows with no target = 0).  d_weight [vocab, d_model] bf16, the
+ *   sum of both terms' contributions (written), or NULL to skip it.
+ *   enc_layout.n_units must equal layout.n_units (unit u of the canvas is
+ *   unit u of the encoder sequence); unit_loss[u] sums both terms of unit u.
+ *   Requires d_model % 64 == 0, vocab % 8 == 0, 16-byte aligned pointers and
+ *   fewer than 2^31 rows in total; otherwise DLM_ERR_INVALID_ARGUMENT before
+ *   anything is enqueued.  Ids outside [0, vocab) set DLM_DEV_BAD_TOKEN_ID in
+ *   the device status word; their rows are skipped.
+ * Workspace: dlm_linear_loss_uniform_workspace_size(layout, enc_layout,
+ * d_model, vocab) bytes, 1024-byte aligned (enc_layout may be NULL).
+ * ---------------------------------------------------------------------- */
+DLM_API size_t dlm_linear_loss_uniform_workspace_size(const dlm_layout_t *layout,
+                                              const dlm_layout_t *enc_layout,
+                                              int32_t d_model, int32_t vocab);
+
+DLM_API dlm_status_t dlm_linear_loss_uniform_fwd_bwd(const dlm_layout_t *layout,
+                                             const uint16_t *hidden,
+                                             const dlm_layout_t *enc_layout,
+                                             const uint16_t *enc_hidden, const int32_t *enc_ids,
+                                             const uint16_t *weight, int32_t d_model,
+                                             int32_t vocab, const int32_t *clean_ids,
+                                             int32_t align, float enc_ar_weight, float grad_scale,
+                                             float *loss, float *unit_loss, uint16_t *d_hidden,
+                                             uint16_t *d_enc_hidden, uint16_t *d_weight,
+                                             void *workspace, size_t workspace_bytes,
+                                             dlm_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * dlm_get_device_status -- copy the device status word of a loss workspace

@@ -105,6 +105,40 @@ def test_host_side_rejections(L):
     assert L.dlm_selftest_bounded_wait(20_000_000_000, 16, None) == 1
 
 
+def test_linear_uniform_rejections(L):
+    """Host-side checks of dlm_linear_loss_uniform_fwd_bwd: each bad argument
+    returns DLM_ERR_INVALID_ARGUMENT (or WORKSPACE_TOO_SMALL) before anything
+    is enqueued (no GPU is touched)."""
+    can = dlm.Layout(2, 32, 64, None, None)
+    enc = dlm.Layout(2, 48, 96, None, None)
+    need = L.dlm_linear_loss_uniform_workspace_size(ctypes.byref(can), ctypes.byref(enc), 64, 1024)
+
+    def call(layout=can, hidden=16, enc_layout=enc, enc_hidden=16, enc_ids=16, d_model=64, vocab=1024,
+             clean=16, align=0, d_hidden=16, d_enc_hidden=16, ws=1024, ws_bytes=need):
+        e = ctypes.byref(enc_layout) if enc_layout is not None else None
+        return L.dlm_linear_loss_uniform_fwd_bwd(ctypes.byref(layout), hidden, e, enc_hidden, enc_ids, 16,
+                                                 d_model, vocab, clean, align, 1.0, 1.0, 16, None, d_hidden,
+                                                 d_enc_hidden, None, ws, ws_bytes, None)
+    assert call(align=2) == 1
+    assert call(d_model=96) == 1                                  # d_model % 64
+    assert call(vocab=1020) == 1                                  # vocab % 8
+    assert call(enc_layout=dlm.Layout(3, 32, 96, None, None)) == 1  # unit counts differ
+    assert call(enc_hidden=None) == 1
+    assert call(enc_ids=None) == 1
+    assert call(d_enc_hidden=None) == 1
+    assert call(enc_hidden=24) == 1                               # not 16-byte aligned
+    assert call(clean=None) == 1
+    assert call(d_hidden=None) == 1
+    assert call(ws=512) == 1                                      # workspace not 1024-aligned
+    assert call(ws_bytes=need - 1) == 3                           # DLM_ERR_WORKSPACE_TOO_SMALL
+    # without the encoder term the workspace is that of the canvas rows alone;
+    # with it, that of canvas + encoder rows
+    alone = L.dlm_linear_loss_uniform_workspace_size(ctypes.byref(can), None, 64, 1024)
+    assert alone == L.dlm_linear_loss_workspace_size(ctypes.byref(can), 64, 1024)
+    both = dlm.Layout(2, 80, 160, None, None)
+    assert need == L.dlm_linear_loss_workspace_size(ctypes.byref(both), 64, 1024)
+
+
 def test_workspace_size_grows_with_rows(L):
     a = dlm.Layout(1, 4096, 4096, None, None)
     b = dlm.Layout(1, 8192, 8192, None, None)

@@ -210,3 +210,157 @@ def test_linear_full_size():
     assert abs(lhs - rhs) <= 2e-3 * max(abs(lhs), abs(rhs))
     colsum = dW.sum(0).abs().max().item()
     assert colsum <= 1e-2 * dW.abs().sum(0).max().item()
+
+
+# --------------------------------------------------------------------------
+# uniform noise through the fused head: canvas term + encoder AR term
+# ("diffusiongemma-26B-A4B-it-ALWAYS-THINK", Finetuning notes)
+# --------------------------------------------------------------------------
+def run_linear_uniform(spec, case, lam, align=oracle.ALIGNED, grad_scale=1.0, want_dw=True,
+                       canvas_pad=None, enc_pad=None, with_encoder=True):
+    dev = torch.device("cuda")
+    B, C, P = case.n_units, case.seq_len, spec.prefix
+    cp = torch.from_numpy(canvas_pad).to(dev) if canvas_pad is not None else None
+    ep = torch.from_numpy(enc_pad).to(dev) if enc_pad is not None else None
+    lay = dlm.make_layout(B, C, None, cp)
+    enc = dlm.make_layout(B, P + C, None, ep) if with_encoder else None
+    out = dlm.linear_loss_uniform_fwd_bwd(
+        lay, case.hidden, case.weight, case.clean, enc, case.enc_hidden if with_encoder else None,
+        case.enc_clean if with_encoder else None, enc_ar_weight=lam, align=align, grad_scale=grad_scale,
+        want_d_weight=want_dw)
+    torch.cuda.synchronize()
+    assert out.device_status() == 0
+    lay_o = oracle.Layout(B, C, None, canvas_pad)
+    enc_o = oracle.Layout(B, P + C, None, enc_pad) if with_encoder else None
+    ref = oracle.linear_loss_uniform(
+        lay_o, di.bf16_bits(case.hidden), di.bf16_bits(case.weight), case.clean.cpu().numpy(), enc_o,
+        di.bf16_bits(case.enc_hidden) if with_encoder else None,
+        case.enc_clean.cpu().numpy() if with_encoder else None, lam, align, grad_scale=grad_scale,
+        want_grads=True)
+    return out, ref
+
+
+def _uniform_spec(B, C, P, D, V):
+    return di.WORKLOADS["lin_unif_b4_p512_c1024_d4096_v262144"].scaled(
+        n_units=B, seq_len=C, prefix=P, d_model=D, vocab=V, ids_high=V - 1)
+
+
+@pytest.mark.parametrize("B,C,P,D,V,align,seed", [
+    (2, 40, 24, 64, 1000, oracle.ALIGNED, 0),       # ragged vocabulary tile, one row tile
+    (3, 300, 197, 128, 4104, oracle.SHIFTED, 1),    # ~2,400 rows: ten paired row tiles, ragged
+    (4, 256, 128, 256, 20000, oracle.ALIGNED, 2),   # two backward vocabulary chunks
+])
+def test_linear_uniform_elementwise(B, C, P, D, V, align, seed):
+    spec = _uniform_spec(B, C, P, D, V)
+    case = di.make_case(spec, "cuda", seed=seed)
+    out, ref = run_linear_uniform(spec, case, lam=0.8, align=align, grad_scale=0.5)
+    assert_loss_close(float(out.loss.item()), ref["loss"])
+    assert_units_close(out.unit_loss.cpu().numpy()[:B], ref["unit_loss"], ref["loss"])
+    dH = out.d_hidden.double().cpu().numpy()
+    dHe = out.d_enc_hidden.double().cpu().numpy()
+    dW = out.d_weight.double().cpu().numpy()
+    assert rel_fro(dH, ref["dH"]) < GRAD_REL_FRO
+    assert rel_fro(dHe, ref["dHe"]) < GRAD_REL_FRO
+    assert rel_fro(dW, ref["dW"]) < GRAD_REL_FRO
+    # rows with no target are exact zeros: each unit's last canvas row when
+    # shifted, each unit's last encoder row
+    for rows, g in ((ref["rows"], dH), (ref["enc_rows"], dHe)):
+        un = np.ones(g.shape[0], bool)
+        un[rows] = False
+        assert (g[un] == 0).all()
+    assert ref["enc_rows"].shape[0] == B * (P + C - 1)
+
+
+def test_linear_uniform_pads_without_encoder_no_dw():
+    """Padded canvas tokens are never scored; no encoder term; d_weight
+    skipped; negative gradient scale."""
+    B, C, D, V = 3, 200, 128, 4096
+    spec = _uniform_spec(B, C, 0, D, V)
+    case = di.make_case(spec, "cuda", seed=3)
+    pad = np.zeros(B * C, np.uint8)
+    for b, n in enumerate((200, 151, 9)):
+        pad[b * C + n:(b + 1) * C] = 1
+    out, ref = run_linear_uniform(spec, case, lam=1.0, grad_scale=-0.25, want_dw=False, canvas_pad=pad,
+                                  with_encoder=False)
+    assert out.d_weight is None and out.d_enc_hidden is None
+    assert_loss_close(float(out.loss.item()), ref["loss"])
+    dH = out.d_hidden.double().cpu().numpy()
+    assert rel_fro(dH, ref["dH"]) < GRAD_REL_FRO
+    assert (dH[pad == 1] == 0).all()
+
+
+def test_linear_uniform_encoder_pads():
+    """Padded encoder positions: neither scored nor a target."""
+    B, C, P, D, V = 2, 96, 64, 64, 2048
+    spec = _uniform_spec(B, C, P, D, V)
+    case = di.make_case(spec, "cuda", seed=4)
+    epad = np.zeros(B * (P + C), np.uint8)
+    epad[(P + C) - 30:(P + C)] = 1          # unit 0 ends 30 tokens early
+    out, ref = run_linear_uniform(spec, case, lam=2.0, enc_pad=epad)
+    assert_loss_close(float(out.loss.item()), ref["loss"])
+    assert_units_close(out.unit_loss.cpu().numpy()[:B], ref["unit_loss"], ref["loss"])
+    assert rel_fro(out.d_enc_hidden.double().cpu().numpy(), ref["dHe"]) < GRAD_REL_FRO
+    assert rel_fro(out.d_weight.double().cpu().numpy(), ref["dW"]) < GRAD_REL_FRO
+    assert ref["enc_rows"].shape[0] == (P + C - 31) + (P + C - 1)
+
+
+def test_linear_uniform_matches_unfused_gpu_path_on_materialised_logits():
+    """The fused uniform call and dlm_loss_fwd_bwd (uniform, with the
+    encoder term) on logits = H W^T rounded to bf16 agree to that rounding."""
+    B, C, P, D, V = 2, 128, 64, 256, 8192
+    spec = _uniform_spec(B, C, P, D, V)
+    case = di.make_case(spec, "cuda", seed=5)
+    dev = torch.device("cuda")
+    lay = dlm.make_layout(B, C)
+    enc = dlm.make_layout(B, P + C)
+    fused = dlm.linear_loss_uniform_fwd_bwd(lay, case.hidden, case.weight, case.clean, enc, case.enc_hidden,
+                                            case.enc_clean, enc_ar_weight=0.5)
+    logits = (case.hidden.float() @ case.weight.float().T).to(torch.bfloat16)
+    enc_logits = (case.enc_hidden.float() @ case.weight.float().T).to(torch.bfloat16)
+    p = torch.ones(B, dtype=torch.float32, device=dev)
+    corr = torch.ones(B * C, dtype=torch.uint8, device=dev)
+    ref = dlm.loss_fwd_bwd(lay, logits, V, case.clean, corr, p, oracle.UNIFORM, oracle.ALIGNED,
+                           enc_layout=enc, enc_logits=enc_logits, enc_ids=case.enc_clean, enc_ar_weight=0.5)
+    torch.cuda.synchronize()
+    a, b = float(fused.loss.item()), float(ref.loss.item())
+    assert abs(a - b) < 2e-3 * abs(b)
+
+
+def test_linear_uniform_full_size():
+    """DiffusionGemma-like shapes (B=4, prefix 512 + canvas 1024, D=4096,
+    V=262144): dH / dHe on sampled rows against the oracle, zero rows,
+    the loss against a sampled estimate, and identities at any size."""
+    spec = di.WORKLOADS["lin_unif_b4_p512_c1024_d4096_v262144"]
+    case = di.make_case(spec, "cuda")
+    B, C, P = 4, 1024, 512
+    lay = dlm.make_layout(B, C)
+    enc = dlm.make_layout(B, P + C)
+    out = dlm.linear_loss_uniform_fwd_bwd(lay, case.hidden, case.weight, case.clean, enc, case.enc_hidden,
+                                          case.enc_clean, enc_ar_weight=1.0)
+    torch.cuda.synchronize()
+    assert out.device_status() == 0
+    W = di.bf16_bits(case.weight)
+    pc = oracle.plan_diffusion(oracle.Layout(B, C, None, None), case.clean.cpu().numpy(), None, None,
+                               oracle.UNIFORM, oracle.ALIGNED)
+    pe = oracle.plan_encoder(oracle.Layout(B, P + C, None, None), case.enc_clean.cpu().numpy(), 1.0)
+    rng = np.random.default_rng(1)
+    est = 0.0
+    for plan, H, g, n in ((pc, case.hidden, out.d_hidden, B * C), (pe, case.enc_hidden, out.d_enc_hidden,
+                                                                   B * (P + C))):
+        scored = np.nonzero(plan.target >= 0)[0]
+        sample = np.sort(rng.choice(scored, size=10, replace=False))
+        spot = oracle.linear_rows_plan(plan, di.bf16_bits(H), W, sample)
+        assert rel_fro(g.double().cpu().numpy()[sample], spot["dH"]) < GRAD_REL_FRO
+        est += float(spot["ce"].mean()) * (plan.weight[scored].sum())
+        un = np.setdiff1d(np.arange(n), scored)
+        assert (g[torch.from_numpy(un).cuda()] == 0).all()
+    # mean CE of 10 rows per term: within a few standard errors of the loss
+    assert abs(float(out.loss.item()) - est) < 2.0
+    Wd = case.weight.double()
+    dW = out.d_weight.double()
+    lhs = float((dW * Wd).sum())
+    rhs = float((out.d_hidden.double() * case.hidden.double()).sum() +
+                (out.d_enc_hidden.double() * case.enc_hidden.double()).sum())
+    assert abs(lhs - rhs) <= 2e-3 * max(abs(lhs), abs(rhs))
+    colsum = dW.sum(0).abs().max().item()
+    assert colsum <= 1e-2 * dW.abs().sum(0).max().item()
