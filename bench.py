@@ -539,11 +539,14 @@ def _oracle_threads():
     return int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
 
 
-def cpu_baseline(spec, budget_s=15.0, min_steps=3, max_steps=100_000):
+def cpu_baseline(spec, budget_s=15.0, min_steps=3, max_steps=100_000, single_thread_s=8.0):
     """The oracle on a bounded sample: rows per sequence sized so that one
     step takes about budget_s / min_steps (at most 1024 rows, which bounds
     the host memory of its double-precision gradient), then steps with fresh
-    seeds until budget_s of CPU work has run."""
+    seeds until budget_s of CPU work has run.  With single_thread_s > 0 the
+    same is timed again with one thread, in a child process started with
+    OMP_NUM_THREADS=1 (the oracle's OpenMP and numpy's BLAS read it at
+    start-up)."""
     import dlm_inputs as di
 
     rows = _calibrated_rows(spec, budget_s / min_steps)
@@ -555,11 +558,24 @@ def cpu_baseline(spec, budget_s=15.0, min_steps=3, max_steps=100_000):
         scored += oracle_step(sub, case, 1000 + steps, rows)
         steps += 1
     dt = time.perf_counter() - t0
-    return {"value": scored / dt, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
-            "sample": f"{steps} steps (seeds 1000..{999 + steps}) of the same workload cut to its "
-                      f"first {rows} rows per sequence ({spec.vocab}-wide rows; time draw, "
-                      f"corruption, CE of the scored rows, double-precision gradient of every "
-                      f"row): {dt:.1f} s"}
+    res = {"value": scored / dt, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+           "sample": f"{steps} steps (seeds 1000..{999 + steps}) of the same workload cut to its "
+                     f"first {rows} rows per sequence ({spec.vocab}-wide rows; time draw, "
+                     f"corruption, CE of the scored rows, double-precision gradient of every "
+                     f"row): {dt:.1f} s"}
+    if single_thread_s > 0:
+        env = dict(os.environ, OMP_NUM_THREADS="1", OPENBLAS_NUM_THREADS="1", MKL_NUM_THREADS="1")
+        code = ("import json, bench, dlm_inputs as di; "
+                f"print(json.dumps(bench.cpu_baseline(di.WORKLOADS[{spec.key!r}], budget_s={single_thread_s}, "
+                "single_thread_s=0)))")
+        try:
+            r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
+                               text=True, timeout=20 * single_thread_s + 120)
+            one = json.loads(r.stdout.strip().splitlines()[-1])
+            res["single_thread"] = {"value": one["value"], "cores": one["cores"], "sample": one["sample"]}
+        except Exception as e:   # the all-cores figure stands on its own
+            res["single_thread"] = {"value": None, "error": f"{type(e).__name__}: {e}"[:200]}
+    return res
 
 
 def run_reference(args):
