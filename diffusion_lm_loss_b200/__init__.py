@@ -78,8 +78,10 @@ def make_layout(n_units: int, seq_len: int = 0, cu_seqlens: Optional[torch.Tenso
     """A dlm_layout_t over device tensors.  The layout holds references to
     cu_seqlens and pad_mask, whose device pointers it carries, so they stay
     allocated as long as the layout is in use."""
+    if n_units < 0 or seq_len < 0 or (n_tokens is not None and n_tokens < 0):
+        raise ValueError("n_units, seq_len and n_tokens must be non-negative")
     if cu_seqlens is not None:
-        _check(cu_seqlens, torch.int32, "cu_seqlens")
+        _check(cu_seqlens, torch.int32, "cu_seqlens", min_numel=n_units + 1)
         if n_tokens is None:
             raise ValueError("packed layouts need n_tokens (cu_seqlens lives on the device)")
         cu = cu_seqlens.data_ptr()
@@ -88,8 +90,9 @@ def make_layout(n_units: int, seq_len: int = 0, cu_seqlens: Optional[torch.Tenso
         n_tokens = n_units * seq_len if n_tokens is None else n_tokens
     pm = None
     if pad_mask is not None:
-        _check(pad_mask, torch.uint8, "pad_mask")
+        _check(pad_mask, torch.uint8, "pad_mask", min_numel=n_tokens)
         pm = pad_mask.data_ptr()
+    _on_cuda(cu_seqlens=cu_seqlens, pad_mask=pad_mask)
     lay = Layout(n_units, seq_len, n_tokens, cu, pm)
     lay._tensors = (cu_seqlens, pad_mask)
     return lay
@@ -152,11 +155,61 @@ def lib():
     return L
 
 
-def _check(t: torch.Tensor, dtype, name: str):
+def _check(t: Optional[torch.Tensor], dtype, name: str, min_numel: Optional[int] = None,
+           min_rows: Optional[int] = None, min_cols: Optional[int] = None):
+    """A tensor argument before its pointer goes to the library: dtype and
+    size (the C ABI sees only pointers, so a buffer shorter than the layout
+    says would be read or written out of bounds on the device).  The device
+    is checked afterwards, for all arguments of a call together (_on_cuda).
+    min_numel: a contiguous buffer of at least that many elements; min_rows /
+    min_cols: a 2-D tensor with unit column stride and at least that many rows
+    / columns."""
+    if t is None:
+        raise ValueError(f"{name}: required")
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
-    if not t.is_cuda:
-        raise ValueError(f"{name}: must be a CUDA tensor (there is no CPU path)")
+    if min_numel is not None:
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous")
+        if t.numel() < min_numel:
+            raise ValueError(f"{name}: needs at least {min_numel} elements, has {t.numel()}")
+    if min_rows is not None or min_cols is not None:
+        if t.dim() != 2 or (t.shape[1] > 1 and t.stride(1) != 1):
+            raise ValueError(f"{name}: must be 2-D with unit column stride, got shape {tuple(t.shape)}")
+        if min_rows is not None and t.shape[0] < min_rows:
+            raise ValueError(f"{name}: needs at least {min_rows} rows, has {t.shape[0]}")
+        if min_cols is not None and t.shape[1] < min_cols:
+            raise ValueError(f"{name}: needs at least {min_cols} columns, has {t.shape[1]}")
+
+
+def _on_cuda(**tensors):
+    """Every tensor argument of a call (None = not given) on one CUDA device."""
+    dev = None
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError(f"{name}: must be a CUDA tensor (there is no CPU path)")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name}: on {t.device}, the other arguments on {dev}")
+
+
+def _like_rows(t: torch.Tensor, zero: bool = False) -> torch.Tensor:
+    """A buffer with t's shape and strides (a gradient is written with the
+    row stride of its input, which may be wider than the row)."""
+    out = torch.empty_strided(t.shape, t.stride(), dtype=t.dtype, device=t.device)
+    return out.zero_() if zero else out
+
+
+def _check_grad(g: Optional[torch.Tensor], like: torch.Tensor, name: str):
+    """A caller-supplied gradient buffer: same dtype, shape and row stride as
+    the input it is the gradient of."""
+    _check(g, like.dtype, name)
+    if tuple(g.shape) != tuple(like.shape) or (like.dim() == 2 and g.stride(0) != like.stride(0)):
+        raise ValueError(f"{name}: must have the shape {tuple(like.shape)} and row stride "
+                         f"{like.stride(0)} of its input")
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -171,6 +224,16 @@ def _ok(code: int, where: str):
     if code != 0:
         detail = lib().dlm_last_cuda_error().decode() if code == 4 else ""
         raise DlmError(code, where, detail)
+
+
+def _check_out(loss: torch.Tensor, unit_loss: Optional[torch.Tensor], layout: Layout,
+               workspace: torch.Tensor):
+    """The scalar outputs and the workspace of a reused result object (the
+    library itself checks the workspace's size against the call)."""
+    _check(loss, torch.float32, "out.loss", min_numel=1)
+    if unit_loss is not None:
+        _check(unit_loss, torch.float32, "out.unit_loss", min_numel=layout.n_units)
+    _check(workspace, torch.uint8, "out.workspace", min_numel=0)
 
 
 def _bits(t: torch.Tensor) -> torch.Tensor:
@@ -194,8 +257,11 @@ def corrupt(layout: Layout, clean_ids: torch.Tensor, p: torch.Tensor, mode: int 
             mask_id: int = 0, vocab: int = 0, seed: int = 0,
             dev_status: Optional[torch.Tensor] = None):
     """(noisy int32, corrupted uint8), same length as clean_ids."""
-    _check(clean_ids, torch.int32, "clean_ids")
-    _check(p, torch.float32, "p")
+    _check(clean_ids, torch.int32, "clean_ids", min_numel=layout.n_tokens)
+    _check(p, torch.float32, "p", min_numel=layout.n_units)
+    if dev_status is not None and (dev_status.dtype not in (torch.int32, torch.uint32) or dev_status.numel() < 1):
+        raise ValueError("dev_status: an int32 / uint32 tensor of at least one element")
+    _on_cuda(clean_ids=clean_ids, p=p, dev_status=dev_status)
     noisy = torch.empty_like(clean_ids)
     corr = torch.empty(clean_ids.shape, dtype=torch.uint8, device=clean_ids.device)
     _ok(lib().dlm_corrupt(ctypes.byref(layout), _ptr(clean_ids), _ptr(p), mode, mask_id, vocab, seed,
@@ -230,27 +296,39 @@ def loss_fwd_bwd(layout: Layout, logits: torch.Tensor, vocab: int, clean_ids: to
     """Weighted CE forward + backward (see dlm_loss_fwd_bwd).  logits: bf16
     [rows, ld] (2-D, row stride ld >= vocab).  Reuses the buffers of `out`
     when given (no allocation)."""
-    _check(logits, torch.bfloat16, "logits")
-    _check(clean_ids, torch.int32, "clean_ids")
-    if logits.dim() != 2 or logits.stride(1) != 1:
-        raise ValueError("logits must be 2-D with unit column stride")
+    T = layout.n_tokens
+    _check(logits, torch.bfloat16, "logits", min_rows=T, min_cols=vocab)
+    _check(clean_ids, torch.int32, "clean_ids", min_numel=T)
+    if corrupted is not None or (mode == ABSORBING and T > 0):
+        _check(corrupted, torch.uint8, "corrupted", min_numel=T)
+    if p is not None:
+        _check(p, torch.float32, "p", min_numel=layout.n_units)
     ld = logits.stride(0)
     enc_ld = 0
     if enc_logits is not None:
-        _check(enc_logits, torch.bfloat16, "enc_logits")
-        _check(enc_ids, torch.int32, "enc_ids")
-        if enc_logits.dim() != 2 or enc_logits.stride(1) != 1:
-            raise ValueError("enc_logits must be 2-D with unit column stride")
+        if enc_layout is None:
+            raise ValueError("enc_logits needs enc_layout")
+        _check(enc_logits, torch.bfloat16, "enc_logits", min_rows=enc_layout.n_tokens, min_cols=vocab)
+        _check(enc_ids, torch.int32, "enc_ids", min_numel=enc_layout.n_tokens)
         enc_ld = enc_logits.stride(0)
+    if out is not None:
+        _check_out(out.loss, out.unit_loss, layout, out.workspace)
+        _check_grad(out.dlogits, logits, "out.dlogits")
+        if enc_logits is not None:
+            _check_grad(out.enc_dlogits, enc_logits, "out.enc_dlogits")
+    o = out if out is not None else LossOut(None, None, None, None, None)
+    _on_cuda(logits=logits, clean_ids=clean_ids, corrupted=corrupted, p=p, enc_logits=enc_logits,
+             enc_ids=enc_ids, loss=o.loss, unit_loss=o.unit_loss, workspace=o.workspace, dlogits=o.dlogits,
+             enc_dlogits=o.enc_dlogits if enc_logits is not None else None)
     dev = logits.device
+    keep = options is not None and options.keep_unscored_rows
     if out is None:
         ws = torch.empty(loss_workspace_size(layout, enc_layout), dtype=torch.uint8, device=dev)
         # rows the call leaves untouched must start as zeros
-        grad_buf = torch.zeros_like if (options is not None and options.keep_unscored_rows) else torch.empty_like
         out = LossOut(torch.empty(1, dtype=torch.float32, device=dev),
                       torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
-                      grad_buf(logits),
-                      grad_buf(enc_logits) if enc_logits is not None else None, ws)
+                      _like_rows(logits, keep),
+                      _like_rows(enc_logits, keep) if enc_logits is not None else None, ws)
     if options is None:
         _ok(lib().dlm_loss_fwd_bwd(
             ctypes.byref(layout), _ptr(logits), ld, vocab, _ptr(clean_ids), _ptr(corrupted), _ptr(p),
@@ -281,6 +359,18 @@ class LinearOut:
         return device_status(self.workspace)
 
 
+def _check_head(layout: Layout, hidden: torch.Tensor, weight: torch.Tensor):
+    """hidden [n_tokens, D] and weight [V, D], contiguous bf16; returns (T, D, V)."""
+    T = layout.n_tokens
+    _check(hidden, torch.bfloat16, "hidden", min_numel=0)
+    _check(weight, torch.bfloat16, "weight", min_numel=0)
+    if hidden.dim() != 2 or weight.dim() != 2 or hidden.shape[1] != weight.shape[1]:
+        raise ValueError("hidden [tokens, d_model] and weight [vocab, d_model] must share d_model")
+    if hidden.shape[0] < T:
+        raise ValueError(f"hidden: needs at least {T} rows, has {hidden.shape[0]}")
+    return T, int(hidden.shape[1]), int(weight.shape[0])
+
+
 def linear_loss_workspace_size(layout: Layout, d_model: int, vocab: int) -> int:
     return int(lib().dlm_linear_loss_workspace_size(ctypes.byref(layout), d_model, vocab))
 
@@ -291,14 +381,18 @@ def linear_loss_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: torch.Tens
                         out: Optional[LinearOut] = None, align: int = ALIGNED) -> LinearOut:
     """Fused lm_head + absorbing loss (see dlm_linear_loss_fwd_bwd; align =
     SHIFTED goes through dlm_linear_loss_fwd_bwd_ex)."""
-    _check(hidden, torch.bfloat16, "hidden")
-    _check(weight, torch.bfloat16, "weight")
-    if not (hidden.is_contiguous() and weight.is_contiguous()):
-        raise ValueError("hidden and weight must be contiguous")
-    T, D = hidden.shape
-    V, D2 = weight.shape
-    if D != D2:
-        raise ValueError("hidden / weight d_model mismatch")
+    T, D, V = _check_head(layout, hidden, weight)
+    _check(clean_ids, torch.int32, "clean_ids", min_numel=T)
+    _check(corrupted, torch.uint8, "corrupted", min_numel=T)
+    _check(p, torch.float32, "p", min_numel=layout.n_units)
+    if out is not None:
+        _check_out(out.loss, out.unit_loss, layout, out.workspace)
+        _check_grad(out.d_hidden, hidden, "out.d_hidden")
+        if out.d_weight is not None:
+            _check_grad(out.d_weight, weight, "out.d_weight")
+    o = out if out is not None else LinearOut(None, None, None, None, None)
+    _on_cuda(hidden=hidden, weight=weight, clean_ids=clean_ids, corrupted=corrupted, p=p, loss=o.loss,
+             unit_loss=o.unit_loss, workspace=o.workspace, d_hidden=o.d_hidden, d_weight=o.d_weight)
     dev = hidden.device
     if out is None:
         ws = torch.empty(linear_loss_workspace_size(layout, D, V), dtype=torch.uint8, device=dev)
@@ -335,20 +429,25 @@ def linear_loss_uniform_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: to
                                 out: Optional[LinearOut] = None) -> LinearOut:
     """Fused lm_head + uniform-noise loss with the optional encoder
     next-token term (see dlm_linear_loss_uniform_fwd_bwd)."""
-    _check(hidden, torch.bfloat16, "hidden")
-    _check(weight, torch.bfloat16, "weight")
-    if not (hidden.is_contiguous() and weight.is_contiguous()):
-        raise ValueError("hidden and weight must be contiguous")
-    T, D = hidden.shape
-    V, D2 = weight.shape
-    if D != D2:
-        raise ValueError("hidden / weight d_model mismatch")
+    T, D, V = _check_head(layout, hidden, weight)
+    _check(clean_ids, torch.int32, "clean_ids", min_numel=T)
     if enc_layout is not None:
-        if enc_hidden is None or enc_ids is None:
-            raise ValueError("enc_layout needs enc_hidden and enc_ids")
-        _check(enc_hidden, torch.bfloat16, "enc_hidden")
-        if not enc_hidden.is_contiguous() or enc_hidden.shape[1] != D:
-            raise ValueError("enc_hidden must be contiguous [enc_tokens, d_model]")
+        Te = enc_layout.n_tokens
+        _check(enc_hidden, torch.bfloat16, "enc_hidden", min_numel=Te * D)
+        if enc_hidden.dim() != 2 or enc_hidden.shape[1] != D:
+            raise ValueError("enc_hidden must be [enc_tokens, d_model]")
+        _check(enc_ids, torch.int32, "enc_ids", min_numel=Te)
+    if out is not None:
+        _check_out(out.loss, out.unit_loss, layout, out.workspace)
+        _check_grad(out.d_hidden, hidden, "out.d_hidden")
+        if out.d_weight is not None:
+            _check_grad(out.d_weight, weight, "out.d_weight")
+        if enc_layout is not None:
+            _check_grad(out.d_enc_hidden, enc_hidden, "out.d_enc_hidden")
+    o = out if out is not None else LinearOut(None, None, None, None, None)
+    _on_cuda(hidden=hidden, weight=weight, clean_ids=clean_ids, enc_hidden=enc_hidden, enc_ids=enc_ids,
+             loss=o.loss, unit_loss=o.unit_loss, workspace=o.workspace, d_hidden=o.d_hidden,
+             d_weight=o.d_weight, d_enc_hidden=o.d_enc_hidden if enc_layout is not None else None)
     dev = hidden.device
     if out is None:
         ws = torch.empty(linear_loss_uniform_workspace_size(layout, enc_layout, D, V), dtype=torch.uint8,
