@@ -359,6 +359,15 @@ class LinearOut:
         return device_status(self.workspace)
 
 
+def _aligned_workspace(nbytes: int, device, align: int = 1024) -> torch.Tensor:
+    """A uint8 workspace whose first byte is `align`-byte aligned (the fused
+    head needs 1024; the caching allocator guarantees only 512): a slice of a
+    slightly larger buffer, which the slice keeps alive."""
+    buf = torch.empty(nbytes + align - 1, dtype=torch.uint8, device=device)
+    off = (-buf.data_ptr()) % align
+    return buf[off:off + nbytes]
+
+
 def _check_head(layout: Layout, hidden: torch.Tensor, weight: torch.Tensor):
     """hidden [n_tokens, D] and weight [V, D], contiguous bf16; returns (T, D, V)."""
     T = layout.n_tokens
@@ -395,7 +404,7 @@ def linear_loss_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: torch.Tens
              unit_loss=o.unit_loss, workspace=o.workspace, d_hidden=o.d_hidden, d_weight=o.d_weight)
     dev = hidden.device
     if out is None:
-        ws = torch.empty(linear_loss_workspace_size(layout, D, V), dtype=torch.uint8, device=dev)
+        ws = _aligned_workspace(linear_loss_workspace_size(layout, D, V), dev)
         out = LinearOut(torch.empty(1, dtype=torch.float32, device=dev),
                         torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
                         torch.empty_like(hidden),
@@ -450,8 +459,7 @@ def linear_loss_uniform_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: to
              d_weight=o.d_weight, d_enc_hidden=o.d_enc_hidden if enc_layout is not None else None)
     dev = hidden.device
     if out is None:
-        ws = torch.empty(linear_loss_uniform_workspace_size(layout, enc_layout, D, V), dtype=torch.uint8,
-                         device=dev)
+        ws = _aligned_workspace(linear_loss_uniform_workspace_size(layout, enc_layout, D, V), dev)
         out = LinearOut(torch.empty(1, dtype=torch.float32, device=dev),
                         torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
                         torch.empty_like(hidden),

@@ -545,6 +545,10 @@ struct LinWs {
     int tpad, n_tiles;
 };
 
+// Rows (canvas + encoder) the fused head accepts: the row count padded to
+// the 256-row pair tile must stay an int.
+constexpr int64_t kMaxLinRows = (int64_t(1) << 31) - 1 - kRowPad;
+
 static LinWs lin_ws(int64_t T, int64_t units, int D, int V) {
     LinWs w;
     w.tpad = int(align_up(size_t(T > 0 ? T : 1), kRowPad));
@@ -647,15 +651,17 @@ static dlm_status_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, cons
 using namespace dlm;
 
 extern "C" size_t dlm_linear_loss_workspace_size(const dlm_layout_t* layout, int32_t d_model, int32_t vocab) {
-    if (!layout || d_model <= 0 || vocab <= 0) return 0;
+    if (!layout || d_model <= 0 || vocab <= 0 || layout->n_tokens < 0 || layout->n_tokens > kMaxLinRows) return 0;
     return lin_ws(layout->n_tokens, layout->n_units, d_model, vocab).total;
 }
 
 extern "C" size_t dlm_linear_loss_uniform_workspace_size(const dlm_layout_t* layout,
                                                          const dlm_layout_t* enc_layout, int32_t d_model,
                                                          int32_t vocab) {
-    if (!layout || d_model <= 0 || vocab <= 0) return 0;
+    if (!layout || d_model <= 0 || vocab <= 0 || layout->n_tokens < 0) return 0;
+    if (enc_layout && enc_layout->n_tokens < 0) return 0;
     const int64_t rows = layout->n_tokens + (enc_layout ? enc_layout->n_tokens : 0);
+    if (rows > kMaxLinRows) return 0;
     return lin_ws(rows, layout->n_units, d_model, vocab).total;
 }
 
@@ -688,7 +694,7 @@ static dlm_status_t linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16
     const int64_t T = layout->n_tokens;
     const int64_t Te = has_enc ? enc_layout->n_tokens : 0;
     const int64_t R = T + Te;
-    if (R >= (int64_t(1) << 31)) return DLM_ERR_INVALID_ARGUMENT;
+    if (R > kMaxLinRows) return DLM_ERR_INVALID_ARGUMENT;
     if (T > 0 && (!hidden || !weight || !clean_ids || !d_hidden)) return DLM_ERR_INVALID_ARGUMENT;
     if (T > 0 && mode == DLM_ABSORBING && (!corrupted || !p)) return DLM_ERR_INVALID_ARGUMENT;
     if (T > 0 && !layout->cu_seqlens && layout->seq_len == 0) return DLM_ERR_INVALID_ARGUMENT;

@@ -39,7 +39,9 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *     default stream) and never synchronise, except dlm_get_device_status.
  *   - The library allocates no device memory.  Scratch comes from a caller
- *     workspace of at least dlm_*_workspace_size() bytes, 256-byte aligned.
+ *     workspace of at least dlm_*_workspace_size() bytes, 256-byte aligned
+ *     (1024-byte aligned for the dlm_linear_* calls).  A *_workspace_size()
+ *     call returns 0 for arguments its loss call would refuse.
  *     A workspace may be reused by calls ordered on one stream; calls that
  *     overlap on the GPU need separate workspaces.
  *   - Host-checkable errors return before anything is enqueued.  Errors that
@@ -290,7 +292,9 @@ DLM_API dlm_status_t dlm_loss_fwd_bwd_static(const dlm_layout_t *layout, const u
  *   d_hidden [n_tokens, d_model] bf16 (written; rows of unscored tokens = 0).
  *   d_weight [vocab, d_model] bf16 (written), or NULL to skip it.
  *   loss / unit_loss as for dlm_loss_fwd_bwd (unit_loss may be NULL).
- * Requires d_model % 64 == 0 and vocab % 8 == 0, 16-byte aligned pointers.
+ * Requires d_model % 64 == 0 and vocab % 8 == 0, 16-byte aligned pointers,
+ * a 1024-byte aligned workspace and fewer than 2^31 - 256 tokens; otherwise
+ * DLM_ERR_INVALID_ARGUMENT before anything is enqueued.
  * ---------------------------------------------------------------------- */
 DLM_API size_t dlm_linear_loss_workspace_size(const dlm_layout_t *layout, int32_t d_model,
                                       int32_t vocab);
@@ -343,8 +347,8 @@ DLM_API dlm_status_t dlm_linear_loss_fwd_bwd_ex(const dlm_layout_t *layout, cons
  *   enc_layout.n_units must equal layout.n_units (unit u of the canvas is
  *   unit u of the encoder sequence); unit_loss[u] sums both terms of unit u.
  *   Requires d_model % 64 == 0, vocab % 8 == 0, 16-byte aligned pointers and
- *   fewer than 2^31 rows in total; otherwise DLM_ERR_INVALID_ARGUMENT before
- *   anything is enqueued.  Ids outside [0, vocab) set DLM_DEV_BAD_TOKEN_ID in
+ *   fewer than 2^31 - 256 rows in total; otherwise DLM_ERR_INVALID_ARGUMENT
+ *   before anything is enqueued.  Ids outside [0, vocab) set DLM_DEV_BAD_TOKEN_ID in
  *   the device status word; their rows are skipped.
  * Workspace: dlm_linear_loss_uniform_workspace_size(layout, enc_layout,
  * d_model, vocab) bytes, 1024-byte aligned (enc_layout may be NULL).

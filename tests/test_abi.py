@@ -137,6 +137,12 @@ def test_linear_uniform_rejections(L):
     assert alone == L.dlm_linear_loss_workspace_size(ctypes.byref(can), 64, 1024)
     both = dlm.Layout(2, 80, 160, None, None)
     assert need == L.dlm_linear_loss_workspace_size(ctypes.byref(both), 64, 1024)
+    # rows whose 256-row padding would overflow an int: no workspace size
+    huge = dlm.Layout(1, 0, (1 << 31) - 200, None, None)
+    assert L.dlm_linear_loss_workspace_size(ctypes.byref(huge), 64, 1024) == 0
+    assert L.dlm_linear_loss_uniform_workspace_size(ctypes.byref(huge), None, 64, 1024) == 0
+    half = dlm.Layout(1, 0, 1 << 30, None, None)
+    assert L.dlm_linear_loss_uniform_workspace_size(ctypes.byref(half), ctypes.byref(half), 64, 1024) == 0
 
 
 def test_workspace_size_grows_with_rows(L):

@@ -136,3 +136,10 @@ def test_linear_sizes():
                                         torch.zeros(20, dtype=torch.int32))
     _cpu_only(lambda: dlm.linear_loss_uniform_fwd_bwd(lay, H, W, ids, enc, torch.zeros(24, 64, dtype=bf16),
                                                       torch.zeros(24, dtype=torch.int32)))
+
+
+def test_fused_head_workspace_is_1024_byte_aligned():
+    for n in (1, 1000, 4096, 123457):
+        ws = dlm._aligned_workspace(n, "cpu")
+        assert ws.numel() == n and ws.dtype == torch.uint8 and ws.is_contiguous()
+        assert ws.data_ptr() % 1024 == 0

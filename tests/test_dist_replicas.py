@@ -68,3 +68,16 @@ def test_reference_arm_prints_on_rank0_only():
     line = json.loads(r0.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["value"] > 0 and line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["n_gpus"] == 2
+
+
+def test_cpu_baseline_all_cores_and_one_thread():
+    """The CPU baseline: the oracle on a bounded sample for about its time
+    budget, then again on one thread in a child process."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import dlm_inputs as di
+    r = bench.cpu_baseline(di.WORKLOADS["abs_b2_l64_v1024"], budget_s=0.5, single_thread_s=0.3)
+    assert r["kind"] == "oracle" and r["value"] > 0 and r["cores"] >= 1
+    assert "steps" in r["sample"] and r["unit"] == bench.UNIT
+    one = r["single_thread"]
+    assert one["cores"] == 1 and one["value"] > 0, one
