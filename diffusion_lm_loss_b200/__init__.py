@@ -323,7 +323,7 @@ def loss_fwd_bwd(layout: Layout, logits: torch.Tensor, vocab: int, clean_ids: to
     dev = logits.device
     keep = options is not None and options.keep_unscored_rows
     if out is None:
-        ws = torch.empty(loss_workspace_size(layout, enc_layout), dtype=torch.uint8, device=dev)
+        ws = _aligned_workspace(loss_workspace_size(layout, enc_layout), dev, 256)
         # rows the call leaves untouched must start as zeros
         out = LossOut(torch.empty(1, dtype=torch.float32, device=dev),
                       torch.empty(max(layout.n_units, 1), dtype=torch.float32, device=dev),
@@ -360,9 +360,10 @@ class LinearOut:
 
 
 def _aligned_workspace(nbytes: int, device, align: int = 1024) -> torch.Tensor:
-    """A uint8 workspace whose first byte is `align`-byte aligned (the fused
-    head needs 1024; the caching allocator guarantees only 512): a slice of a
-    slightly larger buffer, which the slice keeps alive."""
+    """A uint8 workspace whose first byte is `align`-byte aligned (the loss
+    needs 256, the fused head 1024; the caching allocator guarantees 512 and
+    other allocators less): a slice of a slightly larger buffer, which the
+    slice keeps alive."""
     buf = torch.empty(nbytes + align - 1, dtype=torch.uint8, device=device)
     off = (-buf.data_ptr()) % align
     return buf[off:off + nbytes]

@@ -143,3 +143,70 @@ def test_fused_head_workspace_is_1024_byte_aligned():
         ws = dlm._aligned_workspace(n, "cpu")
         assert ws.numel() == n and ws.dtype == torch.uint8 and ws.is_contiguous()
         assert ws.data_ptr() % 1024 == 0
+
+
+# --------------------------------------------------------------------------
+# valid calls get past every host-side check: the binding's (device check
+# stubbed out) and the library's, and stop only at the library's own check
+# for a B200, which fails here without a device
+# --------------------------------------------------------------------------
+@pytest.fixture
+def host_only(monkeypatch):
+    from diffusion_lm_loss_b200 import build as dlm_build
+    dlm_build.build()
+    monkeypatch.setattr(dlm, "_on_cuda", lambda **kw: None)
+    monkeypatch.setattr(dlm, "_stream", lambda: None)
+
+
+def _stops_at_device_check(fn):
+    with pytest.raises(dlm.DlmError) as e:
+        fn()
+    assert e.value.code in (2, 4), e.value      # DLM_ERR_UNSUPPORTED / DLM_ERR_CUDA, nothing earlier
+
+
+def test_valid_loss_calls_pass_host_checks(host_only):
+    V = 1000
+    lay = dlm.make_layout(2, 24)
+    logits = torch.zeros(48, V, dtype=bf16)
+    ids = torch.zeros(48, dtype=torch.int32)
+    corr = torch.zeros(48, dtype=torch.uint8)
+    p = torch.full((2,), 0.5)
+    _stops_at_device_check(lambda: dlm.corrupt(lay, ids, p, dlm.ABSORBING, V - 1, V, 0))
+    _stops_at_device_check(lambda: dlm.loss_fwd_bwd(lay, logits, V, ids, corr, p))
+    # padded row stride: logits a column slice of a wider buffer, own gradient buffer reused
+    wide = torch.zeros(48, 1010, dtype=bf16)
+    out = dlm.LossOut(torch.zeros(1), torch.zeros(2), dlm._like_rows(wide[:, :V]), None,
+                      dlm._aligned_workspace(dlm.loss_workspace_size(lay), "cpu", 256))
+    _stops_at_device_check(lambda: dlm.loss_fwd_bwd(lay, wide[:, :V], V, ids, corr, p, out=out))
+    # uniform noise with the encoder term and the objective options
+    enc = dlm.make_layout(2, 32)
+    kw = dict(enc_layout=enc, enc_logits=torch.zeros(64, V, dtype=bf16),
+              enc_ids=torch.zeros(64, dtype=torch.int32), enc_ar_weight=1.0)
+    _stops_at_device_check(lambda: dlm.loss_fwd_bwd(lay, logits, V, ids, None, None, dlm.UNIFORM, **kw))
+    opts = dlm.LossOptions(dlm.TIME_WEIGHT_INV_ONE_MINUS_T, 10.0, dlm.REDUCE_EXAMPLE_MEAN)
+    _stops_at_device_check(lambda: dlm.loss_fwd_bwd(lay, logits, V, ids, corr, p, dlm.UNIFORM, options=opts,
+                                                    **kw))
+    # empty input
+    empty = dlm.make_layout(2, 0)
+    _stops_at_device_check(lambda: dlm.loss_fwd_bwd(empty, torch.zeros(0, 4096, dtype=bf16), 4096,
+                                                    torch.zeros(0, dtype=torch.int32),
+                                                    torch.zeros(0, dtype=torch.uint8), p))
+
+
+def test_valid_fused_head_calls_pass_host_checks(host_only):
+    D, V = 64, 1024
+    lay = dlm.make_layout(2, 24)
+    H = torch.zeros(48, D, dtype=bf16)
+    W = torch.zeros(V, D, dtype=bf16)
+    ids = torch.zeros(48, dtype=torch.int32)
+    corr = torch.zeros(48, dtype=torch.uint8)
+    p = torch.full((2,), 0.5)
+    for align in (dlm.ALIGNED, dlm.SHIFTED):
+        _stops_at_device_check(lambda: dlm.linear_loss_fwd_bwd(lay, H, W, ids, corr, p, align=align))
+    _stops_at_device_check(lambda: dlm.linear_loss_fwd_bwd(lay, H, W, ids, corr, p, want_d_weight=False))
+    enc = dlm.make_layout(2, 40)
+    He = torch.zeros(80, D, dtype=bf16)
+    eids = torch.zeros(80, dtype=torch.int32)
+    _stops_at_device_check(lambda: dlm.linear_loss_uniform_fwd_bwd(lay, H, W, ids, enc, He, eids, 0.5))
+    _stops_at_device_check(lambda: dlm.linear_loss_uniform_fwd_bwd(lay, H, W, ids, align=dlm.SHIFTED,
+                                                                   want_d_weight=False))
