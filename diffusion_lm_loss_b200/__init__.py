@@ -43,7 +43,8 @@ EXPORTS = ("dlm_status_string", "dlm_last_cuda_error", "dlm_version", "dlm_sampl
            "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_loss_fwd_bwd_ex", "dlm_loss_fwd_bwd_static",
            "dlm_linear_loss_workspace_size",
            "dlm_linear_loss_fwd_bwd", "dlm_linear_loss_fwd_bwd_ex", "dlm_linear_loss_uniform_workspace_size",
-           "dlm_linear_loss_uniform_fwd_bwd", "dlm_get_device_status", "dlm_selftest_bounded_wait")
+           "dlm_linear_loss_uniform_fwd_bwd", "dlm_get_device_status", "dlm_selftest_bounded_wait",
+           "dlm_test_skip_device_check")
 
 
 class DlmError(RuntimeError):
@@ -147,6 +148,8 @@ def lib():
     L.dlm_linear_loss_uniform_fwd_bwd.restype = ctypes.c_int
     L.dlm_linear_loss_uniform_fwd_bwd.argtypes = [lp, vp, lp, vp, vp, vp, i32, i32, vp, i32, f32, f32,
                                                   vp, vp, vp, vp, vp, vp, sz, vp]
+    L.dlm_test_skip_device_check.restype = ctypes.c_int
+    L.dlm_test_skip_device_check.argtypes = [i32]
     L.dlm_selftest_bounded_wait.restype = ctypes.c_int
     L.dlm_selftest_bounded_wait.argtypes = [u64, vp, vp]
     L.dlm_get_device_status.restype = ctypes.c_int

@@ -1,5 +1,6 @@
 // dlm_api.cu -- status strings, version, the device check and the
 // device-status read-back of the C ABI.
+#include <atomic>
 #include <mutex>
 
 #include "dlm_device.cuh"
@@ -16,7 +17,13 @@ void record_cuda_error(cudaError_t e, const char* where) {
                   cudaGetErrorName(e));
 }
 
+// Test hook (dlm_test_skip_device_check): when set, check_device passes
+// without asking the runtime, so that on a host without a usable device each
+// call goes on to its own CUDA calls and their error paths run.
+static std::atomic<int> g_skip_device_check{0};
+
 dlm_status_t check_device() {
+    if (g_skip_device_check.load(std::memory_order_relaxed)) return DLM_OK;
     // compute capability 10.0 (B200) only; cached per device ordinal
     static std::mutex mu;
     static int known[64];   // 0 = unknown, 1 = ok, 2 = unsupported
@@ -27,10 +34,11 @@ dlm_status_t check_device() {
     std::lock_guard<std::mutex> g(mu);
     if (known[dev] == 0) {
         int major = 0, minor = 0;
-        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (e != cudaSuccess) {
             cudaGetLastError();
-            return DLM_ERR_CUDA;
+            return cuda_status(e, "cudaDeviceGetAttribute (compute capability)");
         }
         known[dev] = (major == 10 && minor == 0) ? 1 : 2;
     }
@@ -73,6 +81,12 @@ extern "C" const char* dlm_status_string(dlm_status_t status) {
 extern "C" int dlm_version(void) { return 200; }   // 0.2.0: + dlm_loss_fwd_bwd_ex
 
 extern "C" const char* dlm_last_cuda_error(void) { return dlm::g_last_error; }
+
+extern "C" dlm_status_t dlm_test_skip_device_check(int32_t enabled) {
+    if (enabled != 0 && enabled != 1) return DLM_ERR_INVALID_ARGUMENT;
+    dlm::g_skip_device_check.store(enabled, std::memory_order_relaxed);
+    return DLM_OK;
+}
 
 extern "C" dlm_status_t dlm_get_device_status(const void* workspace, uint32_t* host_status,
                                               dlm_stream_t stream) {

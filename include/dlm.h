@@ -379,6 +379,20 @@ DLM_API dlm_status_t dlm_get_device_status(const void *workspace, uint32_t *host
                                    dlm_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * dlm_test_skip_device_check -- test hook, off by default; not for use in
+ * training.  With enabled = 1 every call skips its check for a B200 and goes
+ * straight on to its CUDA calls.  On a host without a usable device those
+ * calls fail, and each entry point must turn the failure into
+ * DLM_ERR_CUDA with a message (dlm_last_cuda_error) instead of crashing:
+ * this is how the library's CUDA error paths are tested without a GPU.  On a
+ * host with a device, enabling it lets a call launch its kernels on whatever
+ * device is current (sm_100a code only runs on a B200).  enabled = 0 restores
+ * the check; any other value returns DLM_ERR_INVALID_ARGUMENT.  The setting
+ * is process-wide.
+ * ---------------------------------------------------------------------- */
+DLM_API dlm_status_t dlm_test_skip_device_check(int32_t enabled);
+
+/* ------------------------------------------------------------------------
  * dlm_selftest_bounded_wait -- exercise the library's failure detection on
  * the device.  Every on-chip wait of the kernels above (mbarrier phases of
  * the TMA / tensor-core pipelines) gives up after a time limit, records
