@@ -41,6 +41,7 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 CE_SOURCE = os.path.join(ROOT, "diffusion_lm_loss_b200", "csrc", "dlm_ce.cu")
 CE_PROFILE = os.path.join(ROOT, "profiles", "ce_stream_abs_b1_l4096_v126464.md")
+ABSORBING, UNIFORM = 0, 1          # noise modes, as numbered in include/dlm.h
 
 
 def env_rank():
@@ -470,6 +471,12 @@ def run_linear(args, spec, dev, rank, world):
         dist.destroy_process_group()
     if rank != 0:
         return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        try:
+            cpu = cpu_baseline(spec)
+        except Exception as e:      # the GPU figures above stand without it
+            cpu = {"value": None, "kind": "oracle", "error": f"{type(e).__name__}: {e}"[:300]}
     res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "bf16", "data": "synthetic",
@@ -477,7 +484,7 @@ def run_linear(args, spec, dev, rank, world):
                       "tokens": T, "d_model": D, "encoder_ar_weight": spec.enc_ar_weight if uniform else None,
                       "vocab": V, "documents": case.n_units, "parallelism": f"replicas{world}",
                       "scored_tokens": scored_all, "l2": "inputs larger than L2 (W %.2f GB)" % (V * D * 2 / 1e9)},
-           "roofline": roof, "cpu_baseline": None, "clocks": clk, "e2e": None,
+           "roofline": roof, "cpu_baseline": cpu, "clocks": clk, "e2e": None,
            # per step: time draw, corruption, plan, gather, forward GEMM, lse,
            # dZ + dH + dW per 16,384-column vocabulary chunk, scatter, reduce
            "gpu_launches": K * (6 + 3 * ((V + 16383) // 16384) + 2)}
@@ -487,6 +494,47 @@ def run_linear(args, spec, dev, rank, world):
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline leg and reference arm)
 # ---------------------------------------------------------------------------
+def sample_spec(spec, rows):
+    """The workload cut to its first `rows` rows per sequence (packed
+    documents: to its first `rows` tokens, the same documents up to the cut)."""
+    if spec.kind == "linear" and spec.mode == ABSORBING:
+        return spec.scaled(n_tokens_packed=rows)
+    return spec.scaled(seq_len=rows, prefix=min(spec.prefix, rows))
+
+
+def sample_words(spec, rows):
+    """How a bounded sample of the workload is described in the JSON line."""
+    cut = (f"its first {rows} tokens of packed documents" if spec.kind == "linear" and spec.mode == ABSORBING
+           else f"its first {rows} rows per sequence")
+    work = ("time draw, corruption, CE of the scored rows, double-precision gradient of every row"
+            + (", dH and dW through the head" if spec.kind == "linear" else ""))
+    return cut, work
+
+
+def oracle_inputs(spec, case_cpu):
+    """Bit patterns of the fused-head inputs, converted once per case, before
+    any timing (the logits workloads convert their sample inside the step)."""
+    import dlm_inputs as di
+
+    if spec.kind == "linear" and "W" not in case_cpu.extra:
+        case_cpu.extra["W"] = di.bf16_bits(case_cpu.weight)
+        case_cpu.extra["H"] = di.bf16_bits(case_cpu.hidden)
+        if case_cpu.enc_hidden is not None:
+            case_cpu.extra["He"] = di.bf16_bits(case_cpu.enc_hidden)
+
+
+def oracle_host_bytes(spec, rows):
+    """Peak host memory of one fused-head oracle step on `rows` rows per
+    sequence (double-precision dW per term and their sum, W as bf16 in torch
+    and numpy, Z and dZ of the rows), or 0 for the logits workloads."""
+    if spec.kind != "linear":
+        return 0
+    V, D = spec.vocab, spec.d_model
+    terms = 2 if spec.mode == UNIFORM else 1
+    units = spec.n_units if spec.mode == UNIFORM else 1
+    return V * D * (8 * (terms + 1) + 2 * 2) + 2 * rows * units * V * 8 + 16384 * D * 8
+
+
 def oracle_step(spec, case_cpu, seed, rows_sample):
     """The oracle as it stands on the first `rows_sample` rows of each unit's
     sequence: time draw, corruption, CE of the scored rows, gradient of all
@@ -495,6 +543,9 @@ def oracle_step(spec, case_cpu, seed, rows_sample):
 
     import dlm_inputs as di
     import oracle
+
+    if spec.kind == "linear":
+        return _oracle_linear_step(spec, case_cpu, seed)
 
     B = spec.n_units
     L = min(spec.seq_len, rows_sample)
@@ -521,10 +572,57 @@ def oracle_step(spec, case_cpu, seed, rows_sample):
     return int(tc.rows.shape[0] + te.rows.shape[0])
 
 
+def _oracle_linear_step(spec, case, seed):
+    """The fused-head oracle on a case already cut to its sample: time draw,
+    corruption, then the loss from hidden states and the head with dH and dW
+    (absorbing: packed documents; uniform: canvas and encoder rows)."""
+    import oracle
+
+    oracle_inputs(spec, case)
+    H, W = case.extra["H"], case.extra["W"]
+    clean = case.clean.numpy()
+    V = spec.vocab
+    if spec.mode == UNIFORM:
+        B, C, P = case.n_units, case.seq_len, spec.prefix
+        lay = oracle.Layout(B, C, None, None)
+        _, p = oracle.sample_t(seed, B, UNIFORM, spec.eps)
+        oracle.corrupt(lay, clean, p, UNIFORM, spec.mask_id, V, seed)
+        out = oracle.linear_loss_uniform(lay, H, W, clean, oracle.Layout(B, P + C, None, None),
+                                         case.extra["He"], case.enc_clean.numpy(), spec.enc_ar_weight,
+                                         spec.align)
+        return int(out["rows"].shape[0] + out["enc_rows"].shape[0])
+    lay = oracle.Layout(case.n_units, 0, case.cu_seqlens.numpy(), None)
+    _, p = oracle.sample_t(seed, case.n_units, ABSORBING, spec.eps)
+    _, corr = oracle.corrupt(lay, clean, p, ABSORBING, spec.mask_id, V, seed)
+    out = oracle.linear_loss(lay, H, W, clean, corr, p, align=spec.align)
+    return int(out["rows"].shape[0])
+
+
+def _full_rows(spec):
+    if spec.kind == "linear" and spec.mode == ABSORBING:
+        return spec.n_tokens_packed
+    return spec.seq_len
+
+
 def _calibrated_rows(spec, per_step_s, cap=1024):
     """Rows per sequence such that one oracle step takes about per_step_s."""
     import dlm_inputs as di
 
+    if spec.kind == "linear":
+        # a large fixed cost per step (W converted to double for each GEMM):
+        # two probe sizes separate it from the cost per row
+        times = []
+        for n in (16, 48):
+            sub = sample_spec(spec, n)
+            case = di.make_case(sub, "cpu")
+            oracle_step(sub, case, 0, n)                    # conversions, first-call costs
+            t0 = time.perf_counter()
+            oracle_step(sub, case, 1, n)
+            times.append(time.perf_counter() - t0)
+        per_row = max((times[1] - times[0]) / 32, 1e-9)
+        fixed = max(times[0] - 16 * per_row, 0.0)
+        rows = int(max(per_step_s - fixed, 0.0) / per_row)
+        return max(4, min(_full_rows(spec), cap, rows))
     probe = spec.scaled(seq_len=min(spec.seq_len, 16), prefix=min(spec.prefix, 16))
     case = di.make_case(probe, "cpu")
     oracle_step(probe, case, 0, probe.seq_len)          # first call builds / loads the oracle
@@ -548,10 +646,18 @@ def cpu_baseline(spec, budget_s=15.0, min_steps=3, max_steps=100_000, single_thr
     OMP_NUM_THREADS=1 (the oracle's OpenMP and numpy's BLAS read it at
     start-up)."""
     import dlm_inputs as di
+    import psutil
 
+    need = oracle_host_bytes(spec, 1024)
+    avail = psutil.virtual_memory().available
+    if need > 0.6 * avail:
+        return {"value": None, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+                "skipped": f"the oracle step needs ~{need / 1e9:.0f} GB of host memory, "
+                           f"{avail / 1e9:.0f} GB available"}
     rows = _calibrated_rows(spec, budget_s / min_steps)
-    sub = spec.scaled(seq_len=rows, prefix=min(spec.prefix, rows))
+    sub = sample_spec(spec, rows)
     case = di.make_case(sub, "cpu")
+    oracle_inputs(sub, case)
     t0 = time.perf_counter()
     scored = steps = 0
     while steps < min_steps or (steps < max_steps and time.perf_counter() - t0 < budget_s):
@@ -559,20 +665,22 @@ def cpu_baseline(spec, budget_s=15.0, min_steps=3, max_steps=100_000, single_thr
         steps += 1
     dt = time.perf_counter() - t0
     res = {"value": scored / dt, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
-           "sample": f"{steps} steps (seeds 1000..{999 + steps}) of the same workload cut to its "
-                     f"first {rows} rows per sequence ({spec.vocab}-wide rows; time draw, "
-                     f"corruption, CE of the scored rows, double-precision gradient of every "
-                     f"row): {dt:.1f} s"}
+           "sample": f"{steps} steps (seeds 1000..{999 + steps}) of the same workload cut to "
+                     f"{sample_words(spec, rows)[0]} (V = {spec.vocab}; {sample_words(spec, rows)[1]}): "
+                     f"{dt:.1f} s"}
     if single_thread_s > 0:
         env = dict(os.environ, OMP_NUM_THREADS="1", OPENBLAS_NUM_THREADS="1", MKL_NUM_THREADS="1")
+        import dataclasses
+        fields = json.dumps(dataclasses.asdict(spec))
         code = ("import json, bench, dlm_inputs as di; "
-                f"print(json.dumps(bench.cpu_baseline(di.WORKLOADS[{spec.key!r}], budget_s={single_thread_s}, "
-                "single_thread_s=0)))")
+                f"spec = di.Spec(**json.loads({fields!r})); "
+                f"print(json.dumps(bench.cpu_baseline(spec, budget_s={single_thread_s}, single_thread_s=0)))")
         try:
             r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True,
                                text=True, timeout=20 * single_thread_s + 120)
             one = json.loads(r.stdout.strip().splitlines()[-1])
-            res["single_thread"] = {"value": one["value"], "cores": one["cores"], "sample": one["sample"]}
+            res["single_thread"] = {"value": one["value"], "cores": one["cores"],
+                                    "sample": one.get("sample", one.get("skipped"))}
         except Exception as e:   # the all-cores figure stands on its own
             res["single_thread"] = {"value": None, "error": f"{type(e).__name__}: {e}"[:200]}
     return res
@@ -588,9 +696,16 @@ def run_reference(args):
     import dlm_inputs as di
 
     spec = di.WORKLOADS[args.workload]
+    need = oracle_host_bytes(spec, 1024)
+    if need > 0.6 * __import__("psutil").virtual_memory().available:
+        print(json.dumps({"impl": "reference",
+                          "unavailable": f"the CPU oracle needs ~{need / 1e9:.0f} GB of host memory "
+                                         "for this workload"}), flush=True)
+        return
     rows = _calibrated_rows(spec, 100.0 / (args.steps + args.warmup))
-    sub = spec.scaled(seq_len=rows, prefix=min(spec.prefix, rows))
+    sub = sample_spec(spec, rows)
     case = di.make_case(sub, "cpu")
+    oracle_inputs(sub, case)
     for i in range(args.warmup):
         oracle_step(sub, case, 10 + i, rows)
     t0 = time.perf_counter()
@@ -599,8 +714,8 @@ def run_reference(args):
         scored += oracle_step(sub, case, 1000 + i, rows)
     dt = time.perf_counter() - t0
     val = scored / dt
-    sample = (f"each step: the workload cut to its first {rows} rows per sequence (V={spec.vocab}); "
-              f"the oracle's whole path (time draw, corruption, CE, double-precision gradient)")
+    cut, work = sample_words(spec, rows)
+    sample = f"each step: the workload cut to {cut} (V = {spec.vocab}); the oracle's whole path ({work})"
     res = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",

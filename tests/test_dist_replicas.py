@@ -81,3 +81,27 @@ def test_cpu_baseline_all_cores_and_one_thread():
     assert "steps" in r["sample"] and r["unit"] == bench.UNIT
     one = r["single_thread"]
     assert one["cores"] == 1 and one["value"] > 0, one
+
+
+def test_cpu_baseline_fused_head_workloads(monkeypatch):
+    """The fused-head oracle as a CPU baseline, on small versions of both
+    fused-head workloads; and the skip when its host memory would not fit."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import dlm_inputs as di
+    small = {"lin_t16384_d4096_v126464": dict(n_tokens_packed=300, d_model=64, vocab=2048, ids_high=2000,
+                                              mask_id=2047),
+             "lin_unif_b4_p512_c1024_d4096_v262144": dict(n_units=2, seq_len=64, prefix=16, d_model=64,
+                                                          vocab=2048, ids_high=2047)}
+    for key, kw in small.items():
+        spec = di.WORKLOADS[key].scaled(**kw)
+        r = bench.cpu_baseline(spec, budget_s=0.5, single_thread_s=0.3)
+        assert r["value"] > 0 and "dH and dW" in r["sample"], r
+        assert r["single_thread"]["value"] > 0 and r["single_thread"]["cores"] == 1, r
+    import psutil
+
+    class _Mem:
+        available = 1 << 30
+    monkeypatch.setattr(psutil, "virtual_memory", lambda: _Mem())
+    r = bench.cpu_baseline(di.WORKLOADS["lin_unif_b4_p512_c1024_d4096_v262144"], single_thread_s=0)
+    assert r["value"] is None and "host memory" in r["skipped"]
