@@ -392,28 +392,11 @@ def linear_loss(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
     the unfused loss; dZ = grad_scale * w * (softmax - onehot); dH_M = dZ W,
     dW = dZ^T H_M, other rows of dH exactly zero."""
     plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, align)
-    rows = np.nonzero(plan.target >= 0)[0]
-    V, D = W.shape
-    Z = linear_logits(H[rows], W)
-    local = np.arange(rows.shape[0], dtype=np.int64)
-    lse, ce = ce_rows(Z, V, local, plan.target[rows])
-    row_loss = np.zeros(plan.target.shape[0], np.float64)
-    row_loss[rows] = plan.weight[rows] * ce
+    rows, lse, ce, row_loss, dH, dW = _linear_term(plan, H, W, grad_scale, want_grads)
     unit_loss = np.zeros(layout.n_units, np.float64)
     np.add.at(unit_loss, plan.unit, row_loss)
-    out = dict(loss=float(unit_loss.sum()), unit_loss=unit_loss, rows=rows, lse=lse, ce=ce,
-               plan=plan)
+    out = dict(loss=float(unit_loss.sum()), unit_loss=unit_loss, rows=rows, lse=lse, ce=ce, plan=plan)
     if want_grads:
-        dZ = grad_rows(Z, V, local, plan.target[rows], grad_scale * plan.weight[rows], lse)
-        del Z
-        Hd = bf16_to_f64(H[rows])
-        dH = np.zeros((H.shape[0], D), np.float64)
-        dW = np.zeros((V, D), np.float64)
-        chunk = 16384
-        for v0 in range(0, V, chunk):
-            Wd = bf16_to_f64(W[v0:v0 + chunk])
-            dH[rows] += dZ[:, v0:v0 + chunk] @ Wd
-            dW[v0:v0 + chunk] = dZ[:, v0:v0 + chunk].T @ Hd
         out.update(dH=dH, dW=dW)
     return out
 
@@ -424,19 +407,9 @@ def linear_rows(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
     """Full-size spot check: for a few scored rows only, their CE, weight*ce
     and their row of dH (which needs only that row's own softmax)."""
     plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, align)
-    sample_rows = np.asarray(sample_rows, np.int64)
-    assert (plan.target[sample_rows] >= 0).all()
-    V, D = W.shape
-    Z = linear_logits(H[sample_rows], W)
-    local = np.arange(sample_rows.shape[0], dtype=np.int64)
-    tgt = plan.target[sample_rows]
-    lse, ce = ce_rows(Z, V, local, tgt)
-    coef = grad_scale * plan.weight[sample_rows]
-    dZ = grad_rows(Z, V, local, tgt, coef, lse)
-    dH = np.zeros((sample_rows.shape[0], D), np.float64)
-    for v0 in range(0, V, 16384):
-        dH += dZ[:, v0:v0 + 16384] @ bf16_to_f64(W[v0:v0 + 16384])
-    return dict(ce=ce, lse=lse, weighted=plan.weight[sample_rows] * ce, dH=dH, plan=plan)
+    out = linear_rows_plan(plan, H, W, sample_rows, grad_scale)
+    out["plan"] = plan
+    return out
 
 
 def _linear_term(plan: RowPlan, H: np.ndarray, W: np.ndarray, grad_scale: float, want_grads: bool):
