@@ -11,6 +11,13 @@ than L2, so no flush between steps is needed).  Each timed step draws a new t
 (seed = 1000 + step), so the scored rows vary like in training.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+  python bench.py --workload lin_t16384_d4096_v126464      # fused head, absorbing
+  python bench.py --workload lin_unif_b4_p512_c1024_d4096_v262144   # fused head, uniform
+
+Besides the device-timed value, rank 0 at N=1 reports the CPU oracle on a
+bounded sample of the same workload (all cores and one thread) and, for the
+logits workloads, the same metric end to end with the inputs copied from
+pinned host memory every step.
 
 Multi-GPU: replicas only (the path has no data exchange); every rank runs the
 same workload on its own GPU, timing is the max over ranks, value = scored

@@ -10,9 +10,11 @@ Two layers:
     ``include/dlm.h`` (``dlm_sample_t``, ``dlm_corrupt``,
     ``dlm_loss_fwd_bwd``, ``dlm_linear_loss_fwd_bwd``, ...);
   * tensor helpers with the same names minus the prefix (``sample_t``,
-    ``corrupt``, ``loss_fwd_bwd``, ``linear_loss_fwd_bwd``) that allocate
-    outputs and workspace with torch on the current device and call the ABI
-    on the current torch stream.
+    ``corrupt``, ``loss_fwd_bwd``, ``linear_loss_fwd_bwd``,
+    ``linear_loss_uniform_fwd_bwd``) that check every tensor argument's
+    dtype, size against the layout and device, allocate outputs and
+    workspace with torch on the current device and call the ABI on the
+    current torch stream.
 """
 from __future__ import annotations
 
