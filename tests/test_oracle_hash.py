@@ -139,6 +139,22 @@ def test_p_floor_and_ceiling_exhaustive():
     assert np.array_equal(p[idx], po)
 
 
+def test_time_draw_is_stream_zero_of_the_unit():
+    """t of unit u is u24 of the hash at counter (stream 0, unit u, position
+    0), from the published generator and the counter layout pinned above."""
+    for mode in (oracle.ABSORBING, oracle.UNIFORM):
+        t, _ = oracle.sample_t(2024, 300, mode, 1e-3)
+        u = np.array([oracle.splitmix64_at(2024, oracle.counter(0, k, 0)) >> 40 for k in range(300)],
+                     np.float64) * 2.0 ** -24
+        if mode == oracle.ABSORBING:
+            assert np.array_equal(t.astype(np.float64), u)
+        else:   # t = fl(fl((1 - eps) u) + eps), monotone in u
+            order = np.argsort(u, kind="stable")
+            assert (np.diff(t[order]) >= 0).all()
+            c1 = np.float32(1.0) - np.float32(1e-3)
+            assert np.array_equal(t, (c1 * u.astype(np.float32)).astype(np.float32) + np.float32(1e-3))
+
+
 def test_time_draw_depends_on_seed_and_unit_only():
     t1, _ = oracle.sample_t(42, 10, oracle.ABSORBING, 1e-3)
     t2, _ = oracle.sample_t(42, 20, oracle.ABSORBING, 1e-3)
@@ -176,6 +192,22 @@ def test_corruption_threshold_is_strict_and_exact():
     for i in range(n):
         u24 = oracle.splitmix64_at(77, base + i) >> 40
         assert corr[i] == (1 if u24 < thr else 0)
+
+
+def test_corruption_threshold_equality_is_not_corrupted():
+    """A token whose draw equals p * 2^24 exactly is not corrupted (strict
+    compare): p is set to k / 2^24 for the k one token drew, exact in fp32."""
+    n = 4000
+    base = oracle.counter(1, 0, 0)
+    u24 = np.array([oracle.splitmix64_at(91, base + i) >> 40 for i in range(n)], np.int64)
+    i0 = int(np.argmax(u24 > 0))
+    k = int(u24[i0])
+    p = np.array([k * 2.0 ** -24], np.float32)
+    assert float(p[0]) * 2 ** 24 == k
+    lay = oracle.Layout(1, n, None, None)
+    _, corr = oracle.corrupt(lay, np.zeros(n, np.int32), p, oracle.ABSORBING, 1, 2, seed=91)
+    assert corr[i0] == 0
+    assert np.array_equal(corr, (u24 < k).astype(np.uint8))
 
 
 def test_uniform_replacement_histogram_and_rate():

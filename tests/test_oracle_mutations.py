@@ -236,3 +236,42 @@ def test_a_planted_mistake_fails_a_pin(monkeypatch, target, mutation, modules):
 
 def test_control_every_pin_passes_on_the_unmutated_oracle():
     assert _failing_pins(loss_pins, hash_pins) == []
+
+
+# ---- mistakes in the C part of the oracle ---------------------------------
+# Each case copies the oracle's C source, makes one textual change, compiles
+# the copy into the test's temporary directory and points the oracle at it;
+# the oracle's own source and library are not touched.
+C_MUTATIONS = [
+    ("splitmix_gamma", "#define DLMO_GAMMA 0x9E3779B97F4A7C15ULL", "#define DLMO_GAMMA 0x9E3779B97F4A7C17ULL"),
+    ("finaliser_shift", "z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ULL;", "z = (z ^ (z >> 29)) * 0xBF58476D1CE4E5B9ULL;"),
+    ("u24_cut", "return (uint32_t)(h >> 40);", "return (uint32_t)(h >> 41);"),
+    ("threshold_not_strict", "int c = (float)u24_of(h1) < thr;", "int c = (float)u24_of(h1) <= thr;"),
+    ("replacement_shift", "(uint64_t)(uint32_t)vocab) >> 32);", "(uint64_t)(uint32_t)vocab) >> 31);"),
+    ("uniform_t_without_floor", "else           { t[u] = v; p[u] = v; }", "else           { t[u] = x; p[u] = v; }"),
+    ("time_draw_stream", "dlmo_counter(0, (uint32_t)u, 0)", "dlmo_counter(1, (uint32_t)u, 0)"),
+    ("lse_without_max", "return m + log(s);", "return log(s);"),
+    ("bf16_decode_shift", "uint32_t w = (uint32_t)b << 16;", "uint32_t w = (uint32_t)b << 15;"),
+    ("grad_bf16_onehot_sign", "o[v] = coef[k] * (exp(buf[v] - lse[k]) - (v == targets[k] ? 1.0 : 0.0));",
+     "o[v] = coef[k] * (exp(buf[v] - lse[k]) + (v == targets[k] ? 1.0 : 0.0));"),
+    ("grad_f64_onehot_sign", "o[v] = coef[k] * (exp(x[v] - lse[k]) - (v == targets[k] ? 1.0 : 0.0));",
+     "o[v] = coef[k] * (exp(x[v] - lse[k]) + (v == targets[k] ? 1.0 : 0.0));"),
+    ("pads_not_skipped", "if (pad_mask && pad_mask[i])", "if (0 && pad_mask)"),
+    ("document_bound", "if (i >= cu[u] && i < cu[u + 1])", "if (i >= cu[u] && i <= cu[u + 1])"),
+]
+
+
+@pytest.mark.parametrize("old,new", [m[1:] for m in C_MUTATIONS], ids=[m[0] for m in C_MUTATIONS])
+def test_a_planted_mistake_in_the_c_oracle_fails_a_pin(monkeypatch, tmp_path, old, new):
+    import subprocess
+    src = open(oracle._build.SRC).read()
+    assert src.count(old) == 1, old
+    mutated = tmp_path / "dlm_oracle_mutated.c"
+    mutated.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mutated.so"
+    subprocess.run(["gcc", "-O2", "-std=c99", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-shared",
+                    "-fPIC", "-o", str(lib), str(mutated), "-lm"], check=True)
+    monkeypatch.setattr(oracle._build, "build", lambda *a, **kw: str(lib))
+    monkeypatch.setattr(oracle, "_lib", None)
+    failed = _failing_pins(loss_pins, hash_pins)
+    assert failed, f"no pin notices the change {old!r} -> {new!r}"
