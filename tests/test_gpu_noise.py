@@ -87,6 +87,20 @@ def test_corrupt_threshold_edges():
         assert np.array_equal(g_corr, o_corr) and np.array_equal(g_noisy, o_noisy)
 
 
+def test_corrupt_draw_exactly_on_the_threshold():
+    """A token whose 24-bit draw equals p * 2^24 stays clean, on the GPU as in
+    the oracle (strict compare): p = k / 2^24 for the k one token drew."""
+    n = 4000
+    base = oracle.counter(1, 0, 0)
+    u24 = np.array([oracle.splitmix64_at(91, base + i) >> 40 for i in range(n)], np.int64)
+    i0 = int(np.argmax(u24 > 0))
+    p = np.array([int(u24[i0]) * 2.0 ** -24], np.float32)
+    clean = np.zeros(n, np.int32)
+    g_noisy, g_corr, o_noisy, o_corr, st = _corrupt_both(1, n, None, None, clean, p, oracle.ABSORBING, 1, 2, 91)
+    assert st == 0 and g_corr[i0] == 0 and o_corr[i0] == 0
+    assert np.array_equal(g_corr, o_corr) and np.array_equal(g_noisy, o_noisy)
+
+
 def test_corrupt_flags_bad_cu_seqlens():
     cu = np.array([0, 10, 4, 20], np.int32)       # not non-decreasing
     clean = np.zeros(20, np.int32)
