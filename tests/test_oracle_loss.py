@@ -271,6 +271,33 @@ def test_encoder_term_is_plain_causal_ce():
     assert abs(loss - (math.log(V) + lam * causal)) < 1e-12
 
 
+def test_encoder_term_with_pads_brute_force():
+    """Encoder sequences with trailing pads: the term is the mean textbook CE
+    over exactly the next-token pairs whose target is a real token of the
+    same sequence, enumerated here one by one."""
+    rng = np.random.default_rng(11)
+    B, S, V = 3, 9, 23
+    lengths = (9, 4, 1)                      # real tokens per sequence, then pads
+    pad = np.zeros(B * S, np.uint8)
+    for b, n in enumerate(lengths):
+        pad[b * S + n:(b + 1) * S] = 1
+    enc = oracle.Layout(B, S, None, pad)
+    ids = rng.integers(0, V, B * S).astype(np.int32)
+    x = rng.standard_normal((B * S, V)) * 2
+    rows, tgts = [], []
+    for b in range(B):
+        for i in range(S - 1):
+            if i + 1 < lengths[b]:
+                rows.append(b * S + i)
+                tgts.append(ids[b * S + i + 1])
+    want = torch.nn.functional.cross_entropy(torch.from_numpy(x[rows]),
+                                             torch.from_numpy(np.array(tgts, np.int64))).item()
+    lam = 1.3
+    tr = oracle.term(x, V, oracle.plan_encoder(enc, ids, lam))
+    assert sorted(tr.rows.tolist()) == rows
+    assert abs(tr.row_loss.sum() - lam * want) < 1e-12
+
+
 # --------------------------------------------------------------------------
 # uniform noise: 1/(1-t) time weighting with a cap, per-example mean
 # --------------------------------------------------------------------------

@@ -153,6 +153,56 @@ def m_reduce_wrong_unit(real):
     return f
 
 
+def m_rhine_cap_ignored(real):
+    def f(layout, clean, corrupted, p, mode, align, time_weighting=oracle.NO_TIME_WEIGHT, weight_clip=0.0,
+          reduction=oracle.TOKEN_MEAN):
+        return real(layout, clean, corrupted, p, mode, align, time_weighting, 0.0, reduction)
+    return f
+
+
+def m_example_mean_over_all_examples(real):
+    def f(layout, clean, corrupted, p, mode, align, time_weighting=oracle.NO_TIME_WEIGHT, weight_clip=0.0,
+          reduction=oracle.TOKEN_MEAN):
+        plan = real(layout, clean, corrupted, p, mode, align, time_weighting, weight_clip, reduction)
+        if reduction == oracle.EXAMPLE_MEAN and layout.n_units > 0:
+            b_eff = len(set(plan.unit[plan.target >= 0].tolist()))
+            plan.weight *= b_eff / layout.n_units
+        return plan
+    return f
+
+
+def m_rhine_inverse_t(real):
+    def f(layout, clean, corrupted, p, mode, align, time_weighting=oracle.NO_TIME_WEIGHT, weight_clip=0.0,
+          reduction=oracle.TOKEN_MEAN):
+        plan = real(layout, clean, corrupted, p, mode, align, time_weighting, weight_clip, reduction)
+        if time_weighting == oracle.INV_ONE_MINUS_T:
+            t = p.astype(np.float64)
+            right = 1.0 / (1.0 - t)
+            wrong = 1.0 / t
+            if weight_clip > 0:
+                right, wrong = np.minimum(right, weight_clip), np.minimum(wrong, weight_clip)
+            s = plan.target >= 0
+            plan.weight[s] *= (wrong / right)[plan.unit[s]]
+        return plan
+    return f
+
+
+def m_encoder_scores_pads(real):
+    def f(layout, clean, lam):
+        plan = real(layout, clean, lam)
+        unit = layout.unit_of_token()
+        nonpad = layout.nonpad()
+        extra = [i for i in range(layout.n_tokens - 1)
+                 if plan.target[i] < 0 and unit[i + 1] == unit[i] and not nonpad[i + 1]]
+        if extra:
+            plan.target[extra] = np.asarray(clean)[np.asarray(extra) + 1]
+            cnt = int((plan.target >= 0).sum())
+            plan.weight[:] = 0.0
+            plan.weight[plan.target >= 0] = lam / cnt
+        return plan
+    return f
+
+
 # ---- mistakes in the fused head -------------------------------------------
 def m_linear_dw_dropped(real):
     def f(plan, H, W, grad_scale, want_grads):
@@ -217,6 +267,10 @@ MUTATIONS = [
     ("plan_encoder", m_encoder_without_lambda, (loss_pins,)),
     ("plan_encoder", m_encoder_crosses_units, (loss_pins,)),
     ("reduce_units", m_reduce_wrong_unit, (loss_pins,)),
+    ("plan_diffusion", m_rhine_cap_ignored, (loss_pins,)),
+    ("plan_diffusion", m_example_mean_over_all_examples, (loss_pins,)),
+    ("plan_diffusion", m_rhine_inverse_t, (loss_pins,)),
+    ("plan_encoder", m_encoder_scores_pads, (loss_pins,)),
     ("_linear_term", m_linear_dw_dropped, (loss_pins,)),
     ("_linear_term", m_linear_dh_on_wrong_rows, (loss_pins,)),
     ("linear_loss_uniform", m_linear_uniform_encoder_dw_dropped, (loss_pins,)),
