@@ -200,3 +200,9 @@ def test_oracle_and_product_share_no_code():
         if f.endswith((".py", ".c")):
             txt = open(os.path.join(ROOT, "oracle", f)).read()
             assert "diffusion_lm_loss_b200" not in txt and "dlm.h" not in txt
+    # the seeded input module both sides use imports neither of them
+    for f in os.listdir(os.path.join(ROOT, "dlm_inputs")):
+        if f.endswith(".py"):
+            txt = open(os.path.join(ROOT, "dlm_inputs", f)).read()
+            for name in ("oracle", "diffusion_lm_loss_b200"):
+                assert f"import {name}" not in txt and f"from {name}" not in txt
