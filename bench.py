@@ -15,9 +15,9 @@ than L2, so no flush between steps is needed).  Each timed step draws a new t
   python bench.py --workload lin_unif_b4_p512_c1024_d4096_v262144   # fused head, uniform
 
 Besides the device-timed value, rank 0 at N=1 reports the CPU oracle on a
-bounded sample of the same workload (all cores and one thread) and, for the
-logits workloads, the same metric end to end with the inputs copied from
-pinned host memory every step.
+bounded sample of the same workload (all cores and one thread), and the same
+metric end to end with each step's inputs copied from pinned host memory
+(the logits workloads at every N, the fused-head workloads at N=1).
 
 Multi-GPU: replicas only (the path has no data exchange); every rank runs the
 same workload on its own GPU, timing is the max over ranks, value = scored
@@ -441,21 +441,34 @@ def run_linear(args, spec, dev, rank, world):
     ms = t0.elapsed_time(t1)
     call_ms = sum(a.elapsed_time(b) for a, b in evs) / K
     clk = clocks.stop() if rank == 0 else None
-    scored = 0
-    for i in range(K if not uniform else 0):
+    per_step = []
+    for i in range(K):
+        if uniform:
+            # every canvas target (each unit's first token is none when
+            # shifted) and every encoder next-token pair
+            per_step.append(B * (C - (1 if align == dlm.SHIFTED else 0)) + B * (P + C - 1))
+            continue
         t, p = dlm.sample_t(1000 + i, case.n_units, spec.mode, spec.eps)
         _, corr = dlm.corrupt(lay, case.clean, p, spec.mode, spec.mask_id, V, 1000 + i)
-        scored += int(corr.sum().item())
+        n = int(corr.sum().item())
         if align == dlm.SHIFTED:
             # a document's first token is never a target when rows score the next token
             cu = case.cu_seqlens.to(torch.int64)
             first = cu[:-1][cu[1:] > cu[:-1]]
-            scored -= int(corr[first].sum().item())
-    if uniform:
-        # every canvas target (each unit's first token is none when shifted)
-        # and every encoder next-token pair
-        scored = K * (B * (C - (1 if align == dlm.SHIFTED else 0)) + B * (P + C - 1))
+            n -= int(corr[first].sum().item())
+        per_step.append(n)
+    scored = sum(per_step)
     ms, call_ms, scored_all = reduce_over_ranks(ms, call_ms, scored, dev)
+
+    # e2e (one GPU): the step's inputs -- hidden states, ids, document
+    # offsets -- copied from pinned host memory every step, the loss read back;
+    # the head's weight is a resident parameter
+    e2e = None
+    if world == 1 and not args.no_e2e:
+        try:
+            e2e = _linear_e2e(args, spec, case, lay, enc if uniform else None, align, per_step, out)
+        except Exception as ex:       # the device-timed figures above stand without it
+            e2e = {"value": None, "error": f"{type(ex).__name__}: {ex}"[:300]}
     value = scored_all / (ms / 1e3)
     M = scored_all / world / K
     flops = 6.0 * M * D * V
@@ -491,11 +504,56 @@ def run_linear(args, spec, dev, rank, world):
                       "tokens": T, "d_model": D, "encoder_ar_weight": spec.enc_ar_weight if uniform else None,
                       "vocab": V, "documents": case.n_units, "parallelism": f"replicas{world}",
                       "scored_tokens": scored_all, "l2": "inputs larger than L2 (W %.2f GB)" % (V * D * 2 / 1e9)},
-           "roofline": roof, "cpu_baseline": cpu, "clocks": clk, "e2e": None,
+           "roofline": roof, "cpu_baseline": cpu, "clocks": clk, "e2e": e2e,
            # per step: time draw, corruption, plan, gather, forward GEMM, lse,
            # dZ + dH + dW per 16,384-column vocabulary chunk, scatter, reduce
            "gpu_launches": K * (6 + 3 * ((V + 16383) // 16384) + 2)}
     print(json.dumps(res), flush=True)
+
+
+def _linear_e2e(args, spec, case, lay, enc, align, per_step, out):
+    """The fused-head call end to end on one GPU: every step copies its inputs
+    from pinned host memory, runs time draw, corruption and the loss through
+    the public API, and reads the loss back.  Seeds 1000.. as the timed
+    steps, so the scored rows are those steps' counts."""
+    import torch
+
+    import diffusion_lm_loss_b200 as dlm
+
+    uniform = enc is not None
+    Ke = max(1, min(args.steps, args.e2e_steps))
+    dev_in = [case.hidden, case.clean] + ([case.enc_hidden, case.enc_clean] if uniform else [case.cu_seqlens])
+    host_in = [t.cpu().pin_memory() for t in dev_in]
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    h_loss = torch.empty(Ke, dtype=torch.float32).pin_memory()
+    V = spec.vocab
+
+    def e2e_step(i):
+        nonlocal out
+        for d, h in zip(dev_in, host_in):
+            d.copy_(h, non_blocking=True)
+        t, p = dlm.sample_t(1000 + i, case.n_units, spec.mode, spec.eps)
+        _, corr = dlm.corrupt(lay, case.clean, p, spec.mode, spec.mask_id, V, 1000 + i)
+        if uniform:
+            out = dlm.linear_loss_uniform_fwd_bwd(lay, case.hidden, case.weight, case.clean, enc, case.enc_hidden,
+                                                  case.enc_clean, enc_ar_weight=spec.enc_ar_weight, align=align,
+                                                  out=out)
+        else:
+            out = dlm.linear_loss_fwd_bwd(lay, case.hidden, case.weight, case.clean, corr, p, out=out, align=align)
+        h_loss[i:i + 1].copy_(out.loss, non_blocking=True)
+
+    e2e_step(0)
+    torch.cuda.synchronize()
+    s0 = torch.cuda.Event(enable_timing=True)
+    s1 = torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for i in range(Ke):
+        e2e_step(i)
+    s1.record()
+    torch.cuda.synchronize()
+    e_ms = s0.elapsed_time(s1)
+    return {"value": sum(per_step[:Ke]) / (e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": 4, "steps": Ke, "ms_per_step": e_ms / Ke}
 
 
 # ---------------------------------------------------------------------------
