@@ -11,13 +11,11 @@
 // process exits.
 //
 // The entry point allocates nothing: it finds the array's device address
-// (once per device, see below) and forwards to dlm_loss_fwd_bwd with that
-// address as the workspace.  Everything the loss needs zeroed at the start of
+// (see below) and forwards to dlm_loss_fwd_bwd with that address as the
+// workspace.  Everything the loss needs zeroed at the start of
 // a call is cleared by the loss itself on every call (its row-plan kernel
 // rewrites the header and the completion counter), so the contents a previous
 // call left in the array do no harm.
-#include <mutex>
-
 #include "dlm_host.h"
 
 namespace dlm {
@@ -27,26 +25,21 @@ namespace dlm {
 // cudaGetSymbolAddress below.
 static __device__ __align__(256) uint8_t g_loss_scratch[DLM_STATIC_SCRATCH_BYTES];
 
-// Device address of g_loss_scratch on the current device, looked up on the
-// first call made on that device (with that device current) and cached.
+// Device address of g_loss_scratch in the context current on the calling
+// thread.  Looked up on every call, not cached: the address belongs to the
+// context that loaded this library's device code, and a caller may run under
+// a context other than the device's primary one, or reset the device between
+// calls, after which a cached address would point at memory that is gone.
+// The lookup is a host-side table query and allocates nothing; the first one
+// in a context also loads the library's device code into it.
 static dlm_status_t scratch_address(void** out) {
-    static std::mutex mu;
-    static void* addr[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) { cudaGetLastError(); return cuda_status(e, "cudaGetDevice"); }
-    if (dev < 0 || dev >= 64) return DLM_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> g(mu);
-    if (!addr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_loss_scratch);
-        if (e != cudaSuccess || !p) {
-            cudaGetLastError();
-            return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
-        }
-        addr[dev] = p;
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_loss_scratch);
+    if (e != cudaSuccess || !p) {
+        cudaGetLastError();
+        return cuda_status(e != cudaSuccess ? e : cudaErrorInvalidSymbol, "cudaGetSymbolAddress(scratch)");
     }
-    *out = addr[dev];
+    *out = p;
     return DLM_OK;
 }
 

@@ -263,9 +263,11 @@ DLM_API dlm_status_t dlm_loss_fwd_bwd_ex(const dlm_layout_t *layout, const uint1
  * exceeds DLM_STATIC_SCRATCH_BYTES is refused with
  * DLM_ERR_WORKSPACE_TOO_SMALL before anything is enqueued (2 MiB fits about
  * 100,000 logits rows, diffusion plus encoder, over a few thousand units).
- * The first call on a device looks up the array's device address with that
- * device current and caches it; make that first call before any stream
- * capture.  All calls share the one array: calls that overlap on the GPU (on
+ * Every call looks up the array's device address in the context current on
+ * the calling thread (no address is cached, so non-primary contexts and a
+ * device reset between calls are safe).  The first call in a context also
+ * loads this library's device code there; make that first call before any
+ * stream capture.  All calls share the one array: calls that overlap on the GPU (on
  * different streams, or from different host threads without ordering) race
  * and corrupt each other's results; order them on one stream.  Each call
  * re-initialises what it needs, so contents left by an earlier call are

@@ -73,7 +73,7 @@ def test_every_entry_point_reports_its_cuda_failure(L):
         _fails_at(L, L.dlm_loss_fwd_bwd_ex(lp, 4096, 1000, 1000, 256, 512, 768, 0, 0, None, None, 0, None,
                                            1.0, 1.0, None, 1024, 1280, 8192, None, WS, ws_l, None), "k_plan")
         _fails_at(L, L.dlm_loss_fwd_bwd_static(lp, 4096, 1000, 1000, 256, 512, 768, 0, 0, None, None, 0,
-                                               None, 1.0, 1.0, 1024, 1280, 8192, None, None), "cudaGetDevice")
+                                               None, 1.0, 1.0, 1024, 1280, 8192, None, None), "cudaGetSymbolAddress(scratch)")
         _fails_at(L, L.dlm_linear_loss_fwd_bwd(lp, 4096, 8192, 64, 1024, 256, 512, 768, 1.0, 1024, 1280,
                                                16384, 32768, WS, ws_h, None), "k_plan")
         _fails_at(L, L.dlm_linear_loss_fwd_bwd_ex(lp, 4096, 8192, 64, 1024, 256, 512, 768, 1, 1.0, 1024,
