@@ -16,6 +16,15 @@ Shapes follow the pages:
 The datasets the pages train on (Nemotron-SFT-Code and others) are not used;
 these synthetic draws stand in for them.
 
+Typed-decision workloads (label slots of multiple-choice, score and yes/no
+questions: "Native diffusion language-model training", Typed-decision
+training and Labels) draw, from the CPU generator: a codebook of 128
+distinct answer-token ids; per slot K ~ U[2, k_max] alternatives, answered by
+the first K codebook tokens (every question spells its answers A, B, C, ...);
+a label kind uniform over hard / dist / set with a uniform gold index, a
+Dirichlet(1) distribution, or a uniform non-empty subset; then, on the
+device generator, the slots' logits rows.
+
 Draw order for a given seed (a fixed recipe, so a seed names one input):
   1. packed-document lengths (packed workloads only; CPU generator);
   2. clean ids;
@@ -59,6 +68,7 @@ class Spec:
     w_std: float = 0.02
     eps: float = 1e-3
     enc_ar_weight: float = 0.0
+    k_max: int = 0             # decision: alternatives per question in [2, k_max]
     data_seed: int = 0
     corrupt_seed: int = 0
     description: str = ""
@@ -108,6 +118,12 @@ WORKLOADS = {
         description="DiffusionGemma-like uniform-token noise through a fused lm_head: B=4, "
                     "prefix 512 + canvas 1024, D=4096, V=262144, canvas and encoder hidden "
                     "states against one head, encoder AR weight 1"),
+    "dec_s128_k26_v126464": Spec(
+        "dec_s128_k26_v126464", "decision", ABSORBING, ALIGNED, vocab=126464, mask_id=126336,
+        ids_high=126335, n_units=128, std=3.0, k_max=26, data_seed=8,
+        description="typed-decision losses at 128 label slots (16 canvases x 8 questions), answer "
+                    "tokens from a 26-letter codebook (K in [2, 26]), hard / dist / set labels, "
+                    "logits at the label slots only, V=126464"),
     "lin_t4096_d4096_v32768": Spec(
         "lin_t4096_d4096_v32768", "linear", ABSORBING, ALIGNED, vocab=32768,
         mask_id=32767, ids_high=32000, n_tokens_packed=4096, d_model=4096,
@@ -177,6 +193,9 @@ def make_case(spec: Spec, device="cpu", seed: Optional[int] = None,
     cpu_gen = torch.Generator()
     cpu_gen.manual_seed(seed)
 
+    if spec.kind == "decision":
+        return _decision_case(spec, dev, gen, cpu_gen, with_tensors)
+
     if spec.kind == "linear" and spec.mode == UNIFORM:
         B, C, P = spec.n_units, spec.seq_len, spec.prefix
         full = torch.randint(0, spec.ids_high + 1, (B, P + C), generator=gen, device=dev,
@@ -231,6 +250,38 @@ def make_case(spec: Spec, device="cpu", seed: Optional[int] = None,
             case.logits = logits
         else:
             case.logits = _normal_bf16(B * L, spec.vocab, spec.std, gen, dev)
+    return case
+
+
+HARD, DIST, SET = 0, 1, 2       # label kinds
+
+
+def _decision_case(spec: Spec, dev, gen, cpu_gen, with_tensors: bool) -> Case:
+    n = spec.n_units
+    codebook = torch.randperm(spec.ids_high + 1, generator=cpu_gen)[:128].to(torch.int32)
+    K = torch.randint(2, spec.k_max + 1, (n,), generator=cpu_gen)
+    kind = torch.randint(0, 3, (n,), generator=cpu_gen).to(torch.int32)
+    off = torch.zeros(n + 1, dtype=torch.int32)
+    off[1:] = torch.cumsum(K, 0).to(torch.int32)
+    ids, vals = [], []
+    for i in range(n):
+        k = int(K[i])
+        ids.append(codebook[:k])
+        v = torch.zeros(k, dtype=torch.float32)
+        if kind[i] == HARD:
+            v[int(torch.randint(0, k, (1,), generator=cpu_gen))] = 1.0
+        elif kind[i] == DIST:
+            e = torch.empty(k, dtype=torch.float64).exponential_(generator=cpu_gen)
+            v = (e / e.sum()).to(torch.float32)
+        else:
+            m = int(torch.randint(1, k + 1, (1,), generator=cpu_gen))
+            v[torch.randperm(k, generator=cpu_gen)[:m]] = 1.0
+        vals.append(v)
+    case = Case(spec, n, 0, None, None, torch.zeros(n, dtype=torch.int32, device=dev))
+    case.extra.update(cand_off=off.to(dev), cand_ids=torch.cat(ids).to(dev), kind=kind.to(dev),
+                      val=torch.cat(vals).to(dev))
+    if with_tensors:
+        case.logits = _normal_bf16(n, spec.vocab, spec.std, gen, dev)
     return case
 
 

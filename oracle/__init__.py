@@ -384,20 +384,23 @@ def linear_logits(H_rows: np.ndarray, W: np.ndarray, chunk: int = 16384) -> np.n
 
 def linear_loss(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
                 corrupted: np.ndarray, p: np.ndarray, grad_scale: float = 1.0,
-                want_grads: bool = True, align: int = ALIGNED):
+                want_grads: bool = True, align: int = ALIGNED, keep_dz: bool = False):
     """[Axolotl] CCE path, absorbing noise.  The rows of H that score a
     target (aligned: row i scores token i, as CCE does on the page; shifted:
     row i scores token i+1 of the same unit, the unfused loss's Dream
     reading carried over) form Z = H_M W^T in double; CE and weights as for
     the unfused loss; dZ = grad_scale * w * (softmax - onehot); dH_M = dZ W,
-    dW = dZ^T H_M, other rows of dH exactly zero."""
+    dW = dZ^T H_M, other rows of dH exactly zero.  keep_dz: also return dZ
+    ([scored rows, V], double) for the tests' error scales."""
     plan = plan_diffusion(layout, clean, corrupted, p, ABSORBING, align)
-    rows, lse, ce, row_loss, dH, dW = _linear_term(plan, H, W, grad_scale, want_grads)
+    rows, lse, ce, row_loss, dH, dW, dZ = _linear_term(plan, H, W, grad_scale, want_grads, keep_dz)
     unit_loss = np.zeros(layout.n_units, np.float64)
     np.add.at(unit_loss, plan.unit, row_loss)
     out = dict(loss=float(unit_loss.sum()), unit_loss=unit_loss, rows=rows, lse=lse, ce=ce, plan=plan)
     if want_grads:
         out.update(dH=dH, dW=dW)
+    if keep_dz:
+        out.update(dZ=dZ)
     return out
 
 
@@ -412,10 +415,12 @@ def linear_rows(layout: Layout, H: np.ndarray, W: np.ndarray, clean: np.ndarray,
     return out
 
 
-def _linear_term(plan: RowPlan, H: np.ndarray, W: np.ndarray, grad_scale: float, want_grads: bool):
+def _linear_term(plan: RowPlan, H: np.ndarray, W: np.ndarray, grad_scale: float, want_grads: bool,
+                 keep_dz: bool = False):
     """One term of a fused-head loss: the scored rows of H (by `plan`) form
-    Z = H_M W^T in double; returns (rows, lse, ce, row_loss, dH, dW), dH over
-    all rows of H (zeros on unscored rows), dW = dZ^T H_M ([V, D])."""
+    Z = H_M W^T in double; returns (rows, lse, ce, row_loss, dH, dW, dZ), dH
+    over all rows of H (zeros on unscored rows), dW = dZ^T H_M ([V, D]), dZ
+    only when keep_dz (else None)."""
     rows = np.nonzero(plan.target >= 0)[0]
     V, D = W.shape
     Z = linear_logits(H[rows], W)
@@ -434,26 +439,31 @@ def _linear_term(plan: RowPlan, H: np.ndarray, W: np.ndarray, grad_scale: float,
             Wd = bf16_to_f64(W[v0:v0 + 16384])
             dH[rows] += dZ[:, v0:v0 + 16384] @ Wd
             dW[v0:v0 + 16384] = dZ[:, v0:v0 + 16384].T @ Hd
-    return rows, lse, ce, row_loss, dH, dW
+        if not keep_dz:
+            dZ = None
+    else:
+        dZ = None
+    return rows, lse, ce, row_loss, dH, dW, dZ
 
 
 def linear_loss_uniform(canvas: Layout, H: np.ndarray, W: np.ndarray, canvas_clean: np.ndarray,
                         encoder: Optional[Layout], He: Optional[np.ndarray],
                         enc_clean: Optional[np.ndarray], lam: float, align: int = ALIGNED,
-                        grad_scale: float = 1.0, want_grads: bool = True):
+                        grad_scale: float = 1.0, want_grads: bool = True, keep_dz: bool = False):
     """[Gemma] uniform-noise objective through a plain linear head, without a
     logits tensor ([Axolotl] Cut Cross Entropy carried to uniform noise):
     canvas term = mean CE of every non-pad canvas target (row i scores token
     i, or token i+1 of the same unit when shifted) on Z = H W^T; encoder term
     = lam * mean next-token CE over the clean full sequence on Ze = He W^T.
     dH, dHe = dZ W, dZe W (zeros on unscored rows); dW = dZ^T H_M + dZe^T He_M,
-    one shared head.  H, He, W: uint16 bf16 bits [T, D], [Te, D], [V, D]."""
+    one shared head.  H, He, W: uint16 bf16 bits [T, D], [Te, D], [V, D].
+    keep_dz: also return dZ and dZe (double, [scored rows, V] per term)."""
     pc = plan_diffusion(canvas, canvas_clean, None, None, UNIFORM, align)
-    tc = _linear_term(pc, H, W, grad_scale, want_grads)
+    tc = _linear_term(pc, H, W, grad_scale, want_grads, keep_dz)
     terms = [(pc, tc)]
     if encoder is not None:
         pe = plan_encoder(encoder, enc_clean, lam)
-        terms.append((pe, _linear_term(pe, He, W, grad_scale, want_grads)))
+        terms.append((pe, _linear_term(pe, He, W, grad_scale, want_grads, keep_dz)))
     unit_loss = np.zeros(canvas.n_units, np.float64)
     for plan, t in terms:
         np.add.at(unit_loss, plan.unit, t[3])
@@ -464,6 +474,8 @@ def linear_loss_uniform(canvas: Layout, H: np.ndarray, W: np.ndarray, canvas_cle
         out.update(dH=tc[4], dW=tc[5] + (terms[1][1][5] if encoder is not None else 0.0))
         if encoder is not None:
             out.update(dHe=terms[1][1][4])
+    if keep_dz:
+        out.update(dZ=tc[6], dZe=terms[1][1][6] if encoder is not None else None)
     return out
 
 
@@ -483,3 +495,114 @@ def linear_rows_plan(plan: RowPlan, H: np.ndarray, W: np.ndarray, sample_rows: n
     for v0 in range(0, V, 16384):
         dH += dZ[:, v0:v0 + 16384] @ bf16_to_f64(W[v0:v0 + 16384])
     return dict(ce=ce, lse=lse, weighted=plan.weight[sample_rows] * ce, dH=dH)
+
+
+# --------------------------------------------------------------------------
+# Typed-decision losses at label slots ([Axolotl] "Typed-decision training",
+# "Labels"; "Adapters, merging and inference": the restricted-label and Brier
+# terms are computed over the allowed answers)
+# --------------------------------------------------------------------------
+HARD, DIST, SET = 0, 1, 2                       # label kinds
+LABEL_RESTRICTED, LABEL_FULL, LABEL_BOTH = 1, 2, 3   # labels.label_softmax
+
+
+def decision_targets(kind: int, val: np.ndarray, smoothing: float):
+    """The CE target q and the Brier target y of one label over its K
+    alternatives, in double.  `val` holds one value per alternative:
+    hard -- 1 at the gold index, 0 elsewhere; dist -- the probabilities;
+    set -- 1 for each allowed index, 0 elsewhere.
+      hard: y = one-hot; q = (1 - smoothing) one-hot + smoothing / K
+            (hard_label_smoothing spreads that fraction of the one-hot CE
+            target uniformly over the question's K answer tokens; the Brier
+            target is unchanged);
+      dist: q = y = the probabilities as given;
+      set:  q = y = uniform over the allowed indexes (reading: each allowed
+            answer equally right)."""
+    val = np.asarray(val, np.float64)
+    K = val.shape[0]
+    if K < 1:
+        raise ValueError("a question has at least one alternative")
+    if kind == HARD:
+        if not (np.count_nonzero(val) == 1 and val.max() == 1.0 and val.min() == 0.0):
+            raise ValueError("hard label: exactly one 1, zeros elsewhere")
+        y = val.copy()
+        q = (1.0 - smoothing) * y + smoothing / K
+    elif kind == DIST:
+        if not (np.isfinite(val).all() and (val >= 0).all()):
+            raise ValueError("dist label: finite, non-negative probabilities")
+        y = val.copy()
+        q = val.copy()
+    elif kind == SET:
+        if not (((val == 0.0) | (val == 1.0)).all() and val.sum() >= 1):
+            raise ValueError("set label: a non-empty 0/1 membership")
+        y = val / val.sum()
+        q = y.copy()
+    else:
+        raise ValueError(f"label kind {kind}")
+    return q, y
+
+
+def decision_loss(logits: np.ndarray, vocab: int, slot_rows: Optional[np.ndarray], cand_off: np.ndarray,
+                  cand_ids: np.ndarray, kind: np.ndarray, val: np.ndarray,
+                  label_softmax: int = LABEL_BOTH, brier_weight: float = 0.1, smoothing: float = 0.0,
+                  grad_scale: float = 1.0):
+    """Typed-decision loss over n label slots, each one logits row z (bf16
+    bits uint16 [rows, ld] or float64) and its question's K answer tokens
+    a_0..a_{K-1} (distinct ids; cand_ids[cand_off[i]:cand_off[i+1]]):
+      r = softmax over the K candidate logits z[a_k] (candidate-restricted);
+      P = softmax over the whole vocabulary;
+      CE_res  = -sum_k q_k log r_k            (label_softmax restricted/both)
+      CE_full = -sum_k q_k log P(a_k)         (label_softmax full/both; the
+                full-vocabulary softmax still penalises probability outside
+                the valid answers)
+      Brier   = sum_k (r_k - y_k)^2,  weighted by brier_weight (0.1 on the
+                page), over the restricted distribution
+      loss    = (1/n) sum over slots of the selected terms (reading: the mean
+                over label slots).
+    Returns loss, the per-slot contribution (its terms / n), the three terms
+    per slot, and dlogits = grad_scale * d loss / dz ([n, vocab], double)."""
+    n = int(cand_off.shape[0]) - 1
+    rows = np.arange(n) if slot_rows is None else np.asarray(slot_rows, np.int64)
+    if logits.dtype == np.uint16:
+        z_all = bf16_to_f64(np.ascontiguousarray(logits[rows, :vocab]))
+    else:
+        z_all = np.asarray(logits[rows, :vocab], np.float64)
+    use_res = label_softmax in (LABEL_RESTRICTED, LABEL_BOTH)
+    use_full = label_softmax in (LABEL_FULL, LABEL_BOTH)
+    ce_res = np.zeros(n)
+    ce_full = np.zeros(n)
+    brier = np.zeros(n)
+    grad = np.zeros((n, vocab))
+    w = 1.0 / n if n > 0 else 0.0
+    for i in range(n):
+        z = z_all[i]
+        a = np.asarray(cand_ids[cand_off[i]:cand_off[i + 1]], np.int64)
+        if a.size == 0 or np.unique(a).size != a.size or a.min() < 0 or a.max() >= vocab:
+            raise ValueError(f"slot {i}: answer tokens must be distinct ids in [0, vocab)")
+        q, y = decision_targets(int(kind[i]), val[cand_off[i]:cand_off[i + 1]], smoothing)
+        Q = q.sum()
+        # full-vocabulary softmax
+        m = z.max()
+        lse = m + np.log(np.exp(z - m).sum())
+        P = np.exp(z - lse)
+        # candidate-restricted softmax
+        c = z[a]
+        cm = c.max()
+        lse_r = cm + np.log(np.exp(c - cm).sum())
+        r = np.exp(c - lse_r)
+        ce_res[i] = -(q * (c - lse_r)).sum()
+        ce_full[i] = -(q * (c - lse)).sum()
+        brier[i] = ((r - y) ** 2).sum()
+        g = np.zeros(vocab)
+        if use_full:                      # d CE_full / dz_v = Q P_v - q(v)
+            g += Q * P
+            g[a] -= q
+        if use_res:                       # d CE_res / dz_{a_k} = Q r_k - q_k
+            g[a] += Q * r - q
+        # d Brier / dz_{a_j} = 2 r_j ((r_j - y_j) - sum_k r_k (r_k - y_k))
+        d = r - y
+        g[a] += brier_weight * 2.0 * r * (d - (r * d).sum())
+        grad[i] = grad_scale * w * g
+    per_slot = (ce_res * use_res + ce_full * use_full + brier_weight * brier) * w
+    return dict(loss=float(per_slot.sum()), slot_loss=per_slot, ce_res=ce_res, ce_full=ce_full,
+                brier=brier, dlogits=grad)

@@ -15,6 +15,7 @@ import numpy as np
 import pytest
 
 import oracle
+import test_oracle_decision as decision_pins
 import test_oracle_hash as hash_pins
 import test_oracle_loss as loss_pins
 
@@ -205,18 +206,18 @@ def m_encoder_scores_pads(real):
 
 # ---- mistakes in the fused head -------------------------------------------
 def m_linear_dw_dropped(real):
-    def f(plan, H, W, grad_scale, want_grads):
-        out = real(plan, H, W, grad_scale, want_grads)
-        return out[:5] + ((None if out[5] is None else np.zeros_like(out[5])),)
+    def f(plan, H, W, grad_scale, want_grads, keep_dz=False):
+        out = real(plan, H, W, grad_scale, want_grads, keep_dz)
+        return out[:5] + ((None if out[5] is None else np.zeros_like(out[5])),) + out[6:]
     return f
 
 
 def m_linear_dh_on_wrong_rows(real):
-    def f(plan, H, W, grad_scale, want_grads):
-        rows, lse, ce, row_loss, dH, dW = real(plan, H, W, grad_scale, want_grads)
+    def f(plan, H, W, grad_scale, want_grads, keep_dz=False):
+        rows, lse, ce, row_loss, dH, dW, dZ = real(plan, H, W, grad_scale, want_grads, keep_dz)
         if dH is not None and rows.size > 1:
             dH[rows] = dH[rows[::-1]]              # gradients land on the wrong rows
-        return rows, lse, ce, row_loss, dH, dW
+        return rows, lse, ce, row_loss, dH, dW, dZ
     return f
 
 
@@ -289,7 +290,46 @@ def test_a_planted_mistake_fails_a_pin(monkeypatch, target, mutation, modules):
 
 
 def test_control_every_pin_passes_on_the_unmutated_oracle():
-    assert _failing_pins(loss_pins, hash_pins) == []
+    assert _failing_pins(loss_pins, hash_pins, decision_pins) == []
+
+
+# ---- mistakes in the typed-decision losses ---------------------------------
+# Each case copies the source of one oracle function, makes one textual
+# change, compiles the copy with the oracle module's globals and puts it in
+# the function's place for the duration of the test.
+PY_MUTATIONS = [
+    ("decision_loss", "full_ce_over_the_answers_only",
+     "ce_full[i] = -(q * (c - lse)).sum()", "ce_full[i] = -(q * (c - lse_r)).sum()"),
+    ("decision_loss", "brier_on_the_full_softmax",
+     "brier[i] = ((r - y) ** 2).sum()", "brier[i] = ((P[a] - y) ** 2).sum()"),
+    ("decision_loss", "restricted_gradient_sign", "g[a] += Q * r - q", "g[a] -= Q * r - q"),
+    ("decision_loss", "full_gradient_without_onehot", "g[a] -= q\n", "g[a] -= 0.0 * q\n"),
+    ("decision_loss", "brier_gradient_without_its_mean",
+     "g[a] += brier_weight * 2.0 * r * (d - (r * d).sum())", "g[a] += brier_weight * 2.0 * r * d"),
+    ("decision_loss", "brier_weight_dropped",
+     "per_slot = (ce_res * use_res + ce_full * use_full + brier_weight * brier) * w",
+     "per_slot = (ce_res * use_res + ce_full * use_full + brier) * w"),
+    ("decision_loss", "sum_over_slots_not_mean", "w = 1.0 / n if n > 0 else 0.0", "w = 1.0"),
+    ("decision_targets", "smoothing_not_spread_over_the_answers",
+     "q = (1.0 - smoothing) * y + smoothing / K", "q = (1.0 - smoothing) * y + smoothing"),
+    ("decision_targets", "smoothing_applied_to_brier",
+     "y = val.copy()\n        q = (1.0 - smoothing) * y + smoothing / K",
+     "y = (1.0 - smoothing) * val + smoothing / K\n        q = y.copy()"),
+    ("decision_targets", "set_target_not_normalised", "y = val / val.sum()", "y = val.copy()"),
+]
+
+
+@pytest.mark.parametrize("fn,old,new", [m[::2][:1] + m[2:] for m in PY_MUTATIONS],
+                         ids=[m[1] for m in PY_MUTATIONS])
+def test_a_planted_mistake_in_the_decision_oracle_fails_a_pin(monkeypatch, fn, old, new):
+    import textwrap
+    src = textwrap.dedent(inspect.getsource(getattr(oracle, fn)))
+    assert src.count(old) == 1, old
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), f"<mutated {fn}>", "exec"), ns)
+    monkeypatch.setattr(oracle, fn, ns[fn])
+    failed = _failing_pins(decision_pins)
+    assert failed, f"no pin notices the change {old!r} -> {new!r} in oracle.{fn}"
 
 
 # ---- mistakes in the C part of the oracle ---------------------------------
