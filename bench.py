@@ -5,13 +5,20 @@ One step = one pass of the whole path over one batch of synthetic input:
 dlm_sample_t -> dlm_corrupt -> dlm_loss_fwd_bwd (fused forward + backward,
 bf16 dlogits for every row), all through the C ABI of libdlm.so.
 
-Default workload: the LLaDA-like absorbing-mask loss, B=1 L=4096 V=126464,
-aligned logits, clean-token logit +4, logits N(0, 3) bf16 (1.04 GB, larger
-than L2, so no flush between steps is needed).  Each timed step draws a new t
-(seed = 1000 + step), so the scored rows vary like in training.
+Default (the workload "suite"): the headline is the DiffusionGemma-like
+uniform-noise loss, B=4, prefix 512 + canvas 1024, V=262,144 -- canvas CE
+plus the encoder's causal CE, every row scored, 10.7 GB of logits read and
+gradients written per step, the largest of the logits workloads.  The same
+JSON line then carries, under "workloads", the LLaDA-like absorbing loss
+(B=1 L=4096 V=126,464), the Dream-like shifted loss (B=8 L=2048 V=152,064)
+and the fused-head loss on packed documents (T=16,384, D=4,096, V=126,464),
+each timed the same way with its own clocks, roofline and end-to-end leg.
+Inputs are larger than L2 in every workload, so no flush between steps is
+needed.  Each timed step draws a new t (seed = 1000 + step), so the scored
+rows vary like in training.
 
   python bench.py [--gpus N --steps K --warmup W] [--impl reference]
-  python bench.py --workload lin_t16384_d4096_v126464      # fused head, absorbing
+  python bench.py --workload abs_b1_l4096_v126464          # one workload alone
   python bench.py --workload lin_unif_b4_p512_c1024_d4096_v262144   # fused head, uniform
 
 Besides the device-timed value, rank 0 at N=1 reports the CPU oracle on a
@@ -43,11 +50,14 @@ sys.path.insert(0, ROOT)
 
 METRIC = "diffusion-loss fwd+bwd scored tokens/s; achieved HBM GB/s vs B200 peak"
 UNIT = "scored tokens/s"
-DEFAULT_WORKLOAD = "abs_b1_l4096_v126464"
+SUITE = "suite"
+SUITE_HEADLINE = "unif_b4_p512_c1024_v262144"
+SUITE_OTHERS = ("abs_b1_l4096_v126464", "shift_b8_l2048_v152064", "lin_t16384_d4096_v126464",
+                "dec_s128_k26_v126464")
+DEFAULT_WORKLOAD = SUITE
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 CE_SOURCE = os.path.join(ROOT, "diffusion_lm_loss_b200", "csrc", "dlm_ce.cu")
-CE_PROFILE = os.path.join(ROOT, "profiles", "ce_stream_abs_b1_l4096_v126464.md")
 ABSORBING, UNIFORM = 0, 1          # noise modes, as numbered in include/dlm.h
 
 
@@ -66,11 +76,12 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def ce_traffic_ratio():
-    """DRAM bytes / algorithmic bytes of the CE kernel from the committed ncu
-    summary, or None when the kernel source changed since the capture."""
+def ce_traffic_ratio(workload: str):
+    """DRAM bytes / algorithmic bytes of the CE kernel on `workload` from its
+    committed ncu summary (profiles/ce_stream_<workload>.md), or None when
+    there is none or the kernel source changed since the capture."""
     try:
-        txt = open(CE_PROFILE).read()
+        txt = open(os.path.join(ROOT, "profiles", f"ce_stream_{workload}.md")).read()
     except OSError:
         return None
     m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
@@ -85,31 +96,95 @@ def ce_traffic_ratio():
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
+    """SM clock, power and clock-event reasons sampled every few milliseconds
+    by a background thread through NVML while the timed steps run (a timed
+    region of a few tens of milliseconds still gets samples); falls back to
+    `nvidia-smi -lms 50` when NVML is unavailable."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4), ("hw_power_brake_slowdown", 0x80))
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index, device=None, period_s: float = 0.002):
         self.gpu = gpu_index
+        self.device = device
+        self.period = period_s
         self.proc = None
+        self.thread = None
+        self.samples = []
         self.t0 = self.t1 = None
+        self.nvml = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+
+        pynvml.nvmlInit()
+        if self.device is not None:
+            try:
+                uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+                return pynvml, pynvml.nvmlDeviceGetHandleByUUID("GPU-" + uuid)
+            except Exception:
+                pass
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu))
 
     def start(self):
+        import threading
+
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu=timestamp,{self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            nv, h = self._nvml_handle()
+            self.nvml = (nv, h)
+            self.sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
         except Exception:
-            self.proc = None
+            self.nvml = None
+        if self.nvml is None:
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu=timestamp,{self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", "50"],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                self.proc = None
+            return
+        self.stop_flag = threading.Event()
+
+        def loop():
+            nv, h = self.nvml
+            while not self.stop_flag.is_set():
+                try:
+                    t = time.perf_counter()
+                    sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                    rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    self.samples.append((t, sm, rs, pw))
+                except Exception:
+                    pass
+                time.sleep(self.period)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
 
     def mark_begin(self):
         self.t0 = datetime.datetime.now()
+        self.p0 = time.perf_counter()
 
     def mark_end(self):
         self.t1 = datetime.datetime.now()
+        self.p1 = time.perf_counter()
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            inside = [s for s in self.samples if self.p0 <= s[0] <= self.p1]
+            use = inside or self.samples[len(self.samples) // 2:len(self.samples) // 2 + 1]
+            if not use:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "source": "nvml"}
+            reasons = sorted({n for _, _, rs, _ in use for n, bit in self.REASONS if rs & bit})
+            return {"sm_mhz": statistics.median(s[1] for s in use), "sm_max_mhz": self.sm_max,
+                    "reasons": reasons, "power_w_max": max(s[3] for s in use), "samples": len(use),
+                    "samples_in_timed_region": len(inside), "source": "nvml, every 2 ms"}
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.15)
@@ -144,7 +219,7 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(use),
-                "samples_in_timed_region": len(inside)}
+                "samples_in_timed_region": len(inside), "source": "nvidia-smi, every 50 ms"}
 
 
 # ---------------------------------------------------------------------------
@@ -173,11 +248,16 @@ def algorithmic_ce_bytes(rows: int, scored: int, vocab: int) -> int:
 
 
 def run_ours(args):
+    """Our arm.  The default workload "suite" times the headline workload
+    (the DiffusionGemma-like uniform loss, the largest logits workload) and
+    then, each in the same way with its own clocks, roofline and end-to-end
+    leg, the LLaDA-like, the Dream-like and the fused-head workloads; rank 0
+    prints one JSON line, the headline at top level and the others under
+    "workloads"."""
     import torch
     import torch.distributed as dist
 
     import dlm_inputs as di
-    import diffusion_lm_loss_b200 as dlm
 
     rank, local_rank, world = env_rank()
     if args.gpus != world:
@@ -188,10 +268,48 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
+    keys = [SUITE_HEADLINE, *SUITE_OTHERS] if args.workload == SUITE else [args.workload]
+    recs = []
+    for i, key in enumerate(keys):
+        spec = di.WORKLOADS[key]
+        run = {"linear": run_linear, "decision": run_decision}.get(spec.kind, run_logits)
+        if i == 0 or world > 1:
+            recs.append(run(args, spec, dev, rank, world, headline=(i == 0)))
+        else:
+            # one GPU: a failing sub-record is recorded and the line still prints
+            try:
+                recs.append(run(args, spec, dev, rank, world, headline=False))
+            except Exception as ex:
+                recs.append({"config": {"workload": key}, "value": None,
+                             "error": f"{type(ex).__name__}: {ex}"[:300]})
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    res = recs[0]
+    if len(recs) > 1:
+        res["config"]["suite"] = ("headline: the largest logits workload; the other workloads of the suite "
+                                  "under \"workloads\", each timed the same way")
+        res["workloads"] = {r["config"]["workload"]: {k: v for k, v in r.items()
+                                                      if k not in ("metric", "higher_is_better", "scaling",
+                                                                   "vs_baseline", "data", "n_gpus")}
+                            for r in recs[1:]}
+    print(json.dumps(res), flush=True)
 
-    spec = di.WORKLOADS[args.workload]
-    if spec.kind == "linear":
-        return run_linear(args, spec, dev, rank, world)
+
+def run_logits(args, spec, dev, rank, world, headline=True):
+    """One logits workload: time draw, corruption, weighted CE forward +
+    backward through dlm_loss_fwd_bwd; returns the record of its JSON line."""
+    import torch
+    import torch.distributed as dist
+
+    import dlm_inputs as di
+    import diffusion_lm_loss_b200 as dlm
+
+    local_rank = dev.index
     case = di.make_case(spec, dev, seed=spec.data_seed + rank)
     V = spec.vocab
     mode, align = spec.mode, spec.align
@@ -237,7 +355,7 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
-    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else local_rank)
+    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else local_rank, device=dev)
     if rank == 0:
         clocks.start()
         time.sleep(0.3)
@@ -337,7 +455,7 @@ def run_ours(args):
         n_sc = scored / K if world == 1 else scored_all / world / K
         alg_bytes = 4.0 * V * n_sc + 20.0 * rows
     achieved = alg_bytes / (loss_ms / 1e3) / 1e9
-    ratio = ce_traffic_ratio()
+    ratio = ce_traffic_ratio(spec.key)
     roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm,
             # the profiled traffic ratio belongs to the default (zero-writing) call
@@ -349,13 +467,7 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(spec)
-
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return
+        cpu = cpu_baseline(spec) if headline else cpu_baseline(spec, budget_s=4.0, single_thread_s=0)
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -371,10 +483,10 @@ def run_ours(args):
         "roofline": roof, "cpu_baseline": cpu, "clocks": clk, "e2e": e2e,
         "gpu_launches": 5 * K,
     }
-    print(json.dumps(res), flush=True)
+    return res
 
 
-def run_linear(args, spec, dev, rank, world):
+def run_linear(args, spec, dev, rank, world, headline=True):
     """The fused lm_head workload: time draw, corruption, and the loss from
     hidden states and the head (dlm_linear_loss_fwd_bwd, dH and dW; uniform
     workloads: dlm_linear_loss_uniform_fwd_bwd, canvas and encoder hidden
@@ -420,7 +532,7 @@ def run_linear(args, spec, dev, rank, world):
     torch.cuda.synchronize()
     vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
     lr = int(os.environ.get("LOCAL_RANK", "0"))
-    clocks = ClockSampler(vis[lr] if lr < len(vis) else lr)
+    clocks = ClockSampler(vis[lr] if lr < len(vis) else lr, device=dev)
     if rank == 0:
         clocks.start()
         time.sleep(0.3)
@@ -486,15 +598,10 @@ def run_linear(args, spec, dev, rank, world):
                       "6*M*D*V; executed 8*M*D*V with the backward recompute)",
             "algorithmic_flops_per_call": flops, "launch_ms": call_ms,
             "frac_of_burst_peak": achieved / bf16, "peak_source": f"{kind} bf16 sustained (burst in frac_of_burst_peak)"}
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank != 0:
-        return
     cpu = None
-    if world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         try:
-            cpu = cpu_baseline(spec)
+            cpu = cpu_baseline(spec) if headline else cpu_baseline(spec, budget_s=4.0, single_thread_s=0)
         except Exception as e:      # the GPU figures above stand without it
             cpu = {"value": None, "kind": "oracle", "error": f"{type(e).__name__}: {e}"[:300]}
     res = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
@@ -508,7 +615,126 @@ def run_linear(args, spec, dev, rank, world):
            # per step: time draw, corruption, plan, gather, forward GEMM, lse,
            # dZ + dH + dW per 16,384-column vocabulary chunk, scatter, reduce
            "gpu_launches": K * (6 + 3 * ((V + 16383) // 16384) + 2)}
-    print(json.dumps(res), flush=True)
+    return res
+
+
+def run_decision(args, spec, dev, rank, world, headline=True):
+    """The typed-decision workload: dlm_decision_loss_fwd_bwd on the logits
+    rows of the label slots.  Its inputs (n_slots x V bf16) fit in L2, so a
+    256 MB buffer is written between timed calls (outside each call's
+    events) and the call is timed alone."""
+    import torch
+
+    import dlm_inputs as di
+    import diffusion_lm_loss_b200 as dlm
+
+    case = di.make_case(spec, dev, seed=spec.data_seed + rank)
+    e = case.extra
+    n, V = spec.n_units, spec.vocab
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    out = None
+
+    def call(logits, ev=None):
+        nonlocal out
+        if ev is not None:
+            ev[0].record()
+        out = dlm.decision_loss_fwd_bwd(logits, V, e["cand_off"], e["cand_ids"], e["kind"], e["val"],
+                                        brier_weight=0.1, out=out)
+        if ev is not None:
+            ev[1].record()
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        flush.fill_(1)
+        call(case.logits)
+    torch.cuda.synchronize()
+    vis = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    lr = int(os.environ.get("LOCAL_RANK", "0"))
+    clocks = ClockSampler(vis[lr] if lr < len(vis) else lr, device=dev)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks.mark_begin()
+    for i in range(K):
+        flush.fill_(i & 0xff)
+        call(case.logits, evs[i])
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    if world > 1:
+        torch.distributed.barrier()
+    call_ms = sum(a.elapsed_time(b) for a, b in evs) / K
+    clk = clocks.stop() if rank == 0 else None
+    ms, call_ms, slots_all = reduce_over_ranks(call_ms * K, call_ms, float(n * K), dev)
+    value = slots_all / (ms / 1e3)
+    e2e = None
+    if not args.no_e2e:
+        Ke = max(1, min(K, args.e2e_steps))
+        dev_in = [case.logits, e["cand_off"], e["cand_ids"], e["kind"], e["val"]]
+        host_in = [t.cpu().pin_memory() for t in dev_in]
+        h_loss = torch.empty(Ke, dtype=torch.float32).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_in)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def e2e_step(i):
+            for d, h in zip(dev_in, host_in):
+                d.copy_(h, non_blocking=True)
+            call(case.logits)
+            h_loss[i:i + 1].copy_(out.loss, non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        s0.record()
+        for i in range(Ke):
+            e2e_step(i)
+        s1.record()
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([s0.elapsed_time(s1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(e_ms, op=torch.distributed.ReduceOp.MAX)
+        e2e = {"value": n * world * Ke / (float(e_ms[0]) / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": 4, "steps": Ke, "ms_per_step": float(e_ms[0]) / Ke}
+    hbm, _, peak_kind = peaks()
+    alg = 4.0 * n * V + 8.0 * n
+    roof = {"bound": "hbm", "achieved": alg / (call_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
+            "frac": alg / (call_ms / 1e3) / 1e9 / hbm, "traffic": None,
+            "kernel": "k_dec_partial + k_dec_grad + k_dec_reduce (timed as the whole dlm_decision_loss_fwd_bwd call)",
+            "algorithmic_bytes_per_launch": alg, "launch_ms": call_ms,
+            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = _decision_cpu_baseline(spec, case)
+    return {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": spec.key, "description": spec.description, "label_slots": n, "vocab": V,
+                       "parallelism": f"replicas{world}", "label_softmax": "both", "brier_weight": 0.1,
+                       "l2": "inputs smaller than L2: a 256 MB buffer is written before each call, outside "
+                             "its events; a step is the call alone",
+                       "unit_note": "scored tokens = label slots"},
+            "roofline": roof, "cpu_baseline": cpu, "clocks": clk, "e2e": e2e, "gpu_launches": 3 * K}
+
+
+def _decision_cpu_baseline(spec, case, budget_s=4.0):
+    """The decision oracle on the whole workload, repeated for about
+    budget_s seconds."""
+    import dlm_inputs as di
+    import oracle
+
+    e = {k: v.cpu().numpy() for k, v in case.extra.items()}
+    x = di.bf16_bits(case.logits)
+    t0 = time.perf_counter()
+    steps = 0
+    while steps < 1 or time.perf_counter() - t0 < budget_s:
+        oracle.decision_loss(x, spec.vocab, None, e["cand_off"], e["cand_ids"], e["kind"], e["val"])
+        steps += 1
+    dt = time.perf_counter() - t0
+    return {"value": spec.n_units * steps / dt, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"{steps} runs of the whole workload ({spec.n_units} label slots, V = {spec.vocab}; "
+                      f"the three terms and the double-precision gradient of every logit): {dt:.1f} s"}
 
 
 def _linear_e2e(args, spec, case, lay, enc, align, per_step, out):
@@ -760,7 +986,7 @@ def run_reference(args):
         return
     import dlm_inputs as di
 
-    spec = di.WORKLOADS[args.workload]
+    spec = di.WORKLOADS[SUITE_HEADLINE if args.workload == SUITE else args.workload]
     need = oracle_host_bytes(spec, 1024)
     if need > 0.6 * __import__("psutil").virtual_memory().available:
         print(json.dumps({"impl": "reference",
@@ -797,8 +1023,8 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -6,13 +6,28 @@ Tolerances (the floating-point bar of the path):
   * bf16 gradients: |gpu - exact| <= max(2e-3, one bf16 ulp of the exact
     value) -- 2e-3 absolute, except where a gradient is so large (w = 1/(pN)
     with small p and small N) that bf16 itself cannot hold 2e-3 -- and the
-    GPU value is at most one ulp away from the exact value rounded to bf16.
+    GPU value is at most one ulp away from the exact value rounded to bf16
+    (values below 2^-126, the smallest normal, count as zero in that last
+    check: the kernels' exponentials flush subnormal results to zero, and
+    2^-126 is far inside the 2e-3 absolute bar);
+  * fused-head gradients dH = dZ W and dW = dZ^T H_M, element by element:
+    each is a bf16 rounding of an fp32 sum of products a_k b_k in which a_k
+    (dZ) was itself rounded to bf16, a relative error of at most u = 2^-8
+    per product.  The bar is
+        |gpu - exact| <= ulp(max(|gpu|, |exact|)) + 8 u s,
+        s = sqrt(sum_k (a_k b_k)^2) over that element's products:
+    the first term is the output's own rounding; u s bounds the standard
+    deviation the sum can get from independent roundings of the a_k, and
+    8 u s also covers their worst case u sum_k |a_k b_k| whenever at most 64
+    products matter.  The fp32 accumulation (relative ~1e-6) is far below it.
 """
 import numpy as np
 import torch
 
 LOSS_RTOL = 1e-5
 GRAD_ATOL = 2e-3
+BF16_U = 2.0 ** -8          # unit roundoff of bf16 (8 significant bits)
+SUM_SIGMAS = 8.0
 
 
 def bf16_ulp(x: np.ndarray) -> np.ndarray:
@@ -60,3 +75,37 @@ def assert_units_close(gpu: np.ndarray, exact: np.ndarray, total: float):
     err = np.abs(gpu - exact)
     tol = LOSS_RTOL * np.abs(exact) + 1e-7 * abs(total)
     assert (err <= tol).all(), f"unit_loss: max err {err.max():.3e}"
+
+
+def product_rms_scale(a: np.ndarray, b: np.ndarray, transpose_a: bool = False,
+                      chunk: int = 16384) -> np.ndarray:
+    """s = sqrt((a*a) @ (b*b)) (or sqrt((a*a)^T @ (b*b))) in float32: for
+    C = a @ b the root of the sum of squared products of each element of C.
+    Streams the shared dimension in chunks to bound host memory."""
+    n = a.shape[0] if transpose_a else a.shape[1]
+    out = None
+    for k0 in range(0, n, chunk):
+        ak = (a[k0:k0 + chunk] if transpose_a else a[:, k0:k0 + chunk]).astype(np.float32)
+        ak *= ak
+        bk = b[k0:k0 + chunk].astype(np.float32)
+        bk *= bk
+        part = (ak.T @ bk) if transpose_a else (ak @ bk)
+        out = part if out is None else out + part
+    return np.sqrt(out)
+
+
+def assert_bf16_sum_close(gpu: np.ndarray, exact: np.ndarray, scale: np.ndarray, what: str):
+    """Element-wise bar for a bf16 sum of products whose one operand was
+    rounded to bf16 (see the module docstring); `scale` = product_rms_scale
+    of that sum.  Also returns the relative Frobenius error, for reports."""
+    gpu = np.asarray(gpu, np.float64)
+    exact = np.asarray(exact, np.float64)
+    assert gpu.shape == exact.shape == scale.shape, (gpu.shape, exact.shape, scale.shape)
+    err = np.abs(gpu - exact)
+    tol = bf16_ulp(np.maximum(np.abs(gpu), np.abs(exact))) + SUM_SIGMAS * BF16_U * scale
+    bad = err > tol
+    if bad.any():
+        i = np.unravel_index(int(np.argmax(err - tol)), err.shape)
+        raise AssertionError(f"{what}: {int(bad.sum())} of {err.size} elements out of tolerance; worst at {i}: "
+                             f"gpu {gpu[i]!r} exact {exact[i]!r} tol {tol[i]:.3e}")
+    return float(np.linalg.norm(gpu - exact) / max(np.linalg.norm(exact), 1e-300))
