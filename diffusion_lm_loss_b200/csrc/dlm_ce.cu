@@ -496,6 +496,9 @@ __device__ __forceinline__ void row_ptrs(const CeParams& P, int q, const uint16_
 // The producer warp also zero-fills unscored rows (taken by ticket too) with
 // bulk shared->global copies from a zeroed shared block, interleaved with
 // the scored rows so the zero stream overlaps the consumers' work.
+#ifndef DLM_CE_RESIDENT
+#define DLM_CE_RESIDENT -1          // chunks held in the ring between the passes (-1: stages - 2)
+#endif
 constexpr int kChunk = 8192;        // bf16 elements per ring stage (16 KB)
 constexpr int kZeroBytes = 4096;    // zero block the producer copies over unscored rows
 
@@ -514,6 +517,12 @@ struct StreamShape {
     static constexpr int kChunkE = WARPS >= 24 ? WARPS * 512 : kChunk;
     static constexpr int kVec = kChunkE / 8 / kConsumers;   // 16-byte vectors per thread per chunk
     static_assert(kVec * 8 * kConsumers == kChunkE, "chunk split");
+    // Chunks of a scored row that stay in the ring between the two passes:
+    // the last kResident chunks of pass 1 are not released, pass 2 uses
+    // them first, and only the rest of the row is read again (from L2).  Two
+    // stages stay free for the producer to run ahead meanwhile.
+    static constexpr int kResident = DLM_CE_RESIDENT < 0 ? STAGES - 2
+                                   : (DLM_CE_RESIDENT < STAGES ? DLM_CE_RESIDENT : STAGES);
 };
 
 constexpr int kRowQ = 16;          // row entries in flight between producer and consumers (> stages / 2)
@@ -546,6 +555,7 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
     const int V = P.vocab;
     constexpr int kChunkE = Sh::kChunkE;
     const int nch = (V + kChunkE - 1) / kChunkE;
+    const int res = Sh::kResident < nch ? Sh::kResident : nch;   // chunks kept in the ring between the passes
     volatile int* abort = &S.abort;
 
     for (int i = tid; i < kZeroBytes / 16; i += kStreamThreads) S.zero[i] = make_uint4(0, 0, 0, 0);
@@ -611,7 +621,9 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
                 uint16_t* dr;
                 row_ptrs(P, e.x, xr, dr);
                 for (int pass = 0; pass < 2 && ok; ++pass) {
-                    for (int c = 0; c < nch; ++c, ++seq) {
+                    // pass 2 reads again only the chunks the ring did not keep
+                    const int nc = pass == 0 ? nch : nch - res;
+                    for (int c = 0; c < nc; ++c, ++seq) {
                         const int st = seq % kStages;
                         if (!mbar_wait_or_abort(smem_addr(&S.empty[st]), ((seq / kStages) & 1) ^ 1, P.status,
                                                 abort)) { ok = false; break; }
@@ -619,7 +631,9 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
                         const uint32_t bytes = uint32_t(min(kChunkE, V - e0)) * 2u;
                         const uint32_t fb = smem_addr(&S.full[st]);
                         mbar_arrive_expect_tx(fb, bytes);
-                        bulk_g2s_hint(smem_addr(S.ring[st]), xr + e0, bytes, fb, pass == 0 ? pol_keep : pol_drop);
+                        // only the chunks read again need to stay in L2
+                        const bool again = pass == 0 && c < nch - res;
+                        bulk_g2s_hint(smem_addr(S.ring[st]), xr + e0, bytes, fb, again ? pol_keep : pol_drop);
                     }
                 }
                 ++k;
@@ -662,6 +676,7 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
         named_barrier_sync(2, kConsumers);
         const int4 e = S.cur[k & 1];
         if (e.x < 0) break;
+        const int seq0 = seq;            // ring sequence number of the row's first chunk
         const int q = e.x, y = e.y;
         const float w = __int_as_float(e.z);
         const int par = k & 1;
@@ -696,7 +711,8 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&S.empty[st]));
+            // the row's last `res` chunks stay in the ring for pass 2
+            if (lane == 0 && c < nch - res) mbar_arrive(smem_addr(&S.empty[st]));
             if (cm > m) {
                 s = (m == -INFINITY) ? 0.f : s * ex2((m - cm) * kLog2e);
                 m = cm;
@@ -744,10 +760,19 @@ __global__ void __launch_bounds__(StreamShape<WARPS, STAGES>::kThreads, CTAS) k_
         const uint64_t l2e = f2pack(kLog2e, kLog2e);
         const uint64_t nlb = f2pack(-lb, -lb);
 
-        // pass 2: gradient
-        for (int c = 0; c < nch; ++c, ++seq) {
-            const int st = seq % kStages;
-            mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort);
+        // pass 2: gradient -- first the chunks still in the ring (the row's
+        // tail, no wait), then the head, delivered again by the producer
+        for (int i = 0; i < nch; ++i) {
+            const bool kept = i < res;
+            const int c = kept ? nch - res + i : i - res;
+            int st;
+            if (kept) {
+                st = (seq0 + c) % kStages;
+            } else {
+                st = seq % kStages;
+                mbar_wait_or_abort(smem_addr(&S.full[st]), (seq / kStages) & 1, P.status, abort);
+                ++seq;
+            }
             const int e0 = c * kChunkE;
             uint4 outv[kVecPerThread];
             #pragma unroll
