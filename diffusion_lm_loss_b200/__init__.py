@@ -11,10 +11,16 @@ Two layers:
     ``dlm_loss_fwd_bwd``, ``dlm_linear_loss_fwd_bwd``, ...);
   * tensor helpers with the same names minus the prefix (``sample_t``,
     ``corrupt``, ``loss_fwd_bwd``, ``linear_loss_fwd_bwd``,
-    ``linear_loss_uniform_fwd_bwd``) that check every tensor argument's
+    ``linear_loss_uniform_fwd_bwd``, ``decision_loss_fwd_bwd``) that check every tensor argument's
     dtype, size against the layout and device, allocate outputs and
     workspace with torch on the current device and call the ABI on the
-    current torch stream.
+    current torch stream;
+  * ``torch.autograd.Function`` wrappers of the four losses
+    (``diffusion_loss``, ``linear_diffusion_loss``,
+    ``linear_uniform_loss``, ``decision_loss``): the forward runs the fused
+    forward + backward call and keeps its gradients; the backward hands them
+    over, multiplied by the upstream gradient in the library
+    (``dlm_scale_bf16``, which does nothing when that gradient is 1).
 """
 from __future__ import annotations
 
@@ -36,6 +42,12 @@ REDUCE_TOKEN_MEAN, REDUCE_EXAMPLE_MEAN = 0, 1
 DEV_BAD_TOKEN_ID = 0x1
 DEV_BAD_LAYOUT = 0x2
 DEV_WAIT_TIMEOUT = 0x4
+DEV_BAD_LABEL = 0x8
+
+LABEL_HARD, LABEL_DIST, LABEL_SET = 0, 1, 2
+LABEL_SOFTMAX_RESTRICTED, LABEL_SOFTMAX_FULL, LABEL_SOFTMAX_BOTH = 1, 2, 3
+DECISION_MAX_ANSWERS = 128
+DECISION_MAX_SLOTS = 65535
 
 STATUS = {0: "DLM_OK", 1: "DLM_ERR_INVALID_ARGUMENT", 2: "DLM_ERR_UNSUPPORTED",
           3: "DLM_ERR_WORKSPACE_TOO_SMALL", 4: "DLM_ERR_CUDA"}
@@ -45,7 +57,8 @@ EXPORTS = ("dlm_status_string", "dlm_last_cuda_error", "dlm_version", "dlm_sampl
            "dlm_loss_workspace_size", "dlm_loss_fwd_bwd", "dlm_loss_fwd_bwd_ex", "dlm_loss_fwd_bwd_static",
            "dlm_linear_loss_workspace_size",
            "dlm_linear_loss_fwd_bwd", "dlm_linear_loss_fwd_bwd_ex", "dlm_linear_loss_uniform_workspace_size",
-           "dlm_linear_loss_uniform_fwd_bwd", "dlm_get_device_status", "dlm_selftest_bounded_wait",
+           "dlm_linear_loss_uniform_fwd_bwd", "dlm_decision_workspace_size", "dlm_decision_loss_fwd_bwd",
+           "dlm_scale_bf16", "dlm_get_device_status", "dlm_selftest_bounded_wait",
            "dlm_test_skip_device_check")
 
 
@@ -150,6 +163,13 @@ def lib():
     L.dlm_linear_loss_uniform_fwd_bwd.restype = ctypes.c_int
     L.dlm_linear_loss_uniform_fwd_bwd.argtypes = [lp, vp, lp, vp, vp, vp, i32, i32, vp, i32, f32, f32,
                                                   vp, vp, vp, vp, vp, vp, sz, vp]
+    L.dlm_decision_workspace_size.restype = sz
+    L.dlm_decision_workspace_size.argtypes = [i32, i32]
+    L.dlm_decision_loss_fwd_bwd.restype = ctypes.c_int
+    L.dlm_decision_loss_fwd_bwd.argtypes = [i32, vp, i64, i32, vp, vp, vp, vp, vp, i32, f32, f32, f32, vp, vp,
+                                            vp, i64, vp, sz, vp]
+    L.dlm_scale_bf16.restype = ctypes.c_int
+    L.dlm_scale_bf16.argtypes = [vp, i64, i64, i64, vp, vp]
     L.dlm_test_skip_device_check.restype = ctypes.c_int
     L.dlm_test_skip_device_check.argtypes = [i32]
     L.dlm_selftest_bounded_wait.restype = ctypes.c_int
@@ -481,9 +501,218 @@ def linear_loss_uniform_fwd_bwd(layout: Layout, hidden: torch.Tensor, weight: to
     return out
 
 
+@dataclass
+class DecisionOut:
+    loss: torch.Tensor            # float32 [1]
+    slot_loss: torch.Tensor       # float32 [n_slots]: each slot's share of the loss
+    dlogits: torch.Tensor         # bf16 [n_slots, vocab]: row i = slot i
+    workspace: torch.Tensor       # uint8; holds the device status word
+
+    def device_status(self) -> int:
+        return device_status(self.workspace)
+
+
+def decision_workspace_size(n_slots: int, vocab: int) -> int:
+    return int(lib().dlm_decision_workspace_size(n_slots, vocab))
+
+
+def decision_loss_fwd_bwd(logits: torch.Tensor, vocab: int, cand_off: torch.Tensor, cand_ids: torch.Tensor,
+                          label_kind: torch.Tensor, label_val: torch.Tensor,
+                          slot_rows: Optional[torch.Tensor] = None,
+                          label_softmax: int = LABEL_SOFTMAX_BOTH, brier_weight: float = 0.1,
+                          hard_label_smoothing: float = 0.0, grad_scale: float = 1.0,
+                          out: Optional[DecisionOut] = None) -> DecisionOut:
+    """Typed-decision losses at label slots (see dlm_decision_loss_fwd_bwd).
+    logits: bf16 [rows, ld]; slot i reads row slot_rows[i] (int64), or row i
+    when slot_rows is None.  cand_off int32 [n_slots + 1]; cand_ids int32 and
+    label_val float32 [cand_off[-1]] (the offsets are on the device: the
+    caller keeps them within these arrays); label_kind int32 [n_slots]."""
+    n = int(cand_off.numel()) - 1
+    if n < 0:
+        raise ValueError("cand_off: needs n_slots + 1 entries")
+    _check(cand_off, torch.int32, "cand_off", min_numel=n + 1)
+    _check(label_kind, torch.int32, "label_kind", min_numel=n)
+    _check(cand_ids, torch.int32, "cand_ids", min_numel=0)
+    _check(label_val, torch.float32, "label_val", min_numel=cand_ids.numel())
+    rows_needed = n
+    if slot_rows is not None:
+        _check(slot_rows, torch.int64, "slot_rows", min_numel=n)
+        rows_needed = 1
+    _check(logits, torch.bfloat16, "logits", min_rows=rows_needed if n > 0 else 0, min_cols=vocab)
+    if out is not None:
+        _check(out.loss, torch.float32, "out.loss", min_numel=1)
+        _check(out.slot_loss, torch.float32, "out.slot_loss", min_numel=n)
+        _check(out.dlogits, torch.bfloat16, "out.dlogits", min_rows=n, min_cols=vocab)
+        _check(out.workspace, torch.uint8, "out.workspace", min_numel=0)
+    o = out if out is not None else DecisionOut(None, None, None, None)
+    _on_cuda(logits=logits, cand_off=cand_off, cand_ids=cand_ids, label_kind=label_kind, label_val=label_val,
+             slot_rows=slot_rows, loss=o.loss, slot_loss=o.slot_loss, dlogits=o.dlogits, workspace=o.workspace)
+    dev = logits.device
+    if out is None:
+        out = DecisionOut(torch.empty(1, dtype=torch.float32, device=dev),
+                          torch.empty(max(n, 1), dtype=torch.float32, device=dev),
+                          torch.empty((n, vocab), dtype=torch.bfloat16, device=dev),
+                          _aligned_workspace(decision_workspace_size(n, vocab), dev, 256))
+    _ok(lib().dlm_decision_loss_fwd_bwd(
+        n, _ptr(logits), logits.stride(0), vocab, _ptr(slot_rows), _ptr(cand_off), _ptr(cand_ids),
+        _ptr(label_kind), _ptr(label_val), label_softmax, brier_weight, hard_label_smoothing, grad_scale,
+        _ptr(out.loss), _ptr(out.slot_loss), _ptr(out.dlogits), out.dlogits.stride(0), _ptr(out.workspace),
+        out.workspace.numel(), _stream()), "dlm_decision_loss_fwd_bwd")
+    return out
+
+
 def device_status(workspace: torch.Tensor) -> int:
     """Device status word of a loss workspace (synchronises the stream)."""
     v = ctypes.c_uint32(0)
     _ok(lib().dlm_get_device_status(_ptr(workspace), ctypes.byref(v), _stream()),
         "dlm_get_device_status")
     return int(v.value)
+
+
+# --------------------------------------------------------------------------
+# autograd wrappers
+# --------------------------------------------------------------------------
+def scale_bf16_(x: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
+    """x *= scale in place on the device (see dlm_scale_bf16); scale is a
+    one-element float32 device tensor.  x: bf16, 1-D or 2-D with unit column
+    stride."""
+    _check(scale, torch.float32, "scale", min_numel=1)
+    _check(x, torch.bfloat16, "x")
+    x2 = x.view(1, -1) if x.dim() == 1 else x
+    if x2.dim() != 2 or (x2.shape[1] > 1 and x2.stride(1) != 1):
+        raise ValueError("x: 1-D contiguous or 2-D with unit column stride")
+    _on_cuda(x=x, scale=scale)
+    _ok(lib().dlm_scale_bf16(_ptr(x2), x2.shape[0], x2.shape[1], x2.stride(0) if x2.shape[0] > 1 else x2.shape[1],
+                             _ptr(scale), _stream()), "dlm_scale_bf16")
+    return x
+
+
+def _upstream(grad: torch.Tensor) -> torch.Tensor:
+    return grad.detach().reshape(1).to(torch.float32).contiguous()
+
+
+class _DiffusionLossFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, logits, enc_logits, layout, vocab, clean_ids, corrupted, p, mode, align, enc_layout,
+                enc_ids, enc_ar_weight, options):
+        out = loss_fwd_bwd(layout, logits, vocab, clean_ids, corrupted, p, mode, align, enc_layout=enc_layout,
+                           enc_logits=enc_logits, enc_ids=enc_ids, enc_ar_weight=enc_ar_weight, options=options)
+        ctx.grads = (out.dlogits, out.enc_dlogits)
+        ctx.out = out
+        return out.loss.view(())
+
+    @staticmethod
+    def backward(ctx, grad):
+        g = _upstream(grad)
+        d, de = ctx.grads
+        ctx.grads = None
+        scale_bf16_(d, g)
+        if de is not None:
+            scale_bf16_(de, g)
+        return (d, de) + (None,) * 11
+
+
+def diffusion_loss(layout: Layout, logits: torch.Tensor, vocab: int, clean_ids: torch.Tensor,
+                   corrupted: Optional[torch.Tensor], p: Optional[torch.Tensor], mode: int = ABSORBING,
+                   align: int = ALIGNED, enc_layout: Optional[Layout] = None,
+                   enc_logits: Optional[torch.Tensor] = None, enc_ids: Optional[torch.Tensor] = None,
+                   enc_ar_weight: float = 1.0, options: Optional[LossOptions] = None) -> torch.Tensor:
+    """The loss of dlm_loss_fwd_bwd as a differentiable scalar of `logits`
+    (and `enc_logits`).  The forward computes the gradient too and keeps it
+    (memory of one logits tensor) until backward hands it to autograd.
+    Logits are [rows, vocab] here (the gradient has their shape)."""
+    for t, name in ((logits, "logits"), (enc_logits, "enc_logits")):
+        if t is not None and (t.dim() != 2 or t.shape[1] != vocab):
+            raise ValueError(f"{name}: [rows, vocab]")
+    return _DiffusionLossFn.apply(logits, enc_logits, layout, vocab, clean_ids, corrupted, p, mode, align,
+                                  enc_layout, enc_ids, enc_ar_weight, options)
+
+
+class _LinearLossFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, hidden, weight, layout, clean_ids, corrupted, p, align):
+        out = linear_loss_fwd_bwd(layout, hidden, weight, clean_ids, corrupted, p,
+                                  want_d_weight=weight.requires_grad, align=align)
+        ctx.grads = (out.d_hidden, out.d_weight)
+        ctx.out = out
+        return out.loss.view(())
+
+    @staticmethod
+    def backward(ctx, grad):
+        g = _upstream(grad)
+        dh, dw = ctx.grads
+        ctx.grads = None
+        scale_bf16_(dh, g)
+        if dw is not None:
+            scale_bf16_(dw, g)
+        return (dh, dw) + (None,) * 5
+
+
+def linear_diffusion_loss(layout: Layout, hidden: torch.Tensor, weight: torch.Tensor, clean_ids: torch.Tensor,
+                          corrupted: torch.Tensor, p: torch.Tensor, align: int = ALIGNED) -> torch.Tensor:
+    """The loss of dlm_linear_loss_fwd_bwd as a differentiable scalar of
+    `hidden` and `weight` (dW is skipped when weight does not require a
+    gradient, e.g. a frozen head)."""
+    return _LinearLossFn.apply(hidden, weight, layout, clean_ids, corrupted, p, align)
+
+
+class _LinearUniformLossFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, hidden, enc_hidden, weight, layout, clean_ids, enc_layout, enc_ids, enc_ar_weight, align):
+        out = linear_loss_uniform_fwd_bwd(layout, hidden, weight, clean_ids, enc_layout, enc_hidden, enc_ids,
+                                          enc_ar_weight=enc_ar_weight, align=align,
+                                          want_d_weight=weight.requires_grad)
+        ctx.grads = (out.d_hidden, out.d_enc_hidden, out.d_weight)
+        ctx.out = out
+        return out.loss.view(())
+
+    @staticmethod
+    def backward(ctx, grad):
+        g = _upstream(grad)
+        grads = ctx.grads
+        ctx.grads = None
+        for t in grads:
+            if t is not None:
+                scale_bf16_(t, g)
+        return grads + (None,) * 6
+
+
+def linear_uniform_loss(layout: Layout, hidden: torch.Tensor, weight: torch.Tensor, clean_ids: torch.Tensor,
+                        enc_layout: Optional[Layout] = None, enc_hidden: Optional[torch.Tensor] = None,
+                        enc_ids: Optional[torch.Tensor] = None, enc_ar_weight: float = 1.0,
+                        align: int = ALIGNED) -> torch.Tensor:
+    """The loss of dlm_linear_loss_uniform_fwd_bwd as a differentiable
+    scalar of `hidden`, `enc_hidden` and `weight`."""
+    return _LinearUniformLossFn.apply(hidden, enc_hidden, weight, layout, clean_ids, enc_layout, enc_ids,
+                                      enc_ar_weight, align)
+
+
+class _DecisionLossFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, logits, vocab, cand_off, cand_ids, label_kind, label_val, label_softmax, brier_weight,
+                hard_label_smoothing):
+        out = decision_loss_fwd_bwd(logits, vocab, cand_off, cand_ids, label_kind, label_val,
+                                    label_softmax=label_softmax, brier_weight=brier_weight,
+                                    hard_label_smoothing=hard_label_smoothing)
+        ctx.grads = out.dlogits
+        ctx.out = out
+        return out.loss.view(())
+
+    @staticmethod
+    def backward(ctx, grad):
+        d = ctx.grads
+        ctx.grads = None
+        scale_bf16_(d, _upstream(grad))
+        return (d,) + (None,) * 8
+
+
+def decision_loss(logits: torch.Tensor, vocab: int, cand_off: torch.Tensor, cand_ids: torch.Tensor,
+                  label_kind: torch.Tensor, label_val: torch.Tensor, label_softmax: int = LABEL_SOFTMAX_BOTH,
+                  brier_weight: float = 0.1, hard_label_smoothing: float = 0.0) -> torch.Tensor:
+    """The typed-decision loss of dlm_decision_loss_fwd_bwd as a
+    differentiable scalar of `logits` ([n_slots, vocab], one row per label
+    slot)."""
+    if logits.dim() != 2 or tuple(logits.shape) != (cand_off.numel() - 1, vocab):
+        raise ValueError("logits: [n_slots, vocab], one row per label slot")
+    return _DecisionLossFn.apply(logits, vocab, cand_off, cand_ids, label_kind, label_val, label_softmax,
+                                 brier_weight, hard_label_smoothing)

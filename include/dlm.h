@@ -17,6 +17,9 @@
  *                            (dlm_linear_loss_fwd_bwd_ex: aligned or shifted
  *                            targets; dlm_linear_loss_uniform_fwd_bwd: the
  *                            uniform-noise loss with its encoder term)
+ *   dlm_decision_loss_fwd_bwd  typed-decision losses at label slots
+ *                            (candidate-restricted CE, full-vocabulary CE,
+ *                            Brier), forward + backward
  *
  * The method (page title, section):
  *   "LLaDA-8B-MDLM-LoRA", Training table, row "Objective": t ~ U(0,1) per
@@ -87,6 +90,7 @@ enum { DLM_ALIGNED = 0, DLM_SHIFTED = 1 };
 #define DLM_DEV_BAD_TOKEN_ID   0x1u  /* a scored target id outside [0, vocab)      */
 #define DLM_DEV_BAD_LAYOUT     0x2u  /* cu_seqlens not 0..n_tokens non-decreasing  */
 #define DLM_DEV_WAIT_TIMEOUT   0x4u  /* a bounded on-chip wait gave up             */
+#define DLM_DEV_BAD_LABEL      0x8u  /* a malformed typed-decision label           */
 
 /* Opaque CUDA stream (ABI-compatible with cudaStream_t / CUstream). */
 typedef struct CUstream_st *dlm_stream_t;
@@ -408,6 +412,92 @@ DLM_API dlm_status_t dlm_test_skip_device_check(int32_t enabled);
  * ---------------------------------------------------------------------- */
 DLM_API dlm_status_t dlm_selftest_bounded_wait(uint64_t limit_ns, uint32_t *dev_status,
                                                dlm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * dlm_decision_loss_fwd_bwd -- typed-decision losses at label slots,
+ * forward + backward ("Native diffusion language-model training",
+ * Typed-decision training: candidate-restricted CE, full-vocabulary CE and a
+ * 0.1 Brier term; Labels: hard / dist / set labels, labels.label_softmax,
+ * hard_label_smoothing; Adapters, merging and inference: the restricted-label
+ * and Brier terms are computed over the allowed answers).
+ *
+ * A label slot is the canvas position of one question's answer; its logits
+ * row z covers the whole vocabulary, and its question has K (1..128)
+ * distinct answer tokens a_0..a_{K-1} in canonical order.  With r = softmax
+ * of the K candidate logits, P = softmax over the vocabulary, q the CE
+ * target and y the Brier target over the K answers:
+ *   CE_res  = -sum_k q_k log r_k             (label_softmax RESTRICTED, BOTH)
+ *   CE_full = -sum_k q_k log P(a_k)          (label_softmax FULL, BOTH)
+ *   Brier   = sum_k (r_k - y_k)^2, times brier_weight (0.1 on the page)
+ *   loss    = (1 / n_slots) * sum over slots of its terms
+ * Targets by label kind (label_kind[i]; label_val holds one float per
+ * answer, at cand_off[i] .. cand_off[i+1]-1):
+ *   DLM_LABEL_HARD: val = 1 at the gold answer, 0 elsewhere.  y = val,
+ *       q = (1 - hard_label_smoothing) val + hard_label_smoothing / K.
+ *   DLM_LABEL_DIST: val = the probabilities (finite, >= 0).  q = y = val.
+ *   DLM_LABEL_SET:  val = 1 for each allowed answer, 0 elsewhere (at least
+ *       one 1).  q = y = val / (number of allowed answers).
+ * Arguments (device pointers unless stated):
+ *   logits [rows, ld] bf16; slot_rows [n_slots] int64: the logits row of
+ *       each slot, or NULL for row i = slot i (logits computed at the label
+ *       slots only).  ld >= vocab.
+ *   cand_off [n_slots + 1] int32 (offsets into cand_ids and label_val,
+ *       non-decreasing from 0), cand_ids int32 answer token ids,
+ *       label_kind [n_slots] int32, label_val float.
+ *   grad_scale g: the gradient written is g * d loss / d z.
+ *   loss [1] float (written); slot_loss [n_slots] float: each slot's
+ *       contribution (its terms / n_slots; sums to loss), or NULL.
+ *   dlogits [n_slots, ld_out] bf16 (row i = slot i; columns 0..vocab-1
+ *       written, the rest untouched); ld_out >= vocab.
+ *   workspace: at least dlm_decision_workspace_size(n_slots, vocab) bytes,
+ *       256-byte aligned; its status word is read by dlm_get_device_status.
+ * Errors: n_slots outside 0..DLM_DECISION_MAX_SLOTS, vocab <= 0, a bad
+ * label_softmax, a negative or non-finite brier_weight, smoothing outside
+ * [0, 1], a null pointer or ld / ld_out < vocab return
+ * DLM_ERR_INVALID_ARGUMENT before anything is enqueued.  On the device, a
+ * slot whose answer id is outside [0, vocab) sets DLM_DEV_BAD_TOKEN_ID; K
+ * outside 1..128, repeated answer ids, an unknown kind or a malformed label
+ * set DLM_DEV_BAD_LABEL; such a slot adds 0 to the loss (the mean still
+ * divides by n_slots) and its dlogits row is all zeros.  n_slots = 0 writes
+ * loss = 0.  The 16-byte load path needs ld and ld_out multiples of 8 and
+ * 16-byte aligned logits and dlogits; other shapes take a scalar path.
+ * Not built: full_ce_weighting: dft (the page gives no formula).
+ * ---------------------------------------------------------------------- */
+#define DLM_LABEL_HARD 0
+#define DLM_LABEL_DIST 1
+#define DLM_LABEL_SET 2
+#define DLM_LABEL_SOFTMAX_RESTRICTED 1
+#define DLM_LABEL_SOFTMAX_FULL 2
+#define DLM_LABEL_SOFTMAX_BOTH 3
+#define DLM_DECISION_MAX_ANSWERS 128
+#define DLM_DECISION_MAX_SLOTS 65535
+
+DLM_API size_t dlm_decision_workspace_size(int32_t n_slots, int32_t vocab);
+
+DLM_API dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_t *logits, int64_t ld,
+                                       int32_t vocab, const int64_t *slot_rows,
+                                       const int32_t *cand_off, const int32_t *cand_ids,
+                                       const int32_t *label_kind, const float *label_val,
+                                       int32_t label_softmax, float brier_weight,
+                                       float hard_label_smoothing, float grad_scale, float *loss,
+                                       float *slot_loss, uint16_t *dlogits, int64_t ld_out,
+                                       void *workspace, size_t workspace_bytes, dlm_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * dlm_scale_bf16 -- x[r, c] *= *scale in place for r < rows, c < cols (bf16,
+ * row stride ld >= cols), where scale is a DEVICE float: the upstream
+ * gradient of a scalar loss, applied by an autograd backward to a gradient
+ * the loss call has already written with grad_scale = 1.  When *scale is
+ * exactly 1 (loss.backward() on the loss itself) the kernel reads it and
+ * returns without touching x, so the host never needs to read the scalar.
+ * Otherwise each element is rounded to bf16 again after the product (one
+ * more rounding than passing the factor as grad_scale to the loss call).
+ * The pages have no counterpart: this serves the autograd wrappers of the
+ * Python binding.  rows or cols = 0 is a no-op; a negative size, ld < cols
+ * or a null pointer return DLM_ERR_INVALID_ARGUMENT.
+ * ---------------------------------------------------------------------- */
+DLM_API dlm_status_t dlm_scale_bf16(uint16_t *x, int64_t rows, int64_t cols, int64_t ld,
+                                    const float *scale, dlm_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -523,7 +523,7 @@ def decision_targets(kind: int, val: np.ndarray, smoothing: float):
     if K < 1:
         raise ValueError("a question has at least one alternative")
     if kind == HARD:
-        if not (np.count_nonzero(val) == 1 and val.max() == 1.0 and val.min() == 0.0):
+        if not (np.count_nonzero(val) == 1 and ((val == 0.0) | (val == 1.0)).all()):
             raise ValueError("hard label: exactly one 1, zeros elsewhere")
         y = val.copy()
         q = (1.0 - smoothing) * y + smoothing / K

@@ -1,0 +1,200 @@
+"""GPU parity of the typed-decision losses at label slots against the CPU
+oracle ("Native diffusion language-model training", Typed-decision training
+and Labels): loss within 1e-5 relative, every slot's share, and the bf16
+gradient of every logit -- on the full 128-slot workload, on ragged
+vocabularies and row strides (the scalar path), with 128 answers per
+question, a slot-row indirection, every label_softmax setting, smoothing,
+and slots whose labels the kernel must refuse.
+
+Gradient bar: entries away from the answer tokens are g w Q P_v, one
+product rounded to bf16 -- the gradient bar of the other losses (2e-3
+absolute and within one bf16 ulp of the rounded exact value).  The K
+answer-token entries add up to five fp32 terms of size up to |g w| (Q +
+2 + 4 b) that may cancel, so their bar is one bf16 ulp plus 2^-20 of that
+size (fp32 rounding of the terms).
+"""
+import numpy as np
+import pytest
+import torch
+
+import dlm_inputs as di
+import oracle
+from parity import assert_grad_close, assert_loss_close, bf16_ulp, gpu_bf16_to_f64
+
+pytestmark = pytest.mark.gpu
+
+dlm = pytest.importorskip("diffusion_lm_loss_b200")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dlm.lib()
+
+
+def _batch(seed, n, V, kmax, kinds=(0, 1, 2), kmin=1):
+    rng = np.random.default_rng(seed)
+    off = [0]
+    ids, kind, vals = [], [], []
+    for i in range(n):
+        K = int(rng.integers(kmin, kmax + 1))
+        ids.append(rng.choice(V, size=K, replace=False))
+        k = kinds[i % len(kinds)]
+        if k == oracle.HARD:
+            v = np.zeros(K, np.float32)
+            v[rng.integers(K)] = 1.0
+        elif k == oracle.DIST:
+            v = rng.dirichlet(np.ones(K))
+            if K > 2:
+                v[rng.integers(K)] = 0.0            # a zero entry is a valid probability
+            v = (v / v.sum()).astype(np.float32)
+        else:
+            v = np.zeros(K, np.float32)
+            v[rng.choice(K, size=int(rng.integers(1, K + 1)), replace=False)] = 1.0
+        kind.append(k)
+        vals.append(v)
+        off.append(off[-1] + K)
+    return (np.array(off, np.int32), np.concatenate(ids).astype(np.int32), np.array(kind, np.int32),
+            np.concatenate(vals).astype(np.float32))
+
+
+def _dev(*arrays):
+    return [torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in arrays]
+
+
+def _check(out, ref, off, ids, kinds_used, grad_scale, brier_w, n, V, label_softmax):
+    assert_loss_close(float(out.loss.item()), ref["loss"])
+    sl = out.slot_loss.cpu().numpy()[:n].astype(np.float64)
+    np.testing.assert_allclose(sl, ref["slot_loss"], rtol=1e-5, atol=1e-7 * abs(ref["loss"]))
+    g = gpu_bf16_to_f64(out.dlogits)[:, :V]
+    exact = ref["dlogits"]
+    cand = np.zeros((n, V), bool)
+    for i in range(n):
+        cand[i, ids[off[i]:off[i + 1]]] = True
+    # away from the answer tokens: one rounded product
+    assert_grad_close(np.where(cand, 0.0, g), np.where(cand, 0.0, exact), "dlogits (dense part)")
+    # at the answer tokens: a few fp32 terms that may cancel
+    Qmax = 1.0 + 1e-4
+    size = abs(grad_scale) / n * (2 * Qmax + 2 + 4 * brier_w)
+    err = np.abs(g[cand] - exact[cand])
+    tol = bf16_ulp(np.maximum(np.abs(g[cand]), np.abs(exact[cand]))) + 2.0 ** -20 * size
+    assert (err <= tol).all(), f"dlogits at answer tokens: max err {err.max():.3e}, worst tol {tol[np.argmax(err - tol)]:.3e}"
+
+
+@pytest.mark.parametrize("label_softmax", [oracle.LABEL_BOTH, oracle.LABEL_RESTRICTED, oracle.LABEL_FULL])
+def test_decision_full_workload(label_softmax):
+    """The 128-slot workload (K in [2, 26] from one codebook, V = 126,464,
+    16-byte path, three CTAs per row) against the oracle, every gradient
+    element."""
+    spec = di.WORKLOADS["dec_s128_k26_v126464"]
+    case = di.make_case(spec, "cuda")
+    e = case.extra
+    out = dlm.decision_loss_fwd_bwd(case.logits, spec.vocab, e["cand_off"], e["cand_ids"], e["kind"], e["val"],
+                                    label_softmax=label_softmax, brier_weight=0.1, hard_label_smoothing=0.05)
+    torch.cuda.synchronize()
+    assert out.device_status() == 0
+    off, ids = e["cand_off"].cpu().numpy(), e["cand_ids"].cpu().numpy()
+    ref = oracle.decision_loss(di.bf16_bits(case.logits), spec.vocab, None, off, ids, e["kind"].cpu().numpy(),
+                               e["val"].cpu().numpy(), label_softmax=label_softmax, brier_weight=0.1,
+                               smoothing=0.05)
+    _check(out, ref, off, ids, None, 1.0, 0.1, spec.n_units, spec.vocab, label_softmax)
+
+
+@pytest.mark.parametrize("n,V,kmin,kmax,ld_pad,seed", [
+    (37, 5003, 1, 128, 3, 0),     # ragged V and row stride: the scalar path; 1 to 128 answers
+    (5, 126464, 2, 26, 0, 1),     # few slots: many CTAs per row
+    (300, 2048, 2, 8, 0, 2),      # many slots, one CTA per row
+    (3, 16, 16, 16, 0, 3),        # every token of the vocabulary an answer
+])
+def test_decision_elementwise(n, V, kmin, kmax, ld_pad, seed):
+    off, ids, kind, val = _batch(seed, n, V, kmax, kmin=kmin)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(seed)
+    base = (torch.randn((n, V + ld_pad), generator=gen, device="cuda") * 2.5).to(torch.bfloat16)
+    logits = base[:, :V] if ld_pad else base
+    d_off, d_ids, d_kind, d_val = _dev(off, ids, kind, val)
+    out = dlm.decision_loss_fwd_bwd(logits, V, d_off, d_ids, d_kind, d_val, brier_weight=0.3,
+                                    hard_label_smoothing=0.1, grad_scale=-0.75)
+    torch.cuda.synchronize()
+    assert out.device_status() == 0
+    ref = oracle.decision_loss(di.bf16_bits(logits), V, None, off, ids, kind, val, brier_weight=0.3,
+                               smoothing=0.1, grad_scale=-0.75)
+    _check(out, ref, off, ids, None, -0.75, 0.3, n, V, oracle.LABEL_BOTH)
+
+
+def test_decision_slot_rows_indirection():
+    """Slots reading rows of a larger logits tensor (slot_rows) give the
+    same results as the same rows passed compactly."""
+    n, V = 24, 4096
+    off, ids, kind, val = _batch(4, n, V, 26)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(4)
+    big = (torch.randn((200, V), generator=gen, device="cuda") * 3).to(torch.bfloat16)
+    rows = torch.randperm(200, generator=torch.Generator().manual_seed(1))[:n].to(torch.int64)
+    d_off, d_ids, d_kind, d_val = _dev(off, ids, kind, val)
+    a = dlm.decision_loss_fwd_bwd(big, V, d_off, d_ids, d_kind, d_val, slot_rows=rows.cuda())
+    b = dlm.decision_loss_fwd_bwd(big[rows.cuda()].contiguous(), V, d_off, d_ids, d_kind, d_val)
+    torch.cuda.synchronize()
+    assert a.loss.item() == b.loss.item()
+    assert torch.equal(a.dlogits.view(torch.int16), b.dlogits.view(torch.int16))
+    ref = oracle.decision_loss(di.bf16_bits(big), V, rows.numpy(), off, ids, kind, val)
+    _check(a, ref, off, ids, None, 1.0, 0.1, n, V, oracle.LABEL_BOTH)
+
+
+def test_decision_invalid_slots_are_flagged_and_skipped():
+    """An answer id outside the vocabulary, a repeated answer id and a hard
+    label with two golds: status bits, zero loss share and zero gradient
+    rows for those slots; the other slots are unaffected (the mean still
+    divides by every slot)."""
+    n, V = 12, 3000
+    off, ids, kind, val = _batch(5, n, V, 10, kmin=3)
+    good = np.ones(n, bool)
+    ids_bad = ids.copy()
+    ids_bad[off[2]] = V + 5                          # slot 2: id outside [0, V)
+    ids_bad[off[5] + 1] = ids_bad[off[5]]            # slot 5: repeated answer
+    val_bad = val.copy()
+    h = int(np.nonzero(kind == oracle.HARD)[0][-1])  # a hard slot: two golds
+    val_bad[off[h]:off[h + 1]] = 0.0
+    val_bad[off[h]:off[h] + 2] = 1.0
+    for s in (2, 5, h):
+        good[s] = False
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(5)
+    logits = (torch.randn((n, V), generator=gen, device="cuda") * 2).to(torch.bfloat16)
+    out = dlm.decision_loss_fwd_bwd(logits, V, *_dev(off, ids_bad, kind, val_bad))
+    torch.cuda.synchronize()
+    st = out.device_status()
+    assert st & dlm.DEV_BAD_TOKEN_ID and st & dlm.DEV_BAD_LABEL
+    g = out.dlogits.float().cpu()
+    sl = out.slot_loss.cpu().numpy()[:n]
+    for s in np.nonzero(~good)[0]:
+        assert sl[s] == 0.0 and bool((g[s] == 0).all())
+    # the valid slots alone, with the mean over all n slots
+    keep = np.nonzero(good)[0]
+    ref = oracle.decision_loss(di.bf16_bits(logits), V, keep, np.concatenate([[0], np.cumsum(np.diff(off)[keep])]),
+                               np.concatenate([ids[off[i]:off[i + 1]] for i in keep]), kind[keep],
+                               np.concatenate([val[off[i]:off[i + 1]] for i in keep]))
+    scale = len(keep) / n
+    assert_loss_close(float(out.loss.item()), ref["loss"] * scale)
+    np.testing.assert_allclose(sl[keep], ref["slot_loss"] * scale, rtol=1e-5)
+    # a call after the failing one starts from a clean status word
+    out2 = dlm.decision_loss_fwd_bwd(logits, V, *_dev(off, ids, kind, val), out=out)
+    assert out2.device_status() == 0
+
+
+def test_decision_no_slots_and_reproducible():
+    V = 1024
+    z = torch.zeros((0, V), dtype=torch.bfloat16, device="cuda")
+    out = dlm.decision_loss_fwd_bwd(z, V, *_dev(np.zeros(1, np.int32), np.zeros(0, np.int32),
+                                                np.zeros(0, np.int32), np.zeros(0, np.float32)))
+    torch.cuda.synchronize()
+    assert float(out.loss.item()) == 0.0 and out.device_status() == 0
+    spec = di.WORKLOADS["dec_s128_k26_v126464"]
+    case = di.make_case(spec, "cuda")
+    e = case.extra
+    a = dlm.decision_loss_fwd_bwd(case.logits, spec.vocab, e["cand_off"], e["cand_ids"], e["kind"], e["val"])
+    b = dlm.decision_loss_fwd_bwd(case.logits, spec.vocab, e["cand_off"], e["cand_ids"], e["kind"], e["val"])
+    torch.cuda.synchronize()
+    assert a.loss.item() == b.loss.item()
+    assert torch.equal(a.dlogits.view(torch.int16), b.dlogits.view(torch.int16))

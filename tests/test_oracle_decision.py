@@ -227,3 +227,13 @@ def test_invalid_labels_are_refused():
         one_slot(z, [1, 2], SET, [0.0, 0.0])                # empty set
     with pytest.raises(ValueError):
         one_slot(z, [1, 2], DIST, [1.5, -0.5])              # negative probability
+
+
+def test_single_answer_question():
+    """K = 1: the restricted softmax is certain (CE_res = 0, Brier = 0 for
+    any label), the full CE is the plain CE of that token."""
+    z = np.array([0.3, -1.2, 2.0, 0.1])
+    for kind in (HARD, DIST, SET):
+        r = one_slot(z, [2], kind, [1.0])
+        assert r["ce_res"][0] == 0.0 and r["brier"][0] == 0.0
+        assert r["ce_full"][0] == pytest.approx(math.log(np.exp(z).sum()) - 2.0, rel=1e-14)
