@@ -33,6 +33,8 @@
 // Invalid slots (an answer id outside [0, V), repeated answer ids, K outside
 // 1..128, a malformed label) set a status bit and contribute a zero loss
 // and a zero gradient row.
+#include <mutex>
+
 #include "dlm_device.cuh"
 #include "dlm_host.h"
 
@@ -62,6 +64,7 @@ struct DecParams {
     uint16_t* dlogits;
     int64_t ld_out;
     uint32_t* status;
+    uint32_t* err;                     // cluster path: [n_slots][n_split] error words, or null
     int vec;                           // 16-byte loads and stores allowed
 };
 
@@ -155,11 +158,155 @@ __device__ __forceinline__ int warp_sum_i(int v) {
     return v;
 }
 
+// Per-slot state in shared memory: what one warp works out about the
+// slot's answers and label.
+struct DecSlot {
+    int id[DLM_DECISION_MAX_ANSWERS];     // answer token ids
+    float z[DLM_DECISION_MAX_ANSWERS];    // their logits
+    float q[DLM_DECISION_MAX_ANSWERS];    // CE target
+    float gr[DLM_DECISION_MAX_ANSWERS];   // restricted-CE + Brier part of d loss / dz (no g w)
+    float g[DLM_DECISION_MAX_ANSWERS];    // the full gradient value written at each answer token
+    float Q, qz, ce_res, brier, coef;     // sum q, sum q z, CE_res, Brier; dense coefficient g w [full] Q
+    int K;                                // answer entries to write (0 for an invalid slot)
+    uint32_t bad;                         // status bits the slot raises (0 when valid)
+};
+
+// One warp, before the row's lse is known: the K answer tokens and the
+// label -- validity, the restricted softmax, the targets, CE_res, Brier and
+// the restricted + Brier part of each answer's gradient.  Needs only the K
+// answer logits, so it runs while the row itself is still being loaded.
+__device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, const uint16_t* x, int lane,
+                                                 DecSlot& S) {
+    const int o0 = P.cand_off[slot], o1 = P.cand_off[slot + 1];
+    const int K = o1 - o0;
+    const int kind = P.kind[slot];
+    int bad = (K < 1 || K > DLM_DECISION_MAX_ANSWERS) ? 2 : 0;
+    bad |= (kind != DLM_LABEL_HARD && kind != DLM_LABEL_DIST && kind != DLM_LABEL_SET) ? 2 : 0;
+    float z[4], v[4];
+    int id[4];
+    int n_one = 0, n_other = 0;    // label checks: values equal to 1, and not in {0, 1}
+    int bad_id = 0, bad_dist = 0;
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int k = lane + 32 * j;
+        id[j] = -1; z[j] = -INFINITY; v[j] = 0.f;
+        if (!bad && k < K) {
+            id[j] = P.cand_ids[o0 + k];
+            v[j] = P.val[o0 + k];
+        }
+    }
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int k = lane + 32 * j;
+        if (!bad && k < K) {
+            if (id[j] < 0 || id[j] >= P.vocab) { bad_id = 1; id[j] = -1; }
+            else z[j] = bf16_bits_to_float(x[id[j]]);
+            n_one += (v[j] == 1.f);
+            n_other += (v[j] != 0.f && v[j] != 1.f);
+            bad_dist |= !(v[j] >= 0.f && v[j] < INFINITY);
+            S.id[k] = id[j];
+        }
+    }
+    __syncwarp();
+    // repeated answer ids: each lane compares its answers with the earlier ones
+    int dup = 0;
+    if (!bad) {
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int k = lane + 32 * j;
+            if (k < K && id[j] >= 0)
+                for (int i = 0; i < k; ++i) dup |= (S.id[i] == id[j]);
+        }
+    }
+    n_one = warp_sum_i(n_one);
+    n_other = warp_sum_i(n_other);
+    bad_id = __any_sync(0xffffffffu, bad_id);
+    dup = __any_sync(0xffffffffu, dup);
+    bad_dist = __any_sync(0xffffffffu, bad_dist);
+    if (!bad) {
+        if (bad_id) bad = 1;
+        else if (dup) bad = 2;
+        else if (kind == DLM_LABEL_HARD && !(n_one == 1 && n_other == 0)) bad = 2;
+        else if (kind == DLM_LABEL_SET && !(n_one >= 1 && n_other == 0)) bad = 2;
+        else if (kind == DLM_LABEL_DIST && bad_dist) bad = 2;
+    }
+    if (!bad) {
+        // candidate-restricted softmax
+        const float cm = warp_max(fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3])));
+        float se = 0.f;
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) se += (lane + 32 * j < K) ? expf(z[j] - cm) : 0.f;
+        const float lse_r = cm + logf(warp_sum(se));
+        const float n_set = float(n_one);
+        float r[4], q[4], y[4];
+        float Q = 0.f, qz = 0.f, ce_res = 0.f, brier = 0.f, D = 0.f;
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const bool on = lane + 32 * j < K;
+            r[j] = on ? expf(z[j] - lse_r) : 0.f;
+            if (kind == DLM_LABEL_HARD) { y[j] = v[j]; q[j] = (1.f - P.smoothing) * v[j] + P.smoothing / float(K); }
+            else if (kind == DLM_LABEL_SET) { y[j] = v[j] / n_set; q[j] = y[j]; }
+            else { y[j] = v[j]; q[j] = v[j]; }
+            if (!on) { q[j] = 0.f; y[j] = 0.f; }
+            Q += q[j];
+            qz += on ? q[j] * z[j] : 0.f;
+            ce_res -= on ? q[j] * (z[j] - lse_r) : 0.f;
+            const float d = r[j] - y[j];
+            brier += d * d;
+            D += r[j] * d;
+        }
+        Q = warp_sum(Q);
+        qz = warp_sum(qz);
+        ce_res = warp_sum(ce_res);
+        brier = warp_sum(brier);
+        D = warp_sum(D);
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int k = lane + 32 * j;
+            if (k < K) {
+                float g = P.brier_w * 2.f * r[j] * ((r[j] - y[j]) - D);
+                if (P.use_res) g += Q * r[j] - q[j];
+                S.gr[k] = g;
+                S.z[k] = z[j];
+                S.q[k] = q[j];
+            }
+        }
+        if (lane == 0) { S.Q = Q; S.qz = qz; S.ce_res = ce_res; S.brier = brier; }
+    }
+    if (lane == 0) {
+        S.K = bad ? 0 : K;
+        S.bad = bad == 0 ? 0u : (bad == 1 ? DLM_DEV_BAD_TOKEN_ID : DLM_DEV_BAD_LABEL);
+    }
+}
+
+// One warp, once lse is known: the full-vocabulary CE and its share of each
+// answer's gradient, the answers' final values (S.g), the dense coefficient
+// (S.coef) and, from split 0, the slot's loss share.  Call after the
+// prepare step is visible to the warp (same warp, or after a barrier).
+__device__ __forceinline__ void dec_slot_finish(const DecParams& P, int slot, int split, float lse, int lane,
+                                                DecSlot& S) {
+    const int K = S.K;
+    const float gw = P.grad_scale * P.w;
+    const float Q = K > 0 ? S.Q : 0.f;
+    for (int k = lane; k < K; k += 32) {
+        float g = S.gr[k];
+        if (P.use_full) g += Q * expf(S.z[k] - lse) - S.q[k];
+        S.g[k] = gw * g;
+    }
+    if (lane == 0) {
+        float slot_loss = 0.f;
+        if (K > 0) {
+            const float ce_full = Q * lse - S.qz;     // -sum q_k (z_k - lse)
+            slot_loss = P.w * (P.use_res * S.ce_res + P.use_full * ce_full + P.brier_w * S.brier);
+        }
+        S.coef = gw * float(P.use_full) * Q;
+        if (split == 0) P.slot_loss[slot] = slot_loss;
+    }
+}
+
 __global__ void __launch_bounds__(kDecThreads) k_dec_grad(DecParams P) {
-    __shared__ int s_id[DLM_DECISION_MAX_ANSWERS];
-    __shared__ float s_g[DLM_DECISION_MAX_ANSWERS];
-    __shared__ float s_lse, s_coef;
-    __shared__ int s_k;
+    __shared__ DecSlot S;
+    __shared__ float s_lse;
     const int split = blockIdx.x, slot = blockIdx.y, tid = threadIdx.x;
     pdl_wait();                        // partials of k_dec_partial
     pdl_launch_dependents();
@@ -175,113 +322,15 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_grad(DecParams P) {
     __syncthreads();
     const float lse = s_lse;
     if (tid < 32) {
-        const int lane = tid;
-        const int o0 = P.cand_off[slot], o1 = P.cand_off[slot + 1];
-        const int K = o1 - o0;
-        const int kind = P.kind[slot];
-        int bad = (K < 1 || K > DLM_DECISION_MAX_ANSWERS) ? 2 : 0;
-        bad |= (kind != DLM_LABEL_HARD && kind != DLM_LABEL_DIST && kind != DLM_LABEL_SET) ? 2 : 0;
-        float z[4], v[4];
-        int id[4];
-        int n_one = 0, n_other = 0;    // label checks: values equal to 1, and not in {0, 1}
-        int bad_id = 0, bad_dist = 0;
-        #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int k = lane + 32 * j;
-            id[j] = -1; z[j] = -INFINITY; v[j] = 0.f;
-            if (!bad && k < K) {
-                id[j] = P.cand_ids[o0 + k];
-                v[j] = P.val[o0 + k];
-                if (id[j] < 0 || id[j] >= P.vocab) { bad_id = 1; id[j] = -1; }
-                else z[j] = bf16_bits_to_float(x[id[j]]);
-                n_one += (v[j] == 1.f);
-                n_other += (v[j] != 0.f && v[j] != 1.f);
-                bad_dist |= !(v[j] >= 0.f && v[j] < INFINITY);
-                s_id[k] = id[j];
-            }
-        }
+        dec_slot_prepare(P, slot, x, tid, S);
         __syncwarp();
-        // repeated answer ids: each lane compares its answers with the earlier ones
-        int dup = 0;
-        if (!bad) {
-            #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int k = lane + 32 * j;
-                if (k < K && id[j] >= 0)
-                    for (int i = 0; i < k; ++i) dup |= (s_id[i] == id[j]);
-            }
-        }
-        n_one = warp_sum_i(n_one);
-        n_other = warp_sum_i(n_other);
-        bad_id = __any_sync(0xffffffffu, bad_id);
-        dup = __any_sync(0xffffffffu, dup);
-        bad_dist = __any_sync(0xffffffffu, bad_dist);
-        if (!bad) {
-            if (bad_id) bad = 1;
-            else if (dup) bad = 2;
-            else if (kind == DLM_LABEL_HARD && !(n_one == 1 && n_other == 0)) bad = 2;
-            else if (kind == DLM_LABEL_SET && !(n_one >= 1 && n_other == 0)) bad = 2;
-            else if (kind == DLM_LABEL_DIST && bad_dist) bad = 2;
-        }
-        float slot_loss = 0.f;
-        if (!bad) {
-            // candidate-restricted softmax
-            const float cm = warp_max(fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3])));
-            float se = 0.f;
-            #pragma unroll
-            for (int j = 0; j < 4; ++j) se += (lane + 32 * j < K) ? expf(z[j] - cm) : 0.f;
-            const float lse_r = cm + logf(warp_sum(se));
-            const float n_set = float(n_one);
-            float r[4], q[4], y[4];
-            float Q = 0.f, ce_res = 0.f, ce_full = 0.f, brier = 0.f, D = 0.f;
-            #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const bool on = lane + 32 * j < K;
-                r[j] = on ? expf(z[j] - lse_r) : 0.f;
-                if (kind == DLM_LABEL_HARD) { y[j] = v[j]; q[j] = (1.f - P.smoothing) * v[j] + P.smoothing / float(K); }
-                else if (kind == DLM_LABEL_SET) { y[j] = v[j] / n_set; q[j] = y[j]; }
-                else { y[j] = v[j]; q[j] = v[j]; }
-                if (!on) { q[j] = 0.f; y[j] = 0.f; }
-                Q += q[j];
-                ce_res -= on ? q[j] * (z[j] - lse_r) : 0.f;
-                ce_full -= on ? q[j] * (z[j] - lse) : 0.f;
-                const float d = r[j] - y[j];
-                brier += d * d;
-                D += r[j] * d;
-            }
-            Q = warp_sum(Q);
-            ce_res = warp_sum(ce_res);
-            ce_full = warp_sum(ce_full);
-            brier = warp_sum(brier);
-            D = warp_sum(D);
-            const float gw = P.grad_scale * P.w;
-            #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int k = lane + 32 * j;
-                if (k < K) {
-                    float g = P.brier_w * 2.f * r[j] * ((r[j] - y[j]) - D);
-                    if (P.use_full) g += Q * expf(z[j] - lse) - q[j];
-                    if (P.use_res) g += Q * r[j] - q[j];
-                    s_g[k] = gw * g;
-                }
-            }
-            slot_loss = P.w * (P.use_res * ce_res + P.use_full * ce_full + P.brier_w * brier);
-            if (lane == 0) s_coef = gw * float(P.use_full) * Q;
-        } else if (lane == 0) {
-            s_coef = 0.f;
-        }
-        if (lane == 0) {
-            s_k = bad ? 0 : K;
-            if (split == 0) {
-                P.slot_loss[slot] = slot_loss;
-                if (bad) atomicOr(P.status, bad == 1 ? DLM_DEV_BAD_TOKEN_ID : DLM_DEV_BAD_LABEL);
-            }
-        }
+        dec_slot_finish(P, slot, split, lse, tid, S);
     }
     __syncthreads();
+    if (tid == 0 && split == 0 && S.bad) atomicOr(P.status, S.bad);
     // the dense part of this split: coef * P_v (zeros for a restricted-only
     // loss or an invalid slot)
-    const float coef = s_coef;
+    const float coef = S.coef;
     const float sh = lse * kDecLog2e;
     uint16_t* out = P.dlogits + int64_t(slot) * P.ld_out;
     const int c0 = split * P.chunk;
@@ -325,24 +374,152 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_grad(DecParams P) {
         out[c] = __bfloat16_as_ushort(__float2bfloat16_rn(g));
     }
     __syncthreads();                   // the dense stores of this CTA come first
-    const int K = s_k;
+    const int K = S.K;
     for (int k = tid; k < K; k += kDecThreads) {
-        const int id = s_id[k];
-        if (id >= c0 && id < c1) out[id] = __bfloat16_as_ushort(__float2bfloat16_rn(s_g[k]));
+        const int id = S.id[k];
+        if (id >= c0 && id < c1) out[id] = __bfloat16_as_ushort(__float2bfloat16_rn(S.g[k]));
     }
+}
+
+// Fast path: one thread-block cluster per slot, one CTA per split of the
+// row (cluster rank = split).  Each CTA brings its split of the row into
+// shared memory once (bulk copies from HBM, one mbarrier per 8 KB piece, so
+// the sums start on the first piece), forms its (max, sum exp), and the
+// cluster exchanges only those two floats through distributed shared
+// memory: every CTA merges the n_split partials in rank order into the
+// same lse.  The gradient of the split is then written from shared memory
+// -- the row is read from HBM exactly once and never from L2 again -- and
+// the answer-token entries rewritten as in k_dec_grad.  The second cluster
+// barrier keeps every CTA's partial alive until all peers have read it.
+constexpr int kDecPieceBytes = 8192;
+constexpr int kDecMaxPieces = 16;     // slices up to 128 KB (65,536 columns)
+
+__global__ void __launch_bounds__(kDecThreads, 6) k_dec_cluster(DecParams P) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    __shared__ __align__(8) uint64_t bars[kDecMaxPieces];
+    __shared__ __align__(8) float2 s_part;
+    __shared__ float sm_m[kDecThreads / 32], sm_s[kDecThreads / 32];
+    __shared__ DecSlot S;
+    __shared__ float s_lse;
+    const int tid = threadIdx.x, lane = tid & 31;
+    const int split = int(cluster_ctarank()), slot = blockIdx.y;
+    const int c0 = split * P.chunk;
+    const int c1 = min(c0 + P.chunk, P.vocab);
+    const int nvec = c1 > c0 ? (c1 - c0) / 8 : 0;                 // the host gives vocab % 8 == 0
+    const uint32_t bytes = uint32_t(nvec) * 16u;
+    const int pieces = int((bytes + kDecPieceBytes - 1) / kDecPieceBytes);
+    const uint16_t* x = P.logits + slot_row(P, slot) * P.ld;
+    if (tid == 0) {
+        for (int i = 0; i < pieces; ++i) mbar_init(smem_addr(&bars[i]), 1);
+        fence_mbar_init_cluster();
+    }
+    __syncthreads();
+    pdl_wait();                        // the previous call may still read the outputs
+    pdl_launch_dependents();
+    if (tid == 0) {
+        const uint64_t pol = policy_evict_first();   // read once
+        for (int i = 0; i < pieces; ++i) {
+            const uint32_t off = uint32_t(i) * kDecPieceBytes;
+            const uint32_t n = bytes - off < uint32_t(kDecPieceBytes) ? bytes - off : uint32_t(kDecPieceBytes);
+            const uint32_t b = smem_addr(&bars[i]);
+            mbar_arrive_expect_tx(b, n);
+            bulk_g2s_hint(smem_addr(dsm) + off, reinterpret_cast<const uint8_t*>(x + c0) + off, n, b, pol);
+        }
+    }
+    // while the row lands: the answers and the label (one warp)
+    if (tid < 32) dec_slot_prepare(P, slot, x, tid, S);
+    const uint4* sv = reinterpret_cast<const uint4*>(dsm);
+    constexpr int kPieceVec = kDecPieceBytes / 16;
+    float m = -INFINITY, s = 0.f;
+    bool ok = true;
+    for (int i = 0; i < pieces; ++i) {
+        ok = ok && mbar_wait_bounded<false>(smem_addr(&bars[i]), 0, nullptr);
+        if (!ok) break;                  // the copy never landed: reported in this CTA's error word
+        const int v1 = min(nvec, (i + 1) * kPieceVec);
+        for (int v = i * kPieceVec + tid; v < v1; v += kDecThreads) acc_vec(sv[v], m, s);
+    }
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+        const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+        lse_merge(m, s, m2, s2);
+    }
+    if (lane == 0) { sm_m[tid >> 5] = m; sm_s[tid >> 5] = s; }
+    __syncthreads();
+    if (tid == 0) {
+        float M = sm_m[0], S = sm_s[0];
+        for (int k = 1; k < kDecThreads / 32; ++k) lse_merge(M, S, sm_m[k], sm_s[k]);
+        s_part = make_float2(M, S);
+    }
+    cluster_sync_all();                // every split's partial is published
+    if (tid == 0) {
+        float M = -INFINITY, S = 0.f;
+        for (int r = 0; r < P.n_split; ++r) {
+            float pm, ps;
+            const uint32_t a = mapa_shared(smem_addr(&s_part), uint32_t(r));
+            asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(pm), "=f"(ps) : "r"(a) : "memory");
+            lse_merge(M, S, pm, ps);
+        }
+        s_lse = M + logf(S);
+    }
+    __syncthreads();
+    const float lse = s_lse;
+    if (tid < 32) dec_slot_finish(P, slot, split, lse, tid, S);
+    // this CTA's error word (every CTA writes its own, every call; the
+    // reduction kernel ors them into the status word)
+    const int all_ok = __syncthreads_and(ok ? 1 : 0);
+    if (tid == 0)
+        P.err[int64_t(slot) * P.n_split + split] = (all_ok ? 0u : DLM_DEV_WAIT_TIMEOUT) | (split == 0 ? S.bad : 0u);
+    const float coef = all_ok ? S.coef : 0.f;
+    const float sh = lse * kDecLog2e;
+    uint16_t* out = P.dlogits + int64_t(slot) * P.ld_out;
+    uint4* ov = reinterpret_cast<uint4*>(out + c0);
+    const uint64_t ef = policy_evict_first();
+    for (int v = tid; v < nvec; v += kDecThreads) {
+        if (!all_ok) { st_global_v4_hint(ov + v, make_uint4(0u, 0u, 0u, 0u), ef); continue; }
+        const uint4 rv = sv[v];
+        const uint32_t w4[4] = {rv.x, rv.y, rv.z, rv.w};
+        uint32_t o4[4];
+        #pragma unroll
+        for (int k = 0; k < 4; ++k)
+            o4[k] = pack_bf16x2(coef * ex2(fmaf(bf16lo(w4[k]), kDecLog2e, -sh)),
+                                coef * ex2(fmaf(bf16hi(w4[k]), kDecLog2e, -sh)));
+        st_global_v4_hint(ov + v, make_uint4(o4[0], o4[1], o4[2], o4[3]), ef);
+    }
+    __syncthreads();                   // the dense stores of this CTA come first
+    const int K = all_ok ? S.K : 0;
+    for (int k = tid; k < K; k += kDecThreads) {
+        const int id = S.id[k];
+        if (id >= c0 && id < c1) out[id] = __bfloat16_as_ushort(__float2bfloat16_rn(S.g[k]));
+    }
+    cluster_sync_all();                // no CTA leaves while a peer may read its partial
 }
 
 constexpr int kDecRedThreads = 256;
 
+// The mean over slots (fixed order, double) and, after the cluster path,
+// the status word: the or of every CTA's error word (written on every call,
+// so nothing needs zeroing between calls).
 __global__ void __launch_bounds__(kDecRedThreads) k_dec_reduce(const float* __restrict__ slot_loss, int n,
-                                                               float* __restrict__ loss) {
+                                                               float* __restrict__ loss,
+                                                               const uint32_t* __restrict__ err, int n_err,
+                                                               uint32_t* __restrict__ status) {
     __shared__ double red[kDecRedThreads];
+    __shared__ uint32_t bits;
     const int tid = threadIdx.x;
-    pdl_wait();                        // slot losses of k_dec_grad
+    pdl_wait();                        // slot losses of the gradient kernel
+    if (tid == 0) bits = 0u;
+    __syncthreads();
+    if (err) {
+        uint32_t b = 0u;
+        for (int i = tid; i < n_err; i += kDecRedThreads) b |= err[i];
+        if (b) atomicOr(&bits, b);
+    }
     double acc = 0.0;
     for (int i = tid; i < n; i += kDecRedThreads) acc += double(slot_loss[i]);
     red[tid] = acc;
     __syncthreads();
+    if (err && tid == 0) *status = bits;
     for (int o = kDecRedThreads / 2; o > 0; o >>= 1) {
         if (tid < o) red[tid] += red[tid + o];
         __syncthreads();
@@ -355,6 +532,25 @@ struct DecPlan {
     size_t partial_off, slot_loss_off, total;
 };
 
+// The cluster path: n_split in {1, 2, 4, 8} (a portable cluster size), the
+// smallest that keeps a slice within 64 KB of shared memory and, below 8,
+// gives about four CTAs per SM (592) without cutting slices under 2,048
+// columns.  Returns false when the row does not fit (the three-kernel path
+// runs instead).
+inline bool dec_cluster_plan(int n_slots, int vocab, int& n_split, int& chunk) {
+    if (n_slots <= 0 || vocab % 8 != 0) return false;
+    const int64_t want = (4 * 148 + n_slots - 1) / n_slots;   // CTAs wanted per slot
+    for (int ns = 1; ns <= 8; ns *= 2) {
+        const int64_t ch = (int64_t(vocab) / 8 + ns - 1) / ns * 8;
+        if (ch * 2 > 65536) continue;                          // slice too large
+        if (ns < 8 && ns < want && ch >= 2 * 2048) continue;   // more CTAs wanted, and slices can shrink
+        n_split = ns;
+        chunk = int(ch);
+        return true;
+    }
+    return false;
+}
+
 // Columns of a row per CTA: enough CTAs for two waves over 148 SMs, at
 // least 2,048 columns each.
 inline DecPlan dec_plan(int n_slots, int vocab) {
@@ -366,8 +562,8 @@ inline DecPlan dec_plan(int n_slots, int vocab) {
     p.chunk = int(((int64_t(vocab) + ns - 1) / ns + 7) / 8 * 8);
     p.n_split = int((int64_t(vocab) + p.chunk - 1) / p.chunk);
     size_t o = kWsAlign;               // status word in the first 256 bytes
-    p.partial_off = o;
-    o = align_up(o + size_t(n_slots) * size_t(p.n_split) * sizeof(float2), kWsAlign);
+    p.partial_off = o;                 // partials, or the cluster path's error words (up to 8 per slot)
+    o = align_up(o + size_t(n_slots) * size_t(p.n_split > 8 ? p.n_split : 8) * sizeof(float2), kWsAlign);
     p.slot_loss_off = o;
     o = align_up(o + size_t(n_slots) * sizeof(float), kWsAlign);
     p.total = o;
@@ -435,7 +631,44 @@ extern "C" dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_
     P.ld_out = ld_out;
     P.status = reinterpret_cast<uint32_t*>(ws);
     P.vec = (ld % 8 == 0) && (ld_out % 8 == 0) && aligned16(logits) && aligned16(dlogits);
-    if (n_slots > 0) {
+    int cl_split = 0, cl_chunk = 0;
+    if (n_slots > 0 && P.vec && dec_cluster_plan(n_slots, vocab, cl_split, cl_chunk)) {
+        // one cluster per slot: the row read once, lse partials through DSMEM
+        P.err = reinterpret_cast<uint32_t*>(ws + plan.partial_off);   // n_slots x cl_split words fit
+        DecParams C = P;
+        C.n_split = cl_split;
+        C.chunk = cl_chunk;
+        const size_t smem = size_t(cl_chunk) * 2;
+        static std::mutex mu;
+        static bool attr_done[64] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        {
+            std::lock_guard<std::mutex> lk(mu);
+            if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+                const cudaError_t e = cudaFuncSetAttribute(k_dec_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                           65536);
+                if (e != cudaSuccess) { cudaGetLastError(); return cuda_status(e, "k_dec_cluster smem attribute"); }
+                attr_done[dev] = true;
+            }
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(unsigned(cl_split), unsigned(n_slots));
+        cfg.blockDim = dim3(kDecThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute at[2];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = unsigned(cl_split);
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        at[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = at;
+        cfg.numAttrs = 2;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, k_dec_cluster, C);
+        if (e != cudaSuccess) { cudaGetLastError(); return cuda_status(e, "k_dec_cluster launch"); }
+    } else if (n_slots > 0) {
         const dim3 grid(unsigned(plan.n_split), unsigned(n_slots));
         if ((st = launch_pdl(k_dec_partial, grid, dim3(kDecThreads), 0, s, "k_dec_partial launch", P)) != DLM_OK)
             return st;
@@ -445,6 +678,8 @@ extern "C" dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_
         cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(uint32_t), s);
         if (e != cudaSuccess) { cudaGetLastError(); return cuda_status(e, "status reset"); }
     }
+    const bool clustered = cl_split > 0;
     return launch_pdl(k_dec_reduce, dim3(1), dim3(kDecRedThreads), 0, s, "k_dec_reduce launch",
-                      (const float*)P.slot_loss, n_slots, loss);
+                      (const float*)P.slot_loss, n_slots, loss, clustered ? (const uint32_t*)P.err : nullptr,
+                      clustered ? n_slots * cl_split : 0, P.status);
 }

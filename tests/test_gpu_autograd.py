@@ -58,7 +58,7 @@ def test_diffusion_loss_autograd():
     logits = case.logits.clone().requires_grad_(True)
     loss = dlm.diffusion_loss(lay, logits, spec.vocab, case.clean, corr, p)
     loss.backward()
-    assert float(loss) == float(direct.loss.item())
+    assert loss.item() == direct.loss.item()
     assert _same_bits(logits.grad, direct.dlogits)
     # a scaled loss: the library multiplies the kept gradient
     logits.grad = None
@@ -70,7 +70,7 @@ def test_diffusion_loss_autograd():
     _, corr_o = oracle.corrupt(lay_o, case.clean.cpu().numpy(), p_o, oracle.ABSORBING, spec.mask_id, spec.vocab, 0)
     x = di.bf16_bits(case.logits)
     loss_o, _, tr = oracle.loss_absorbing(lay_o, x, spec.vocab, case.clean.cpu().numpy(), corr_o, p_o, oracle.ALIGNED)
-    assert_loss_close(float(loss), loss_o)
+    assert_loss_close(loss.item(), loss_o)
     g_o = oracle.term_grad(x, spec.vocab, tr, np.arange(512), 1.0)
     assert_grad_close(direct.dlogits.float().cpu().double().numpy(), g_o)
 
@@ -101,7 +101,7 @@ def test_linear_losses_autograd_and_frozen_head():
     w = case.weight.clone().requires_grad_(True)
     loss = dlm.linear_diffusion_loss(lay, h, w, case.clean, corr, p)
     (loss * 0.5).backward()
-    assert float(loss) == float(direct.loss.item())
+    assert loss.item() == direct.loss.item()
     assert _same_bits(h.grad, (direct.d_hidden.float() * 0.5).to(torch.bfloat16))
     assert _same_bits(w.grad, (direct.d_weight.float() * 0.5).to(torch.bfloat16))
     h2 = case.hidden.clone().requires_grad_(True)
@@ -130,5 +130,5 @@ def test_decision_loss_autograd():
     z = case.logits.clone().requires_grad_(True)
     loss = dlm.decision_loss(z, spec.vocab, e["cand_off"], e["cand_ids"], e["kind"], e["val"])
     (-2.0 * loss).backward()
-    assert float(loss) == float(direct.loss.item())
+    assert loss.item() == direct.loss.item()
     assert _same_bits(z.grad, (direct.dlogits.float() * -2.0).to(torch.bfloat16))

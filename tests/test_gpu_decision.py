@@ -6,6 +6,10 @@ vocabularies and row strides (the scalar path), with 128 answers per
 question, a slot-row indirection, every label_softmax setting, smoothing,
 and slots whose labels the kernel must refuse.
 
+Both kernel paths are covered: the cluster path (one cluster of CTAs per
+slot holds the row in shared memory; aligned rows up to 262,144 columns)
+and the three-kernel path (any shape).
+
 Gradient bar: entries away from the answer tokens are g w Q P_v, one
 product rounded to bf16 -- the gradient bar of the other losses (2e-3
 absolute and within one bf16 ulp of the rounded exact value).  The K
@@ -102,10 +106,11 @@ def test_decision_full_workload(label_softmax):
 
 
 @pytest.mark.parametrize("n,V,kmin,kmax,ld_pad,seed", [
-    (37, 5003, 1, 128, 3, 0),     # ragged V and row stride: the scalar path; 1 to 128 answers
-    (5, 126464, 2, 26, 0, 1),     # few slots: many CTAs per row
+    (37, 5003, 1, 128, 3, 0),     # ragged V and row stride: three kernels, scalar loads; 1 to 128 answers
+    (5, 126464, 2, 26, 0, 1),     # few slots: clusters of 8 CTAs per row
     (300, 2048, 2, 8, 0, 2),      # many slots, one CTA per row
     (3, 16, 16, 16, 0, 3),        # every token of the vocabulary an answer
+    (4, 300000, 2, 26, 0, 4),     # a row too long for a cluster's shared memory: three kernels, 16-byte loads
 ])
 def test_decision_elementwise(n, V, kmin, kmax, ld_pad, seed):
     off, ids, kind, val = _batch(seed, n, V, kmax, kmin=kmin)
