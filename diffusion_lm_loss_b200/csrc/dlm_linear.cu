@@ -48,7 +48,13 @@ namespace dlm {
 constexpr int kBM = 128, kBN = 256, kBK = 64;   // per-CTA accumulator tile 128 x 256, K step 64
 constexpr int kGemmThreads = 192;
 constexpr uint32_t kStageA = kBM * kBK * 2;   // 16 KB: this CTA's 128 A rows x 64
-constexpr int kVc = 16384;                    // vocabulary chunk of the backward pass
+#ifndef DLM_LIN_VC
+#define DLM_LIN_VC 16384
+#endif
+#ifndef DLM_DH_N_FASTEST
+#define DLM_DH_N_FASTEST 1
+#endif
+constexpr int kVc = DLM_LIN_VC;               // vocabulary chunk of the backward pass
 constexpr int kRowPad = 256;                  // masked-row buffers are padded to the paired tile height
 
 // PAIR = 2: a CTA pair (cluster of 2) computes a 256 x 256 tile with
@@ -788,7 +794,7 @@ static dlm_status_t linear_loss_fwd_bwd(const dlm_layout_t* layout, const uint16
 
         GemmArgs h = g;
         h.m_dev = 1; h.n_cols = d_model; h.k_dev = 0; h.k_len = int(align_up(vc, kBK)); h.b_off = c0;
-        h.dh = dh; h.accumulate = c0 > 0; h.n_fastest = 1;
+        h.dh = dh; h.accumulate = c0 > 0; h.n_fastest = DLM_DH_N_FASTEST;
         if ((st = launch_gemm<EPI_DH, false, true>(mDZ_K, mW_MN, oDH, h, sms, s)) != DLM_OK) return st;
 
         if (d_weight) {
