@@ -43,7 +43,7 @@ def _corrupt_both(n_units, seq_len, cu, pad, clean, p, mode, mask_id, vocab, see
     return noisy.cpu().numpy(), corr.cpu().numpy(), no, co, int(status.item())
 
 
-@pytest.mark.parametrize("key", list(di.WORKLOADS))
+@pytest.mark.parametrize("key", [k for k, s in di.WORKLOADS.items() if s.kind != "decision"])   # label slots are not corrupted
 def test_corrupt_bit_exact_on_every_workload_shape(key):
     spec = di.WORKLOADS[key]
     case = di.make_case(spec, "cpu", with_tensors=False)

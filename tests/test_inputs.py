@@ -1,4 +1,5 @@
 """Host checks of the seeded synthetic-input generator (no method arithmetic)."""
+import numpy as np
 import torch
 
 import dlm_inputs as di
@@ -40,3 +41,31 @@ def test_shapes_and_ranges():
                                                         ids_high=990, mask_id=991)
     cl = di.make_case(l, "cpu")
     assert int(cl.cu_seqlens[-1]) == 512 and cl.hidden.shape == (512, 64) and cl.weight.shape == (1000, 64)
+
+
+def test_decision_workload_recipe():
+    """The typed-decision draws: K in [2, k_max] answers per slot, the first
+    K codebook tokens, distinct ids inside the vocabulary, valid labels of
+    every kind, and the same draw for the same seed."""
+    spec = di.WORKLOADS["dec_s128_k26_v126464"].scaled(n_units=40, vocab=5000, ids_high=4999)
+    a = di.make_case(spec, "cpu")
+    b = di.make_case(spec, "cpu")
+    e = a.extra
+    off, ids, kind, val = (e[k].numpy() for k in ("cand_off", "cand_ids", "kind", "val"))
+    assert off[0] == 0 and (np.diff(off) >= 2).all() and (np.diff(off) <= spec.k_max).all()
+    assert ids.min() >= 0 and ids.max() < spec.vocab
+    longest = int(np.argmax(np.diff(off)))
+    book = ids[off[longest]:off[longest + 1]]
+    for i in range(spec.n_units):
+        seg = ids[off[i]:off[i + 1]]
+        assert len(np.unique(seg)) == len(seg) and np.array_equal(seg, book[:len(seg)])
+        v = val[off[i]:off[i + 1]]
+        if kind[i] == di.HARD:
+            assert (v == 1).sum() == 1 and ((v == 0) | (v == 1)).all()
+        elif kind[i] == di.DIST:
+            assert (v >= 0).all() and abs(v.sum() - 1) < 1e-4
+        else:
+            assert (v == 1).sum() >= 1 and ((v == 0) | (v == 1)).all()
+    assert set(kind.tolist()) == {di.HARD, di.DIST, di.SET}
+    assert torch.equal(a.logits, b.logits) and torch.equal(a.extra["val"], b.extra["val"])
+    assert tuple(a.logits.shape) == (40, 5000)
