@@ -21,20 +21,18 @@
 // The work is a streaming pass over n_slots rows of V bf16 values, read
 // twice (the second time from L2) and written once: HBM-bound, a few tens
 // of MB per call.  A handful of rows cannot fill 148 SMs, so each row is
-// split over several CTAs by columns:
-//   1. k_dec_partial (splits x slots): (max, sum exp) of each split;
-//   2. k_dec_grad    (same grid): every CTA of a row merges that row's
-//      partials in split order into lse; warp 0 forms the restricted
-//      softmax, the targets, the terms and the K candidate gradients; the
-//      CTA writes its split of the gradient row (the dense part
-//      g w [full] Q P_v), then, after a CTA barrier, rewrites the candidate
-//      entries of its split with their full value;
-//   3. k_dec_reduce  (1 CTA): the mean over slots in a fixed order, double.
+// split over several CTAs by columns.  Fast path (16-byte aligned rows):
+//   1. k_dec_cluster (one cluster of 1-8 CTAs per slot): each CTA's
+//      (max, sum exp) of its split, exchanged through distributed shared
+//      memory, then the gradient of its split and the answer entries;
+//   2. k_dec_reduce  (1 CTA): the mean over slots in a fixed order, double,
+//      and the status word.
+// General path (any row stride or alignment): k_dec_partial (per-split
+// partials to the workspace), k_dec_grad (every CTA of a row merges them and
+// writes its split), k_dec_reduce.
 // Invalid slots (an answer id outside [0, V), repeated answer ids, K outside
 // 1..128, a malformed label) set a status bit and contribute a zero loss
 // and a zero gradient row.
-#include <mutex>
-
 #include "dlm_device.cuh"
 #include "dlm_host.h"
 
@@ -381,22 +379,29 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_grad(DecParams P) {
     }
 }
 
-// Fast path: one thread-block cluster per slot, one CTA per split of the
-// row (cluster rank = split).  Each CTA brings its split of the row into
-// shared memory once (bulk copies from HBM, one mbarrier per 8 KB piece, so
-// the sums start on the first piece), forms its (max, sum exp), and the
-// cluster exchanges only those two floats through distributed shared
-// memory: every CTA merges the n_split partials in rank order into the
-// same lse.  The gradient of the split is then written from shared memory
-// -- the row is read from HBM exactly once and never from L2 again -- and
-// the answer-token entries rewritten as in k_dec_grad.  The second cluster
-// barrier keeps every CTA's partial alive until all peers have read it.
-constexpr int kDecPieceBytes = 8192;
-constexpr int kDecMaxPieces = 16;     // slices up to 128 KB (65,536 columns)
+// 16-byte read-only load with an L2 cache policy.
+__device__ __forceinline__ uint4 ldg_v4_hint(const void* p, uint64_t pol) {
+    uint4 r;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p), "l"(pol));
+    return r;
+}
 
-__global__ void __launch_bounds__(kDecThreads, 6) k_dec_cluster(DecParams P) {
-    extern __shared__ __align__(128) uint8_t dsm[];
-    __shared__ __align__(8) uint64_t bars[kDecMaxPieces];
+// Fast path: one thread-block cluster per slot, one CTA per split of the
+// row (cluster rank = split; 1, 2, 4 or 8 splits).  Each CTA reads its split
+// twice: the first time from HBM, kept in L2 with an evict_last policy (a
+// call's label rows are tens of MB), for its (max, sum exp); the cluster
+// exchanges only those two floats through distributed shared memory and
+// every CTA merges the n_split partials in rank order into the same lse; the
+// second read comes from L2 and writes the gradient, then the answer-token
+// entries are rewritten as in k_dec_grad.  One warp works out the label
+// meanwhile.  The CTAs hold nothing but a few KB of shared memory, so every
+// cluster of a call is resident at once and no CTA waits for a second wave
+// (holding each split in shared memory instead measured slower: the call's
+// rows do not fit on chip at once).  The final cluster barrier keeps every
+// CTA's partial alive until all peers have read it.
+__global__ void __launch_bounds__(kDecThreads, 4) k_dec_cluster(DecParams P) {
+    constexpr int kU = 4;              // 16-byte loads in flight per thread
     __shared__ __align__(8) float2 s_part;
     __shared__ float sm_m[kDecThreads / 32], sm_s[kDecThreads / 32];
     __shared__ DecSlot S;
@@ -405,39 +410,25 @@ __global__ void __launch_bounds__(kDecThreads, 6) k_dec_cluster(DecParams P) {
     const int split = int(cluster_ctarank()), slot = blockIdx.y;
     const int c0 = split * P.chunk;
     const int c1 = min(c0 + P.chunk, P.vocab);
-    const int nvec = c1 > c0 ? (c1 - c0) / 8 : 0;                 // the host gives vocab % 8 == 0
-    const uint32_t bytes = uint32_t(nvec) * 16u;
-    const int pieces = int((bytes + kDecPieceBytes - 1) / kDecPieceBytes);
+    const int nvec = c1 > c0 ? (c1 - c0) / 8 : 0;
     const uint16_t* x = P.logits + slot_row(P, slot) * P.ld;
-    if (tid == 0) {
-        for (int i = 0; i < pieces; ++i) mbar_init(smem_addr(&bars[i]), 1);
-        fence_mbar_init_cluster();
-    }
-    __syncthreads();
-    pdl_wait();                        // the previous call may still read the outputs
+    const uint4* xv = reinterpret_cast<const uint4*>(x + c0);
+    pdl_wait();
     pdl_launch_dependents();
-    if (tid == 0) {
-        const uint64_t pol = policy_evict_first();   // read once
-        for (int i = 0; i < pieces; ++i) {
-            const uint32_t off = uint32_t(i) * kDecPieceBytes;
-            const uint32_t n = bytes - off < uint32_t(kDecPieceBytes) ? bytes - off : uint32_t(kDecPieceBytes);
-            const uint32_t b = smem_addr(&bars[i]);
-            mbar_arrive_expect_tx(b, n);
-            bulk_g2s_hint(smem_addr(dsm) + off, reinterpret_cast<const uint8_t*>(x + c0) + off, n, b, pol);
-        }
-    }
-    // while the row lands: the answers and the label (one warp)
-    if (tid < 32) dec_slot_prepare(P, slot, x, tid, S);
-    const uint4* sv = reinterpret_cast<const uint4*>(dsm);
-    constexpr int kPieceVec = kDecPieceBytes / 16;
+    const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
     float m = -INFINITY, s = 0.f;
-    bool ok = true;
-    for (int i = 0; i < pieces; ++i) {
-        ok = ok && mbar_wait_bounded<false>(smem_addr(&bars[i]), 0, nullptr);
-        if (!ok) break;                  // the copy never landed: reported in this CTA's error word
-        const int v1 = min(nvec, (i + 1) * kPieceVec);
-        for (int v = i * kPieceVec + tid; v < v1; v += kDecThreads) acc_vec(sv[v], m, s);
+    {
+        int i = tid;
+        for (; i + (kU - 1) * kDecThreads < nvec; i += kU * kDecThreads) {
+            uint4 r[kU];
+            #pragma unroll
+            for (int u = 0; u < kU; ++u) r[u] = ldg_v4_hint(xv + i + u * kDecThreads, keep);
+            #pragma unroll
+            for (int u = 0; u < kU; ++u) acc_vec(r[u], m, s);
+        }
+        for (; i < nvec; i += kDecThreads) acc_vec(ldg_v4_hint(xv + i, keep), m, s);
     }
+    if (tid < 32) dec_slot_prepare(P, slot, x, tid, S);
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
@@ -447,52 +438,65 @@ __global__ void __launch_bounds__(kDecThreads, 6) k_dec_cluster(DecParams P) {
     if (lane == 0) { sm_m[tid >> 5] = m; sm_s[tid >> 5] = s; }
     __syncthreads();
     if (tid == 0) {
-        float M = sm_m[0], S = sm_s[0];
-        for (int k = 1; k < kDecThreads / 32; ++k) lse_merge(M, S, sm_m[k], sm_s[k]);
-        s_part = make_float2(M, S);
+        float M = sm_m[0], Ssum = sm_s[0];
+        for (int k = 1; k < kDecThreads / 32; ++k) lse_merge(M, Ssum, sm_m[k], sm_s[k]);
+        s_part = make_float2(M, Ssum);
     }
-    cluster_sync_all();                // every split's partial is published
+    cluster_sync_all();
     if (tid == 0) {
-        float M = -INFINITY, S = 0.f;
+        float M = -INFINITY, Ssum = 0.f;
         for (int r = 0; r < P.n_split; ++r) {
             float pm, ps;
             const uint32_t a = mapa_shared(smem_addr(&s_part), uint32_t(r));
             asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(pm), "=f"(ps) : "r"(a) : "memory");
-            lse_merge(M, S, pm, ps);
+            lse_merge(M, Ssum, pm, ps);
         }
-        s_lse = M + logf(S);
+        s_lse = M + logf(Ssum);
     }
     __syncthreads();
     const float lse = s_lse;
     if (tid < 32) dec_slot_finish(P, slot, split, lse, tid, S);
-    // this CTA's error word (every CTA writes its own, every call; the
-    // reduction kernel ors them into the status word)
-    const int all_ok = __syncthreads_and(ok ? 1 : 0);
-    if (tid == 0)
-        P.err[int64_t(slot) * P.n_split + split] = (all_ok ? 0u : DLM_DEV_WAIT_TIMEOUT) | (split == 0 ? S.bad : 0u);
-    const float coef = all_ok ? S.coef : 0.f;
+    __syncthreads();
+    if (tid == 0) P.err[int64_t(slot) * P.n_split + split] = split == 0 ? S.bad : 0u;
+    const float coef = S.coef;
     const float sh = lse * kDecLog2e;
     uint16_t* out = P.dlogits + int64_t(slot) * P.ld_out;
     uint4* ov = reinterpret_cast<uint4*>(out + c0);
-    const uint64_t ef = policy_evict_first();
-    for (int v = tid; v < nvec; v += kDecThreads) {
-        if (!all_ok) { st_global_v4_hint(ov + v, make_uint4(0u, 0u, 0u, 0u), ef); continue; }
-        const uint4 rv = sv[v];
-        const uint32_t w4[4] = {rv.x, rv.y, rv.z, rv.w};
-        uint32_t o4[4];
-        #pragma unroll
-        for (int k = 0; k < 4; ++k)
-            o4[k] = pack_bf16x2(coef * ex2(fmaf(bf16lo(w4[k]), kDecLog2e, -sh)),
-                                coef * ex2(fmaf(bf16hi(w4[k]), kDecLog2e, -sh)));
-        st_global_v4_hint(ov + v, make_uint4(o4[0], o4[1], o4[2], o4[3]), ef);
+    {
+        int i = tid;
+        for (; i + (kU - 1) * kDecThreads < nvec; i += kU * kDecThreads) {
+            uint4 r[kU];
+            #pragma unroll
+            for (int u = 0; u < kU; ++u) r[u] = ldg_v4_hint(xv + i + u * kDecThreads, drop);
+            #pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const uint32_t w4[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+                uint32_t o4[4];
+                #pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    o4[k] = pack_bf16x2(coef * ex2(fmaf(bf16lo(w4[k]), kDecLog2e, -sh)),
+                                        coef * ex2(fmaf(bf16hi(w4[k]), kDecLog2e, -sh)));
+                st_global_v4_hint(ov + i + u * kDecThreads, make_uint4(o4[0], o4[1], o4[2], o4[3]), drop);
+            }
+        }
+        for (; i < nvec; i += kDecThreads) {
+            const uint4 rv = ldg_v4_hint(xv + i, drop);
+            const uint32_t w4[4] = {rv.x, rv.y, rv.z, rv.w};
+            uint32_t o4[4];
+            #pragma unroll
+            for (int k = 0; k < 4; ++k)
+                o4[k] = pack_bf16x2(coef * ex2(fmaf(bf16lo(w4[k]), kDecLog2e, -sh)),
+                                    coef * ex2(fmaf(bf16hi(w4[k]), kDecLog2e, -sh)));
+            st_global_v4_hint(ov + i, make_uint4(o4[0], o4[1], o4[2], o4[3]), drop);
+        }
     }
-    __syncthreads();                   // the dense stores of this CTA come first
-    const int K = all_ok ? S.K : 0;
+    __syncthreads();
+    const int K = S.K;
     for (int k = tid; k < K; k += kDecThreads) {
         const int id = S.id[k];
         if (id >= c0 && id < c1) out[id] = __bfloat16_as_ushort(__float2bfloat16_rn(S.g[k]));
     }
-    cluster_sync_all();                // no CTA leaves while a peer may read its partial
+    cluster_sync_all();
 }
 
 constexpr int kDecRedThreads = 256;
@@ -533,22 +537,17 @@ struct DecPlan {
 };
 
 // The cluster path: n_split in {1, 2, 4, 8} (a portable cluster size), the
-// smallest that keeps a slice within 64 KB of shared memory and, below 8,
-// gives about four CTAs per SM (592) without cutting slices under 2,048
-// columns.  Returns false when the row does not fit (the three-kernel path
-// runs instead).
+// smallest that gives about 512 CTAs in all (3.5 per SM, every cluster
+// resident at once) without cutting splits under 2,048 columns.  Needs
+// vocab % 8 == 0 (16-byte vectors).
 inline bool dec_cluster_plan(int n_slots, int vocab, int& n_split, int& chunk) {
     if (n_slots <= 0 || vocab % 8 != 0) return false;
-    const int64_t want = (4 * 148 + n_slots - 1) / n_slots;   // CTAs wanted per slot
-    for (int ns = 1; ns <= 8; ns *= 2) {
-        const int64_t ch = (int64_t(vocab) / 8 + ns - 1) / ns * 8;
-        if (ch * 2 > 65536) continue;                          // slice too large
-        if (ns < 8 && ns < want && ch >= 2 * 2048) continue;   // more CTAs wanted, and slices can shrink
-        n_split = ns;
-        chunk = int(ch);
-        return true;
-    }
-    return false;
+    const int64_t want = (512 + n_slots - 1) / n_slots;   // CTAs wanted per slot
+    int ns = 1;
+    while (ns < 8 && ns < want && int64_t(vocab) / (2 * ns) >= 2048) ns *= 2;
+    n_split = ns;
+    chunk = int((int64_t(vocab) / 8 + ns - 1) / ns * 8);
+    return true;
 }
 
 // Columns of a row per CTA: enough CTAs for two waves over 148 SMs, at
@@ -633,29 +632,15 @@ extern "C" dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_
     P.vec = (ld % 8 == 0) && (ld_out % 8 == 0) && aligned16(logits) && aligned16(dlogits);
     int cl_split = 0, cl_chunk = 0;
     if (n_slots > 0 && P.vec && dec_cluster_plan(n_slots, vocab, cl_split, cl_chunk)) {
-        // one cluster per slot: the row read once, lse partials through DSMEM
+        // one cluster per slot: lse partials through distributed shared memory
         P.err = reinterpret_cast<uint32_t*>(ws + plan.partial_off);   // n_slots x cl_split words fit
         DecParams C = P;
         C.n_split = cl_split;
         C.chunk = cl_chunk;
-        const size_t smem = size_t(cl_chunk) * 2;
-        static std::mutex mu;
-        static bool attr_done[64] = {};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        {
-            std::lock_guard<std::mutex> lk(mu);
-            if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-                const cudaError_t e = cudaFuncSetAttribute(k_dec_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                           65536);
-                if (e != cudaSuccess) { cudaGetLastError(); return cuda_status(e, "k_dec_cluster smem attribute"); }
-                attr_done[dev] = true;
-            }
-        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(unsigned(cl_split), unsigned(n_slots));
         cfg.blockDim = dim3(kDecThreads);
-        cfg.dynamicSmemBytes = smem;
+        cfg.dynamicSmemBytes = 0;
         cfg.stream = s;
         cudaLaunchAttribute at[2];
         at[0].id = cudaLaunchAttributeClusterDimension;

@@ -7,8 +7,7 @@ question, a slot-row indirection, every label_softmax setting, smoothing,
 and slots whose labels the kernel must refuse.
 
 Both kernel paths are covered: the cluster path (one cluster of CTAs per
-slot holds the row in shared memory; aligned rows up to 262,144 columns)
-and the three-kernel path (any shape).
+slot, 16-byte aligned rows) and the three-kernel path (any row stride).
 
 Gradient bar: entries away from the answer tokens are g w Q P_v, one
 product rounded to bf16 -- the gradient bar of the other losses (2e-3
@@ -110,7 +109,7 @@ def test_decision_full_workload(label_softmax):
     (5, 126464, 2, 26, 0, 1),     # few slots: clusters of 8 CTAs per row
     (300, 2048, 2, 8, 0, 2),      # many slots, one CTA per row
     (3, 16, 16, 16, 0, 3),        # every token of the vocabulary an answer
-    (4, 300000, 2, 26, 0, 4),     # a row too long for a cluster's shared memory: three kernels, 16-byte loads
+    (4, 300000, 2, 26, 0, 4),     # long rows: clusters of 8 CTAs of 37,500 columns
 ])
 def test_decision_elementwise(n, V, kmin, kmax, ld_pad, seed):
     off, ids, kind, val = _batch(seed, n, V, kmax, kmin=kmin)
