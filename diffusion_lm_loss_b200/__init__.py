@@ -166,8 +166,8 @@ def lib():
     L.dlm_decision_workspace_size.restype = sz
     L.dlm_decision_workspace_size.argtypes = [i32, i32]
     L.dlm_decision_loss_fwd_bwd.restype = ctypes.c_int
-    L.dlm_decision_loss_fwd_bwd.argtypes = [i32, vp, i64, i32, vp, vp, vp, vp, vp, i32, f32, f32, f32, vp, vp,
-                                            vp, i64, vp, sz, vp]
+    L.dlm_decision_loss_fwd_bwd.argtypes = [i32, vp, i64, i64, i32, vp, vp, i64, vp, vp, vp, i32, f32, f32, f32, vp,
+                                            vp, vp, i64, vp, sz, vp]
     L.dlm_scale_bf16.restype = ctypes.c_int
     L.dlm_scale_bf16.argtypes = [vp, i64, i64, i64, vp, vp]
     L.dlm_test_skip_device_check.restype = ctypes.c_int
@@ -525,8 +525,9 @@ def decision_loss_fwd_bwd(logits: torch.Tensor, vocab: int, cand_off: torch.Tens
     """Typed-decision losses at label slots (see dlm_decision_loss_fwd_bwd).
     logits: bf16 [rows, ld]; slot i reads row slot_rows[i] (int64), or row i
     when slot_rows is None.  cand_off int32 [n_slots + 1]; cand_ids int32 and
-    label_val float32 [cand_off[-1]] (the offsets are on the device: the
-    caller keeps them within these arrays); label_kind int32 [n_slots]."""
+    label_val float32 of the same length; label_kind int32 [n_slots].  Rows
+    and offsets that leave these arrays (device data) are refused by the
+    kernels (DEV_BAD_LAYOUT)."""
     n = int(cand_off.numel()) - 1
     if n < 0:
         raise ValueError("cand_off: needs n_slots + 1 entries")
@@ -554,7 +555,8 @@ def decision_loss_fwd_bwd(logits: torch.Tensor, vocab: int, cand_off: torch.Tens
                           torch.empty((n, vocab), dtype=torch.bfloat16, device=dev),
                           _aligned_workspace(decision_workspace_size(n, vocab), dev, 256))
     _ok(lib().dlm_decision_loss_fwd_bwd(
-        n, _ptr(logits), logits.stride(0), vocab, _ptr(slot_rows), _ptr(cand_off), _ptr(cand_ids),
+        n, _ptr(logits), max(int(logits.shape[0]), 1), logits.stride(0), vocab, _ptr(slot_rows), _ptr(cand_off),
+        int(cand_ids.numel()), _ptr(cand_ids),
         _ptr(label_kind), _ptr(label_val), label_softmax, brier_weight, hard_label_smoothing, grad_scale,
         _ptr(out.loss), _ptr(out.slot_loss), _ptr(out.dlogits), out.dlogits.stride(0), _ptr(out.workspace),
         out.workspace.numel(), _stream()), "dlm_decision_loss_fwd_bwd")

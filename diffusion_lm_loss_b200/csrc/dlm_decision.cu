@@ -30,9 +30,9 @@
 // General path (any row stride or alignment): k_dec_partial (per-split
 // partials to the workspace), k_dec_grad (every CTA of a row merges them and
 // writes its split), k_dec_reduce.
-// Invalid slots (an answer id outside [0, V), repeated answer ids, K outside
-// 1..128, a malformed label) set a status bit and contribute a zero loss
-// and a zero gradient row.
+// Invalid slots (a row or answer offsets outside the given arrays, an answer
+// id outside [0, V), repeated answer ids, K outside 1..128, a malformed
+// label) set a status bit and contribute a zero loss and a zero gradient row.
 #include "dlm_device.cuh"
 #include "dlm_host.h"
 
@@ -47,7 +47,9 @@ struct DecParams {
     int64_t ld;
     int vocab;
     const int64_t* slot_rows;          // logits row of each slot, or null (row = slot)
+    int64_t n_rows;                    // rows of the logits tensor
     const int32_t* cand_off;           // [n_slots + 1]
+    int64_t n_cands;                   // entries of cand_ids and val
     const int32_t* cand_ids;           // answer token ids
     const int32_t* kind;               // [n_slots] DLM_LABEL_*
     const float* val;                  // one value per answer (see dlm.h)
@@ -95,8 +97,14 @@ __device__ __forceinline__ void acc_vec(uint4 r, float& m, float& s) {
     }
 }
 
-__device__ __forceinline__ int64_t slot_row(const DecParams& P, int slot) {
-    return P.slot_rows ? P.slot_rows[slot] : int64_t(slot);
+// The logits row of `slot` and whether it lies inside the logits tensor
+// (slot_rows is device data the host cannot check); an invalid row reads
+// row 0 instead, harmlessly, and the slot is refused.
+__device__ __forceinline__ bool slot_row_ok(const DecParams& P, int slot, int64_t& row) {
+    row = P.slot_rows ? P.slot_rows[slot] : int64_t(slot);
+    const bool ok = row >= 0 && row < P.n_rows;
+    if (!ok) row = 0;
+    return ok;
 }
 
 __global__ void __launch_bounds__(kDecThreads) k_dec_partial(DecParams P) {
@@ -105,7 +113,9 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_partial(DecParams P) {
     pdl_wait();                        // the previous call may still read the workspace
     pdl_launch_dependents();
     if (split == 0 && slot == 0 && tid == 0) *P.status = 0u;
-    const uint16_t* x = P.logits + slot_row(P, slot) * P.ld;
+    int64_t row;
+    slot_row_ok(P, slot, row);
+    const uint16_t* x = P.logits + row * P.ld;
     const int c0 = split * P.chunk;
     const int c1 = min(c0 + P.chunk, P.vocab);
     float m = -INFINITY, s = 0.f;
@@ -173,13 +183,16 @@ struct DecSlot {
 // label -- validity, the restricted softmax, the targets, CE_res, Brier and
 // the restricted + Brier part of each answer's gradient.  Needs only the K
 // answer logits, so it runs while the row itself is still being loaded.
-__device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, const uint16_t* x, int lane,
-                                                 DecSlot& S) {
+__device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, const uint16_t* x, bool row_ok,
+                                                 int lane, DecSlot& S) {
     const int o0 = P.cand_off[slot], o1 = P.cand_off[slot + 1];
     const int K = o1 - o0;
     const int kind = P.kind[slot];
-    int bad = (K < 1 || K > DLM_DECISION_MAX_ANSWERS) ? 2 : 0;
-    bad |= (kind != DLM_LABEL_HARD && kind != DLM_LABEL_DIST && kind != DLM_LABEL_SET) ? 2 : 0;
+    // 3: the slot's row or its answer offsets lie outside the given arrays;
+    // 2: a malformed label; 1: an answer id outside the vocabulary
+    int bad = (!row_ok || o0 < 0 || o1 < o0 || int64_t(o1) > P.n_cands) ? 3 : 0;
+    if (!bad) bad = (K < 1 || K > DLM_DECISION_MAX_ANSWERS) ? 2 : 0;
+    if (!bad) bad = (kind != DLM_LABEL_HARD && kind != DLM_LABEL_DIST && kind != DLM_LABEL_SET) ? 2 : 0;
     float z[4], v[4];
     int id[4];
     int n_one = 0, n_other = 0;    // label checks: values equal to 1, and not in {0, 1}
@@ -273,7 +286,7 @@ __device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, c
     }
     if (lane == 0) {
         S.K = bad ? 0 : K;
-        S.bad = bad == 0 ? 0u : (bad == 1 ? DLM_DEV_BAD_TOKEN_ID : DLM_DEV_BAD_LABEL);
+        S.bad = bad == 0 ? 0u : bad == 1 ? DLM_DEV_BAD_TOKEN_ID : bad == 2 ? DLM_DEV_BAD_LABEL : DLM_DEV_BAD_LAYOUT;
     }
 }
 
@@ -308,7 +321,9 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_grad(DecParams P) {
     const int split = blockIdx.x, slot = blockIdx.y, tid = threadIdx.x;
     pdl_wait();                        // partials of k_dec_partial
     pdl_launch_dependents();
-    const uint16_t* x = P.logits + slot_row(P, slot) * P.ld;
+    int64_t row;
+    const bool row_ok = slot_row_ok(P, slot, row);
+    const uint16_t* x = P.logits + row * P.ld;
     if (tid == 0) {
         float M = -INFINITY, S = 0.f;
         for (int k = 0; k < P.n_split; ++k) {
@@ -320,7 +335,7 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_grad(DecParams P) {
     __syncthreads();
     const float lse = s_lse;
     if (tid < 32) {
-        dec_slot_prepare(P, slot, x, tid, S);
+        dec_slot_prepare(P, slot, x, row_ok, tid, S);
         __syncwarp();
         dec_slot_finish(P, slot, split, lse, tid, S);
     }
@@ -411,10 +426,12 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_dec_cluster(DecParams P) {
     const int c0 = split * P.chunk;
     const int c1 = min(c0 + P.chunk, P.vocab);
     const int nvec = c1 > c0 ? (c1 - c0) / 8 : 0;
-    const uint16_t* x = P.logits + slot_row(P, slot) * P.ld;
-    const uint4* xv = reinterpret_cast<const uint4*>(x + c0);
-    pdl_wait();
+    pdl_wait();                        // inputs may come from the previous kernel
     pdl_launch_dependents();
+    int64_t row;
+    const bool row_ok = slot_row_ok(P, slot, row);
+    const uint16_t* x = P.logits + row * P.ld;
+    const uint4* xv = reinterpret_cast<const uint4*>(x + c0);
     const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
     float m = -INFINITY, s = 0.f;
     {
@@ -428,7 +445,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_dec_cluster(DecParams P) {
         }
         for (; i < nvec; i += kDecThreads) acc_vec(ldg_v4_hint(xv + i, keep), m, s);
     }
-    if (tid < 32) dec_slot_prepare(P, slot, x, tid, S);
+    if (tid < 32) dec_slot_prepare(P, slot, x, row_ok, tid, S);
     #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
@@ -578,9 +595,9 @@ extern "C" size_t dlm_decision_workspace_size(int32_t n_slots, int32_t vocab) {
     return dec_plan(n_slots, vocab).total;
 }
 
-extern "C" dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_t* logits, int64_t ld,
-                                                  int32_t vocab, const int64_t* slot_rows,
-                                                  const int32_t* cand_off, const int32_t* cand_ids,
+extern "C" dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_t* logits, int64_t n_rows,
+                                                  int64_t ld, int32_t vocab, const int64_t* slot_rows,
+                                                  const int32_t* cand_off, int64_t n_cands, const int32_t* cand_ids,
                                                   const int32_t* label_kind, const float* label_val,
                                                   int32_t label_softmax, float brier_weight,
                                                   float hard_label_smoothing, float grad_scale, float* loss,
@@ -597,7 +614,8 @@ extern "C" dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_
     if (!loss || !workspace) return DLM_ERR_INVALID_ARGUMENT;
     if (n_slots > 0 && (!logits || !cand_off || !cand_ids || !label_kind || !label_val || !dlogits))
         return DLM_ERR_INVALID_ARGUMENT;
-    if (n_slots > 0 && (ld < vocab || ld_out < vocab)) return DLM_ERR_INVALID_ARGUMENT;
+    if (n_slots > 0 && (ld < vocab || ld_out < vocab || n_rows < 1 || n_cands < 0)) return DLM_ERR_INVALID_ARGUMENT;
+    if (n_slots > 0 && !slot_rows && n_rows < n_slots) return DLM_ERR_INVALID_ARGUMENT;
     if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign) return DLM_ERR_INVALID_ARGUMENT;
     const DecPlan plan = dec_plan(n_slots, vocab);
     if (workspace_bytes < plan.total) return DLM_ERR_WORKSPACE_TOO_SMALL;
@@ -610,7 +628,9 @@ extern "C" dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_
     P.ld = ld;
     P.vocab = vocab;
     P.slot_rows = slot_rows;
+    P.n_rows = n_rows;
     P.cand_off = cand_off;
+    P.n_cands = n_cands;
     P.cand_ids = cand_ids;
     P.kind = label_kind;
     P.val = label_val;

@@ -438,12 +438,12 @@ DLM_API dlm_status_t dlm_selftest_bounded_wait(uint64_t limit_ns, uint32_t *dev_
  *   DLM_LABEL_SET:  val = 1 for each allowed answer, 0 elsewhere (at least
  *       one 1).  q = y = val / (number of allowed answers).
  * Arguments (device pointers unless stated):
- *   logits [rows, ld] bf16; slot_rows [n_slots] int64: the logits row of
+ *   logits [n_rows, ld] bf16; slot_rows [n_slots] int64: the logits row of
  *       each slot, or NULL for row i = slot i (logits computed at the label
- *       slots only).  ld >= vocab.
+ *       slots only; then n_rows >= n_slots).  ld >= vocab.
  *   cand_off [n_slots + 1] int32 (offsets into cand_ids and label_val,
- *       non-decreasing from 0), cand_ids int32 answer token ids,
- *       label_kind [n_slots] int32, label_val float.
+ *       non-decreasing, within 0..n_cands), cand_ids [n_cands] int32 answer
+ *       token ids, label_kind [n_slots] int32, label_val [n_cands] float.
  *   grad_scale g: the gradient written is g * d loss / d z.
  *   loss [1] float (written); slot_loss [n_slots] float: each slot's
  *       contribution (its terms / n_slots; sums to loss), or NULL.
@@ -453,12 +453,15 @@ DLM_API dlm_status_t dlm_selftest_bounded_wait(uint64_t limit_ns, uint32_t *dev_
  *       256-byte aligned; its status word is read by dlm_get_device_status.
  * Errors: n_slots outside 0..DLM_DECISION_MAX_SLOTS, vocab <= 0, a bad
  * label_softmax, a negative or non-finite brier_weight, smoothing outside
- * [0, 1], a null pointer or ld / ld_out < vocab return
- * DLM_ERR_INVALID_ARGUMENT before anything is enqueued.  On the device, a
- * slot whose answer id is outside [0, vocab) sets DLM_DEV_BAD_TOKEN_ID; K
- * outside 1..128, repeated answer ids, an unknown kind or a malformed label
- * set DLM_DEV_BAD_LABEL; such a slot adds 0 to the loss (the mean still
- * divides by n_slots) and its dlogits row is all zeros.  n_slots = 0 writes
+ * [0, 1], a null pointer, ld / ld_out < vocab, n_rows < 1 (or < n_slots
+ * without slot_rows) or n_cands < 0 return DLM_ERR_INVALID_ARGUMENT before
+ * anything is enqueued.  On the device, a slot whose row is outside
+ * [0, n_rows) or whose answer offsets leave 0..n_cands sets
+ * DLM_DEV_BAD_LAYOUT; an answer id outside [0, vocab) sets
+ * DLM_DEV_BAD_TOKEN_ID; K outside 1..128, repeated answer ids, an unknown
+ * kind or a malformed label set DLM_DEV_BAD_LABEL; such a slot adds 0 to the
+ * loss (the mean still divides by n_slots) and its dlogits row is all
+ * zeros.  n_slots = 0 writes
  * loss = 0.  The 16-byte load path needs ld and ld_out multiples of 8 and
  * 16-byte aligned logits and dlogits; other shapes take a scalar path.
  * Not built: full_ce_weighting: dft (the page gives no formula).
@@ -474,9 +477,9 @@ DLM_API dlm_status_t dlm_selftest_bounded_wait(uint64_t limit_ns, uint32_t *dev_
 
 DLM_API size_t dlm_decision_workspace_size(int32_t n_slots, int32_t vocab);
 
-DLM_API dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_t *logits, int64_t ld,
-                                       int32_t vocab, const int64_t *slot_rows,
-                                       const int32_t *cand_off, const int32_t *cand_ids,
+DLM_API dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_t *logits, int64_t n_rows,
+                                       int64_t ld, int32_t vocab, const int64_t *slot_rows,
+                                       const int32_t *cand_off, int64_t n_cands, const int32_t *cand_ids,
                                        const int32_t *label_kind, const float *label_val,
                                        int32_t label_softmax, float brier_weight,
                                        float hard_label_smoothing, float grad_scale, float *loss,

@@ -202,3 +202,35 @@ def test_decision_no_slots_and_reproducible():
     torch.cuda.synchronize()
     assert a.loss.item() == b.loss.item()
     assert torch.equal(a.dlogits.view(torch.int16), b.dlogits.view(torch.int16))
+
+
+def test_decision_rows_and_offsets_outside_their_arrays_are_refused():
+    """A slot row outside the logits tensor, and answer offsets that leave
+    the answer arrays (device data the host cannot check): DEV_BAD_LAYOUT,
+    those slots skipped, the others unaffected -- on both kernel paths."""
+    n, V = 10, 4096
+    off, ids, kind, val = _batch(6, n, V, 12, kmin=2)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(6)
+    for ld_pad in (0, 3):                       # the cluster path, then the three-kernel path
+        base = (torch.randn((16, V + ld_pad), generator=gen, device="cuda") * 2).to(torch.bfloat16)
+        logits = base[:, :V] if ld_pad else base
+        rows = np.arange(n, dtype=np.int64)
+        rows[3] = 16                            # one past the last row
+        bad_off = off.copy()
+        bad_off[8] = off[8] + 1000              # slot 7 ends and slot 8 starts beyond the answer arrays
+        out = dlm.decision_loss_fwd_bwd(logits, V, *_dev(bad_off, ids, kind, val),
+                                        slot_rows=torch.from_numpy(rows).cuda())
+        torch.cuda.synchronize()
+        st = out.device_status()
+        assert st & dlm.DEV_BAD_LAYOUT, st
+        g = out.dlogits.float().cpu()
+        sl = out.slot_loss.cpu().numpy()[:n]
+        for s_ in (3, 7, 8):
+            assert sl[s_] == 0.0 and bool((g[s_] == 0).all())
+        keep = np.array([i for i in range(n) if i not in (3, 7, 8)])
+        ref = oracle.decision_loss(di.bf16_bits(logits), V, rows[keep],
+                                   np.concatenate([[0], np.cumsum(np.diff(off)[keep])]),
+                                   np.concatenate([ids[off[i]:off[i + 1]] for i in keep]), kind[keep],
+                                   np.concatenate([val[off[i]:off[i + 1]] for i in keep]))
+        assert_loss_close(float(out.loss.item()), ref["loss"] * len(keep) / n)
