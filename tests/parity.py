@@ -94,18 +94,31 @@ def product_rms_scale(a: np.ndarray, b: np.ndarray, transpose_a: bool = False,
     return np.sqrt(out)
 
 
-def assert_bf16_sum_close(gpu: np.ndarray, exact: np.ndarray, scale: np.ndarray, what: str):
+def assert_bf16_sum_close(gpu: np.ndarray, exact: np.ndarray, scale: np.ndarray, what: str,
+                          block_rows: int = 8192):
     """Element-wise bar for a bf16 sum of products whose one operand was
     rounded to bf16 (see the module docstring); `scale` = product_rms_scale
-    of that sum.  Also returns the relative Frobenius error, for reports."""
-    gpu = np.asarray(gpu, np.float64)
-    exact = np.asarray(exact, np.float64)
+    of that sum.  Compared in blocks of rows (full-size gradients are
+    gigabytes).  Returns the relative Frobenius error, for reports."""
     assert gpu.shape == exact.shape == scale.shape, (gpu.shape, exact.shape, scale.shape)
-    err = np.abs(gpu - exact)
-    tol = bf16_ulp(np.maximum(np.abs(gpu), np.abs(exact))) + SUM_SIGMAS * BF16_U * scale
-    bad = err > tol
-    if bad.any():
-        i = np.unravel_index(int(np.argmax(err - tol)), err.shape)
-        raise AssertionError(f"{what}: {int(bad.sum())} of {err.size} elements out of tolerance; worst at {i}: "
-                             f"gpu {gpu[i]!r} exact {exact[i]!r} tol {tol[i]:.3e}")
-    return float(np.linalg.norm(gpu - exact) / max(np.linalg.norm(exact), 1e-300))
+    n_bad = 0
+    worst = None
+    d2 = e2 = 0.0
+    for r0 in range(0, gpu.shape[0], block_rows):
+        g = np.asarray(gpu[r0:r0 + block_rows], np.float64)
+        e = np.asarray(exact[r0:r0 + block_rows], np.float64)
+        err = np.abs(g - e)
+        tol = bf16_ulp(np.maximum(np.abs(g), np.abs(e))) + SUM_SIGMAS * BF16_U * scale[r0:r0 + block_rows]
+        bad = err > tol
+        d2 += float(np.square(err).sum())
+        e2 += float(np.square(e).sum())
+        if bad.any():
+            n_bad += int(bad.sum())
+            i = np.unravel_index(int(np.argmax(err - tol)), err.shape)
+            cand = (float((err - tol)[i]), (i[0] + r0,) + tuple(i[1:]), g[i], e[i], float(tol[i]))
+            worst = cand if worst is None or cand[0] > worst[0] else worst
+    if n_bad:
+        _, i, gv, ev, tv = worst
+        raise AssertionError(f"{what}: {n_bad} of {gpu.size} elements out of tolerance; worst at {i}: "
+                             f"gpu {gv!r} exact {ev!r} tol {tv:.3e}")
+    return float(np.sqrt(d2) / max(np.sqrt(e2), 1e-300))
