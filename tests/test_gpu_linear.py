@@ -31,9 +31,10 @@ def _cuda():
     dlm.lib()
 
 
-def _host_f64(t):
-    """A bf16 device tensor as a float64 numpy array (exact)."""
-    return t.detach().float().cpu().numpy().astype(np.float64)
+def _host_f32(t):
+    """A bf16 device tensor as a float32 numpy array (exact: every bf16
+    value is a float32 value; half the host memory of float64)."""
+    return t.detach().float().cpu().numpy()
 
 
 def assert_fused_grads(ref, W, terms, dW_gpu):
@@ -42,23 +43,23 @@ def assert_fused_grads(ref, W, terms, dW_gpu):
     [rows, D] device tensor, H [rows, D] device tensor, oracle key of dH,
     oracle key of the scored rows, oracle key of dZ).  Returns the relative
     Frobenius errors, for reports."""
-    Wd = _host_f64(W)
+    Wd = _host_f32(W)
     fro = {}
     s2_dw = None
     for name, g, H, k_dh, k_rows, k_dz in terms:
         rows, dZ = ref[k_rows], ref[k_dz]
-        gd = _host_f64(g)
+        gd = _host_f32(g)
         fro[name] = assert_bf16_sum_close(gd[rows], ref[k_dh][rows], product_rms_scale(dZ, Wd), name)
         un = np.ones(gd.shape[0], bool)
         un[rows] = False
         assert (gd[un] == 0).all(), f"{name}: nonzero rows where nothing is scored"
         del gd
         if dW_gpu is not None:
-            s = product_rms_scale(dZ, _host_f64(H)[rows], transpose_a=True)
+            s = product_rms_scale(dZ, _host_f32(H)[rows], transpose_a=True)
             s2_dw = s * s if s2_dw is None else s2_dw + s * s
             del s
     if dW_gpu is not None:
-        fro["dW"] = assert_bf16_sum_close(_host_f64(dW_gpu), ref["dW"], np.sqrt(s2_dw), "dW")
+        fro["dW"] = assert_bf16_sum_close(_host_f32(dW_gpu), ref["dW"], np.sqrt(s2_dw), "dW")
     return fro
 
 
