@@ -234,3 +234,44 @@ def test_decision_rows_and_offsets_outside_their_arrays_are_refused():
                                    np.concatenate([ids[off[i]:off[i + 1]] for i in keep]), kind[keep],
                                    np.concatenate([val[off[i]:off[i + 1]] for i in keep]))
         assert_loss_close(float(out.loss.item()), ref["loss"] * len(keep) / n)
+
+
+def test_decision_graph_replays_and_dirty_workspace():
+    """Nothing in the workspace needs zeroing between calls: a workspace
+    full of garbage, the same workspace reused by calls of another shape,
+    and a CUDA graph of the call replayed several times all give the direct
+    call's loss bit for bit and a clean status word."""
+    spec = di.WORKLOADS["dec_s128_k26_v126464"].scaled(n_units=40)
+    case = di.make_case(spec, "cuda")
+    e = case.extra
+    args = (case.logits, spec.vocab, e["cand_off"], e["cand_ids"], e["kind"], e["val"])
+    ref = dlm.decision_loss_fwd_bwd(*args)
+    torch.cuda.synchronize()
+    want = ref.loss.item()
+    # garbage in the whole workspace, the ticket included
+    ref.workspace.fill_(0xA5)
+    ref.loss.fill_(float("nan"))
+    again = dlm.decision_loss_fwd_bwd(*args, out=ref)
+    torch.cuda.synchronize()
+    assert again.loss.item() == want and again.device_status() == 0
+    # the same workspace between calls of another shape (other CTA counts)
+    small = di.WORKLOADS["dec_s128_k26_v126464"].scaled(n_units=7)
+    sc = di.make_case(small, "cuda", seed=9)
+    se = sc.extra
+    ws = ref.workspace
+    o2 = dlm.DecisionOut(torch.empty(1, device="cuda"), torch.empty(7, device="cuda"),
+                         torch.empty((7, small.vocab), dtype=torch.bfloat16, device="cuda"), ws)
+    s_ref = dlm.decision_loss_fwd_bwd(sc.logits, small.vocab, se["cand_off"], se["cand_ids"], se["kind"], se["val"])
+    dlm.decision_loss_fwd_bwd(sc.logits, small.vocab, se["cand_off"], se["cand_ids"], se["kind"], se["val"], out=o2)
+    again = dlm.decision_loss_fwd_bwd(*args, out=ref)
+    torch.cuda.synchronize()
+    assert o2.loss.item() == s_ref.loss.item() and again.loss.item() == want
+    # a graph of the call, replayed
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dlm.decision_loss_fwd_bwd(*args, out=ref)
+    for _ in range(3):
+        ref.loss.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        assert ref.loss.item() == want and ref.device_status() == 0
