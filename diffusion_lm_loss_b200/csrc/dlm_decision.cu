@@ -41,6 +41,7 @@ namespace dlm {
 constexpr int kDecThreads = 256;
 constexpr int kDecUnroll = 4;          // 16-byte loads in flight per thread
 constexpr float kDecLog2e = 1.4426950408889634f;
+constexpr float kDecLn2 = 0.6931471805599453f;
 
 struct DecParams {
     const uint16_t* logits;
@@ -78,23 +79,76 @@ __device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2
     m = M;
 }
 
+// Warp max of a float in one instruction (redux.sync .f32, sm_100a).
+__device__ __forceinline__ float warp_max_f32(float v) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+// Every lane's (m, s) merged over the warp: the warp max in one
+// instruction, each lane's sum rescaled to it, then a butterfly sum.
+// Every lane ends with the same bits (the butterfly's additions only swap
+// operands between lanes).  An all-empty warp (max -inf) gives (-inf, 0).
+__device__ __forceinline__ void warp_lse(float& m, float& s) {
+    const float M = warp_max_f32(m);
+    s = (M == -INFINITY) ? 0.f : s * ex2((m - M) * kDecLog2e);
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    m = M;
+}
+
 __device__ __forceinline__ void acc_value(float x, float& m, float& s) {
     if (x == -INFINITY) return;
     if (x > m) { s = s * ex2((m - x) * kDecLog2e); m = x; }   // s = 0 while m = -inf
     s += ex2((x - m) * kDecLog2e);
 }
 
-__device__ __forceinline__ void acc_vec(uint4 r, float& m, float& s) {
-    const float mx = bf16x8_max(r);
-    if (mx == -INFINITY) return;
-    if (mx > m) { s = s * ex2((m - mx) * kDecLog2e); m = mx; }
+// (max, sum exp) over N 16-byte vectors: one max and at most one rescale
+// per batch, the exponents by packed FMAs (two lanes per instruction) and
+// two ex2 per pair.  Once the batch max is folded in, m is finite, so a
+// -inf element gives ex2(-inf) = 0 with no test of its own.
+template <int N>
+__device__ __forceinline__ void acc_batch(const uint4 (&r)[N], float& m, float& s) {
+    float cm = bf16x8_max(r[0]);
+    #pragma unroll
+    for (int u = 1; u < N; ++u) cm = fmaxf(cm, bf16x8_max(r[u]));
+    if (cm == -INFINITY) return;
+    if (cm > m) { s = s * ex2((m - cm) * kDecLog2e); m = cm; }   // s = 0 while m = -inf
+    const uint64_t l2e = f2pack(kDecLog2e, kDecLog2e);
+    const uint64_t nmb = f2pack(-m * kDecLog2e, -m * kDecLog2e);
+    uint64_t acc = f2pack(0.f, 0.f);
+    #pragma unroll
+    for (int u = 0; u < N; ++u) {
+        const uint32_t w4[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float t0, t1;
+            f2unpack(f2fma(f2pack(bf16lo(w4[k]), bf16hi(w4[k])), l2e, nmb), t0, t1);
+            acc = f2add(acc, f2pack(ex2(t0), ex2(t1)));
+        }
+    }
+    float a0, a1;
+    f2unpack(acc, a0, a1);
+    s += a0 + a1;
+}
+
+// The dense gradient of one 16-byte vector: g = coef 2^(x log2e - lse log2e)
+// by packed FMAs; for coef > 0 the factor is folded into the exponent
+// (nlb = log2 coef - lse log2e), otherwise nlb = -lse log2e and each value
+// is multiplied by `mul` = coef.
+__device__ __forceinline__ uint4 dec_dense_vec(uint4 r, uint64_t l2e, uint64_t nlb, bool fold, float mul) {
     const uint32_t w4[4] = {r.x, r.y, r.z, r.w};
+    uint32_t o4[4];
     #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        const float lo = bf16lo(w4[k]), hi = bf16hi(w4[k]);
-        s += (lo == -INFINITY ? 0.f : ex2((lo - m) * kDecLog2e));
-        s += (hi == -INFINITY ? 0.f : ex2((hi - m) * kDecLog2e));
+        float t0, t1;
+        f2unpack(f2fma(f2pack(bf16lo(w4[k]), bf16hi(w4[k])), l2e, nlb), t0, t1);
+        float g0 = ex2(t0), g1 = ex2(t1);
+        if (!fold) { g0 *= mul; g1 *= mul; }
+        o4[k] = pack_bf16x2(g0, g1);
     }
+    return make_uint4(o4[0], o4[1], o4[2], o4[3]);
 }
 
 // The logits row of `slot` and whether it lies inside the logits tensor
@@ -128,10 +182,12 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_partial(DecParams P) {
             uint4 r[kDecUnroll];
             #pragma unroll
             for (int u = 0; u < kDecUnroll; ++u) r[u] = __ldg(xv + i + u * kDecThreads);
-            #pragma unroll
-            for (int u = 0; u < kDecUnroll; ++u) acc_vec(r[u], m, s);
+            acc_batch<kDecUnroll>(r, m, s);
         }
-        for (; i < nv; i += kDecThreads) acc_vec(__ldg(xv + i), m, s);
+        for (; i < nv; i += kDecThreads) {
+            const uint4 r[1] = {__ldg(xv + i)};
+            acc_batch<1>(r, m, s);
+        }
         cv = c0 + nv * 8;
     }
     for (int c = cv + tid; c < c1; c += kDecThreads) acc_value(bf16_bits_to_float(x[c]), m, s);
@@ -155,22 +211,24 @@ __device__ __forceinline__ float warp_sum(float v) {
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
-__device__ __forceinline__ float warp_max(float v) {
+// N independent warp sums, their butterflies interleaved (one shuffle
+// latency per step for all N).
+template <int N>
+__device__ __forceinline__ void warp_sum_n(float (&v)[N]) {
     #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-__device__ __forceinline__ int warp_sum_i(int v) {
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
+    for (int o = 16; o > 0; o >>= 1) {
+        #pragma unroll
+        for (int i = 0; i < N; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+    }
 }
 
 // Per-slot state in shared memory: what one warp works out about the
 // slot's answers and label.
 struct DecSlot {
-    int id[DLM_DECISION_MAX_ANSWERS];     // answer token ids
-    float z[DLM_DECISION_MAX_ANSWERS];    // their logits
+    int id[DLM_DECISION_MAX_ANSWERS];     // answer token ids, as given
+    float v[DLM_DECISION_MAX_ANSWERS];    // label values, as given
+    uint32_t zw[DLM_DECISION_MAX_ANSWERS];   // each answer's logit bits, in the half its id's parity selects
+    float z[DLM_DECISION_MAX_ANSWERS];    // the answers' logits
     float q[DLM_DECISION_MAX_ANSWERS];    // CE target
     float gr[DLM_DECISION_MAX_ANSWERS];   // restricted-CE + Brier part of d loss / dz (no g w)
     float g[DLM_DECISION_MAX_ANSWERS];    // the full gradient value written at each answer token
@@ -179,20 +237,56 @@ struct DecSlot {
     uint32_t bad;                         // status bits the slot raises (0 when valid)
 };
 
-// One warp, before the row's lse is known: the K answer tokens and the
-// label -- validity, the restricted softmax, the targets, CE_res, Brier and
-// the restricted + Brier part of each answer's gradient.  Needs only the K
-// answer logits, so it runs while the row itself is still being loaded.
-__device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, const uint16_t* x, bool row_ok,
-                                                 int lane, DecSlot& S) {
-    const int o0 = P.cand_off[slot], o1 = P.cand_off[slot + 1];
-    const int K = o1 - o0;
-    const int kind = P.kind[slot];
+// A slot's answer range and label kind, and the first verdict on them:
+// bad = 3 when the slot's row or its answer offsets lie outside the given
+// arrays, 2 when K is outside 1..128 or the label kind is unknown, else 0.
+struct DecHead {
+    int o0, K, kind, bad;
+};
+
+__device__ __forceinline__ DecHead dec_slot_head(const DecParams& P, bool row_ok, int o0, int o1, int kind) {
+    DecHead h;
+    h.o0 = o0;
+    h.K = o1 - o0;
+    h.kind = kind;
+    h.bad = (!row_ok || o0 < 0 || o1 < o0 || int64_t(o1) > P.n_cands) ? 3 : 0;
+    if (!h.bad) h.bad = (h.K < 1 || h.K > DLM_DECISION_MAX_ANSWERS) ? 2 : 0;
+    if (!h.bad) h.bad = (kind != DLM_LABEL_HARD && kind != DLM_LABEL_DIST && kind != DLM_LABEL_SET) ? 2 : 0;
+    return h;
+}
+
+// One warp: the answer ids and label values into shared memory.
+__device__ __forceinline__ void dec_fetch_answers(const DecParams& P, const DecHead& h, int lane, DecSlot& S) {
+    if (h.bad) return;
+    for (int k = lane; k < h.K; k += 32) {
+        S.id[k] = P.cand_ids[h.o0 + k];
+        S.v[k] = P.val[h.o0 + k];
+    }
+}
+
+// One warp, after dec_fetch_answers (same lane per answer): each in-range
+// answer's logit, its 16 bits stored in the half of a 32-bit word that
+// the answer id's parity selects.
+__device__ __forceinline__ void dec_fetch_logits(const DecParams& P, const uint16_t* x, const DecHead& h, int lane,
+                                                 DecSlot& S) {
+    if (h.bad) return;
+    for (int k = lane; k < h.K; k += 32) {
+        const int id = S.id[k];
+        if (id >= 0 && id < P.vocab) S.zw[k] = uint32_t(x[id]) << ((id & 1) * 16);
+    }
+}
+
+// One warp, before the row's lse is known, once the fetches are visible to
+// the whole warp: the label's validity, the restricted softmax, the
+// targets, CE_res, Brier and the restricted + Brier part of each answer's
+// gradient.  Needs only the K answer logits, so it overlaps the row's
+// stream.
+__device__ __forceinline__ void dec_slot_compute(const DecParams& P, const DecHead& h, int lane, DecSlot& S) {
+    const int K = h.K;
+    const int kind = h.kind;
     // 3: the slot's row or its answer offsets lie outside the given arrays;
     // 2: a malformed label; 1: an answer id outside the vocabulary
-    int bad = (!row_ok || o0 < 0 || o1 < o0 || int64_t(o1) > P.n_cands) ? 3 : 0;
-    if (!bad) bad = (K < 1 || K > DLM_DECISION_MAX_ANSWERS) ? 2 : 0;
-    if (!bad) bad = (kind != DLM_LABEL_HARD && kind != DLM_LABEL_DIST && kind != DLM_LABEL_SET) ? 2 : 0;
+    int bad = h.bad;
     float z[4], v[4];
     int id[4];
     int n_one = 0, n_other = 0;    // label checks: values equal to 1, and not in {0, 1}
@@ -202,35 +296,32 @@ __device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, c
         const int k = lane + 32 * j;
         id[j] = -1; z[j] = -INFINITY; v[j] = 0.f;
         if (!bad && k < K) {
-            id[j] = P.cand_ids[o0 + k];
-            v[j] = P.val[o0 + k];
-        }
-    }
-    #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int k = lane + 32 * j;
-        if (!bad && k < K) {
+            id[j] = S.id[k];
+            v[j] = S.v[k];
             if (id[j] < 0 || id[j] >= P.vocab) { bad_id = 1; id[j] = -1; }
-            else z[j] = bf16_bits_to_float(x[id[j]]);
+            else z[j] = (id[j] & 1) ? bf16hi(S.zw[k]) : bf16lo(S.zw[k]);
             n_one += (v[j] == 1.f);
             n_other += (v[j] != 0.f && v[j] != 1.f);
             bad_dist |= !(v[j] >= 0.f && v[j] < INFINITY);
-            S.id[k] = id[j];
         }
     }
-    __syncwarp();
-    // repeated answer ids: each lane compares its answers with the earlier ones
+    // repeated answer ids: lanes of one group of 32 that hold the same id
+    // (one match instruction), and each id against the earlier groups (an
+    // out-of-range id never equals a valid one)
     int dup = 0;
     if (!bad) {
         #pragma unroll
         for (int j = 0; j < 4; ++j) {
+            if (32 * j >= K) break;
             const int k = lane + 32 * j;
-            if (k < K && id[j] >= 0)
-                for (int i = 0; i < k; ++i) dup |= (S.id[i] == id[j]);
+            const bool has = k < K && id[j] >= 0;
+            dup |= __popc(__match_any_sync(0xffffffffu, has ? id[j] : -1 - lane)) > 1;
+            if (has)
+                for (int i = 0; i < 32 * j; ++i) dup |= (S.id[i] == id[j]);
         }
     }
-    n_one = warp_sum_i(n_one);
-    n_other = warp_sum_i(n_other);
+    n_one = int(__reduce_add_sync(0xffffffffu, unsigned(n_one)));
+    n_other = int(__reduce_add_sync(0xffffffffu, unsigned(n_other)));
     bad_id = __any_sync(0xffffffffu, bad_id);
     dup = __any_sync(0xffffffffu, dup);
     bad_dist = __any_sync(0xffffffffu, bad_dist);
@@ -242,35 +333,34 @@ __device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, c
         else if (kind == DLM_LABEL_DIST && bad_dist) bad = 2;
     }
     if (!bad) {
-        // candidate-restricted softmax
-        const float cm = warp_max(fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3])));
+        // candidate-restricted softmax (hardware ex2 / lg2: relative error
+        // about 2^-22, far below the bf16 gradient and the loss tolerance)
+        const float cm = warp_max_f32(fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3])));
         float se = 0.f;
         #pragma unroll
-        for (int j = 0; j < 4; ++j) se += (lane + 32 * j < K) ? expf(z[j] - cm) : 0.f;
-        const float lse_r = cm + logf(warp_sum(se));
+        for (int j = 0; j < 4; ++j) se += (lane + 32 * j < K) ? ex2((z[j] - cm) * kDecLog2e) : 0.f;
+        const float lse_r = cm + lg2(warp_sum(se)) * kDecLn2;
         const float n_set = float(n_one);
         float r[4], q[4], y[4];
-        float Q = 0.f, qz = 0.f, ce_res = 0.f, brier = 0.f, D = 0.f;
+        // sums over the answers: Q, sum q z, CE_res, Brier, D = sum r (r - y)
+        float t[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
         #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const bool on = lane + 32 * j < K;
-            r[j] = on ? expf(z[j] - lse_r) : 0.f;
+            r[j] = on ? ex2((z[j] - lse_r) * kDecLog2e) : 0.f;
             if (kind == DLM_LABEL_HARD) { y[j] = v[j]; q[j] = (1.f - P.smoothing) * v[j] + P.smoothing / float(K); }
             else if (kind == DLM_LABEL_SET) { y[j] = v[j] / n_set; q[j] = y[j]; }
             else { y[j] = v[j]; q[j] = v[j]; }
             if (!on) { q[j] = 0.f; y[j] = 0.f; }
-            Q += q[j];
-            qz += on ? q[j] * z[j] : 0.f;
-            ce_res -= on ? q[j] * (z[j] - lse_r) : 0.f;
+            t[0] += q[j];
+            t[1] += on ? q[j] * z[j] : 0.f;
+            t[2] -= on ? q[j] * (z[j] - lse_r) : 0.f;
             const float d = r[j] - y[j];
-            brier += d * d;
-            D += r[j] * d;
+            t[3] += d * d;
+            t[4] += r[j] * d;
         }
-        Q = warp_sum(Q);
-        qz = warp_sum(qz);
-        ce_res = warp_sum(ce_res);
-        brier = warp_sum(brier);
-        D = warp_sum(D);
+        warp_sum_n(t);                 // the five butterflies interleaved
+        const float Q = t[0], D = t[4];
         #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int k = lane + 32 * j;
@@ -282,12 +372,22 @@ __device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, c
                 S.q[k] = q[j];
             }
         }
-        if (lane == 0) { S.Q = Q; S.qz = qz; S.ce_res = ce_res; S.brier = brier; }
+        if (lane == 0) { S.Q = Q; S.qz = t[1]; S.ce_res = t[2]; S.brier = t[3]; }
     }
     if (lane == 0) {
         S.K = bad ? 0 : K;
         S.bad = bad == 0 ? 0u : bad == 1 ? DLM_DEV_BAD_TOKEN_ID : bad == 2 ? DLM_DEV_BAD_LABEL : DLM_DEV_BAD_LAYOUT;
     }
+}
+
+// One warp, all steps in a row with plain loads (rows of any alignment).
+__device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, const uint16_t* x, bool row_ok,
+                                                 int lane, DecSlot& S) {
+    const DecHead h = dec_slot_head(P, row_ok, P.cand_off[slot], P.cand_off[slot + 1], P.kind[slot]);
+    dec_fetch_answers(P, h, lane, S);
+    dec_fetch_logits(P, x, h, lane, S);
+    __syncwarp();
+    dec_slot_compute(P, h, lane, S);
 }
 
 // One warp, once lse is known: the full-vocabulary CE and its share of each
@@ -301,14 +401,15 @@ __device__ __forceinline__ void dec_slot_finish(const DecParams& P, int slot, in
     const float Q = K > 0 ? S.Q : 0.f;
     for (int k = lane; k < K; k += 32) {
         float g = S.gr[k];
-        if (P.use_full) g += Q * expf(S.z[k] - lse) - S.q[k];
+        if (P.use_full) g += Q * ex2((S.z[k] - lse) * kDecLog2e) - S.q[k];
         S.g[k] = gw * g;
     }
     if (lane == 0) {
         float slot_loss = 0.f;
         if (K > 0) {
-            const float ce_full = Q * lse - S.qz;     // -sum q_k (z_k - lse)
-            slot_loss = P.w * (P.use_res * S.ce_res + P.use_full * ce_full + P.brier_w * S.brier);
+            // -sum q_k (z_k - lse); lse is not formed (-inf) when the full CE is off
+            const float ce_full = P.use_full ? Q * lse - S.qz : 0.f;
+            slot_loss = P.w * (P.use_res * S.ce_res + ce_full + P.brier_w * S.brier);
         }
         S.coef = gw * float(P.use_full) * Q;
         if (split == 0) P.slot_loss[slot] = slot_loss;
@@ -344,7 +445,9 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_grad(DecParams P) {
     // the dense part of this split: coef * P_v (zeros for a restricted-only
     // loss or an invalid slot)
     const float coef = S.coef;
-    const float sh = lse * kDecLog2e;
+    const bool fold = coef > 0.f;
+    const float lb = lse * kDecLog2e - (fold ? log2f(coef) : 0.f);
+    const float mul = fold ? 1.f : coef;
     uint16_t* out = P.dlogits + int64_t(slot) * P.ld_out;
     const int c0 = split * P.chunk;
     const int c1 = min(c0 + P.chunk, P.vocab);
@@ -354,36 +457,21 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_grad(DecParams P) {
         const uint4* xv = reinterpret_cast<const uint4*>(x + c0);
         uint4* ov = reinterpret_cast<uint4*>(out + c0);
         const uint64_t ef = policy_evict_first();
+        const uint64_t l2e = f2pack(kDecLog2e, kDecLog2e), nlb = f2pack(-lb, -lb);
         int i = tid;
         for (; i + (kDecUnroll - 1) * kDecThreads < nv; i += kDecUnroll * kDecThreads) {
             uint4 rv[kDecUnroll];
             #pragma unroll
             for (int u = 0; u < kDecUnroll; ++u) rv[u] = __ldg(xv + i + u * kDecThreads);
             #pragma unroll
-            for (int u = 0; u < kDecUnroll; ++u) {
-                const uint32_t w4[4] = {rv[u].x, rv[u].y, rv[u].z, rv[u].w};
-                uint32_t o4[4];
-                #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    o4[k] = pack_bf16x2(coef * ex2(fmaf(bf16lo(w4[k]), kDecLog2e, -sh)),
-                                        coef * ex2(fmaf(bf16hi(w4[k]), kDecLog2e, -sh)));
-                st_global_v4_hint(ov + i + u * kDecThreads, make_uint4(o4[0], o4[1], o4[2], o4[3]), ef);
-            }
+            for (int u = 0; u < kDecUnroll; ++u)
+                st_global_v4_hint(ov + i + u * kDecThreads, dec_dense_vec(rv[u], l2e, nlb, fold, mul), ef);
         }
-        for (; i < nv; i += kDecThreads) {
-            const uint4 rv = __ldg(xv + i);
-            const uint32_t w4[4] = {rv.x, rv.y, rv.z, rv.w};
-            uint32_t o4[4];
-            #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                o4[k] = pack_bf16x2(coef * ex2(fmaf(bf16lo(w4[k]), kDecLog2e, -sh)),
-                                    coef * ex2(fmaf(bf16hi(w4[k]), kDecLog2e, -sh)));
-            st_global_v4_hint(ov + i, make_uint4(o4[0], o4[1], o4[2], o4[3]), ef);
-        }
+        for (; i < nv; i += kDecThreads) st_global_v4_hint(ov + i, dec_dense_vec(__ldg(xv + i), l2e, nlb, fold, mul), ef);
         cv = c0 + nv * 8;
     }
     for (int c = cv + tid; c < c1; c += kDecThreads) {
-        const float g = coef * ex2(fmaf(bf16_bits_to_float(x[c]), kDecLog2e, -sh));
+        const float g = mul * ex2(fmaf(bf16_bits_to_float(x[c]), kDecLog2e, -lb));
         out[c] = __bfloat16_as_ushort(__float2bfloat16_rn(g));
     }
     __syncthreads();                   // the dense stores of this CTA come first
@@ -402,26 +490,42 @@ __device__ __forceinline__ uint4 ldg_v4_hint(const void* p, uint64_t pol) {
     return r;
 }
 
+// loads in flight per thread: six per batch in the first read (seven
+// streaming warps) and four in the second (eight warps) give three and four
+// batches per thread for the 31,616-column splits of V = 126,464 -- fewer
+// serial memory latencies measured faster than more loads per batch
+#ifndef DLM_DEC_CU
+#define DLM_DEC_CU 6
+#endif
+#ifndef DLM_DEC_CU2
+#define DLM_DEC_CU2 4
+#endif
+
 // Fast path: one thread-block cluster per slot, one CTA per split of the
 // row (cluster rank = split; 1, 2, 4 or 8 splits).  Each CTA reads its split
 // twice: the first time from HBM, kept in L2 with an evict_last policy (a
 // call's label rows are tens of MB), for its (max, sum exp); the cluster
-// exchanges only those two floats through distributed shared memory and
-// every CTA merges the n_split partials in rank order into the same lse; the
+// exchanges only those two floats per warp through distributed shared
+// memory and one warp of every CTA merges them into the same lse; the
 // second read comes from L2 and writes the gradient, then the answer-token
-// entries are rewritten as in k_dec_grad.  One warp works out the label
-// meanwhile.  The CTAs hold nothing but a few KB of shared memory, so every
-// cluster of a call is resident at once and no CTA waits for a second wave
-// (holding each split in shared memory instead measured slower: the call's
-// rows do not fit on chip at once).  The final cluster barrier keeps every
-// CTA's partial alive until all peers have read it.
+// entries are rewritten as in k_dec_grad.  Warp 0 is the label warp: it
+// reads the slot's answers and works out the label while the other seven
+// warps stream the first read (the label's chain of dependent loads and
+// warp reductions stays off the critical path); all eight warps stream the
+// second.  With the full CE off the first read is skipped (lse is not
+// needed) and the dense gradient is zero.  The CTAs hold nothing but a few
+// KB of shared memory, so every cluster of a call is resident at once and
+// no CTA waits for a second wave (holding each split in shared memory
+// instead measured slower: the call's rows do not fit on chip at once).
+// The final cluster barrier keeps every CTA's partials alive until all
+// peers have read them.
 __global__ void __launch_bounds__(kDecThreads, 4) k_dec_cluster(DecParams P) {
-    constexpr int kU = 4;              // 16-byte loads in flight per thread
-    __shared__ __align__(8) float2 s_part;
-    __shared__ float sm_m[kDecThreads / 32], sm_s[kDecThreads / 32];
+    constexpr int kU = DLM_DEC_CU;     // 16-byte loads in flight per thread, first read
+    constexpr int kU2 = DLM_DEC_CU2;   // the same, second read
+    __shared__ __align__(8) float2 s_part[kDecThreads / 32];   // (max, sum exp) per warp
     __shared__ DecSlot S;
     __shared__ float s_lse;
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = int(cluster_ctarank()), slot = blockIdx.y;
     const int c0 = split * P.chunk;
     const int c1 = min(c0 + P.chunk, P.vocab);
@@ -434,77 +538,66 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_dec_cluster(DecParams P) {
     const uint4* xv = reinterpret_cast<const uint4*>(x + c0);
     const uint64_t keep = policy_evict_last(), drop = policy_evict_first();
     float m = -INFINITY, s = 0.f;
-    {
-        int i = tid;
-        for (; i + (kU - 1) * kDecThreads < nvec; i += kU * kDecThreads) {
+    if (warp == 0) {
+        // the label warp: the slot's answers and label, while the others stream
+        dec_slot_prepare(P, slot, x, row_ok, lane, S);
+    } else if (P.use_full) {
+        // batches of kU loads in flight per thread, the last one partial
+        // (its missing vectors read as -inf, which adds nothing): one
+        // memory latency per batch, none for a ragged tail
+        constexpr int kStream = kDecThreads - 32;
+        const uint4 ninf = make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+        for (int i = tid - 32; i < nvec; i += kU * kStream) {
             uint4 r[kU];
             #pragma unroll
-            for (int u = 0; u < kU; ++u) r[u] = ldg_v4_hint(xv + i + u * kDecThreads, keep);
-            #pragma unroll
-            for (int u = 0; u < kU; ++u) acc_vec(r[u], m, s);
+            for (int u = 0; u < kU; ++u)
+                r[u] = i + u * kStream < nvec ? ldg_v4_hint(xv + i + u * kStream, keep) : ninf;
+            acc_batch<kU>(r, m, s);
         }
-        for (; i < nvec; i += kDecThreads) acc_vec(ldg_v4_hint(xv + i, keep), m, s);
     }
-    if (tid < 32) dec_slot_prepare(P, slot, x, row_ok, tid, S);
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-        const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-        lse_merge(m, s, m2, s2);
-    }
-    if (lane == 0) { sm_m[tid >> 5] = m; sm_s[tid >> 5] = s; }
-    __syncthreads();
-    if (tid == 0) {
-        float M = sm_m[0], Ssum = sm_s[0];
-        for (int k = 1; k < kDecThreads / 32; ++k) lse_merge(M, Ssum, sm_m[k], sm_s[k]);
-        s_part = make_float2(M, Ssum);
-    }
-    cluster_sync_all();
-    if (tid == 0) {
+    warp_lse(m, s);
+    if (lane == 0) s_part[warp] = make_float2(m, s);
+    cluster_sync_all();                // every warp partial of the cluster is written
+    if (warp == 0) {
+        // lane l merges warp partials l and l + 32 of the cluster (CTA e / 8,
+        // warp e % 8), then a butterfly: lse_merge is symmetric, so every
+        // lane of every CTA ends with the same bits
+        constexpr int kWarps = kDecThreads / 32;
         float M = -INFINITY, Ssum = 0.f;
-        for (int r = 0; r < P.n_split; ++r) {
+        for (int e = lane; e < P.n_split * kWarps; e += 32) {
             float pm, ps;
-            const uint32_t a = mapa_shared(smem_addr(&s_part), uint32_t(r));
+            const uint32_t a = mapa_shared(smem_addr(&s_part[e % kWarps]), uint32_t(e / kWarps));
             asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(pm), "=f"(ps) : "r"(a) : "memory");
             lse_merge(M, Ssum, pm, ps);
         }
-        s_lse = M + logf(Ssum);
+        warp_lse(M, Ssum);
+        const float lse_w = M + logf(Ssum);
+        dec_slot_finish(P, slot, split, lse_w, lane, S);
+        if (lane == 0) s_lse = lse_w;
     }
     __syncthreads();
     const float lse = s_lse;
-    if (tid < 32) dec_slot_finish(P, slot, split, lse, tid, S);
-    __syncthreads();
     if (tid == 0) P.err[int64_t(slot) * P.n_split + split] = split == 0 ? S.bad : 0u;
     const float coef = S.coef;
-    const float sh = lse * kDecLog2e;
     uint16_t* out = P.dlogits + int64_t(slot) * P.ld_out;
     uint4* ov = reinterpret_cast<uint4*>(out + c0);
-    {
-        int i = tid;
-        for (; i + (kU - 1) * kDecThreads < nvec; i += kU * kDecThreads) {
-            uint4 r[kU];
+    if (coef == 0.f) {
+        // restricted-only loss or an invalid slot: zeros, nothing to read
+        for (int i = tid; i < nvec; i += kDecThreads) st_global_v4_hint(ov + i, make_uint4(0u, 0u, 0u, 0u), drop);
+    } else {
+        const bool fold = coef > 0.f;
+        const float lb = lse * kDecLog2e - (fold ? log2f(coef) : 0.f);
+        const float mul = fold ? 1.f : coef;
+        const uint64_t l2e = f2pack(kDecLog2e, kDecLog2e), nlb = f2pack(-lb, -lb);
+        for (int i = tid; i < nvec; i += kU2 * kDecThreads) {
+            uint4 r[kU2];
             #pragma unroll
-            for (int u = 0; u < kU; ++u) r[u] = ldg_v4_hint(xv + i + u * kDecThreads, drop);
+            for (int u = 0; u < kU2; ++u)
+                if (i + u * kDecThreads < nvec) r[u] = ldg_v4_hint(xv + i + u * kDecThreads, drop);
             #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                const uint32_t w4[4] = {r[u].x, r[u].y, r[u].z, r[u].w};
-                uint32_t o4[4];
-                #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    o4[k] = pack_bf16x2(coef * ex2(fmaf(bf16lo(w4[k]), kDecLog2e, -sh)),
-                                        coef * ex2(fmaf(bf16hi(w4[k]), kDecLog2e, -sh)));
-                st_global_v4_hint(ov + i + u * kDecThreads, make_uint4(o4[0], o4[1], o4[2], o4[3]), drop);
-            }
-        }
-        for (; i < nvec; i += kDecThreads) {
-            const uint4 rv = ldg_v4_hint(xv + i, drop);
-            const uint32_t w4[4] = {rv.x, rv.y, rv.z, rv.w};
-            uint32_t o4[4];
-            #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                o4[k] = pack_bf16x2(coef * ex2(fmaf(bf16lo(w4[k]), kDecLog2e, -sh)),
-                                    coef * ex2(fmaf(bf16hi(w4[k]), kDecLog2e, -sh)));
-            st_global_v4_hint(ov + i, make_uint4(o4[0], o4[1], o4[2], o4[3]), drop);
+            for (int u = 0; u < kU2; ++u)
+                if (i + u * kDecThreads < nvec)
+                    st_global_v4_hint(ov + i + u * kDecThreads, dec_dense_vec(r[u], l2e, nlb, fold, mul), drop);
         }
     }
     __syncthreads();

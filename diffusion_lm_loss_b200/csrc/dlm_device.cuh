@@ -48,6 +48,14 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Base-2 logarithm by the hardware instruction (PTX lg2.approx.ftz.f32: one
+// MUFU op, absolute error about 2^-22 near 1).
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction, two lanes,
 // each rounded to nearest like its scalar form).
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
