@@ -226,8 +226,6 @@ __device__ __forceinline__ void warp_sum_n(float (&v)[N]) {
 // slot's answers and label.
 struct DecSlot {
     int id[DLM_DECISION_MAX_ANSWERS];     // answer token ids, as given
-    float v[DLM_DECISION_MAX_ANSWERS];    // label values, as given
-    uint32_t zw[DLM_DECISION_MAX_ANSWERS];   // each answer's logit bits, in the half its id's parity selects
     float z[DLM_DECISION_MAX_ANSWERS];    // the answers' logits
     float q[DLM_DECISION_MAX_ANSWERS];    // CE target
     float gr[DLM_DECISION_MAX_ANSWERS];   // restricted-CE + Brier part of d loss / dz (no g w)
@@ -255,51 +253,31 @@ __device__ __forceinline__ DecHead dec_slot_head(const DecParams& P, bool row_ok
     return h;
 }
 
-// One warp: the answer ids and label values into shared memory.
-__device__ __forceinline__ void dec_fetch_answers(const DecParams& P, const DecHead& h, int lane, DecSlot& S) {
-    if (h.bad) return;
-    for (int k = lane; k < h.K; k += 32) {
-        S.id[k] = P.cand_ids[h.o0 + k];
-        S.v[k] = P.val[h.o0 + k];
-    }
-}
-
-// One warp, after dec_fetch_answers (same lane per answer): each in-range
-// answer's logit, its 16 bits stored in the half of a 32-bit word that
-// the answer id's parity selects.
-__device__ __forceinline__ void dec_fetch_logits(const DecParams& P, const uint16_t* x, const DecHead& h, int lane,
-                                                 DecSlot& S) {
-    if (h.bad) return;
-    for (int k = lane; k < h.K; k += 32) {
-        const int id = S.id[k];
-        if (id >= 0 && id < P.vocab) S.zw[k] = uint32_t(x[id]) << ((id & 1) * 16);
-    }
-}
-
-// One warp, before the row's lse is known, once the fetches are visible to
-// the whole warp: the label's validity, the restricted softmax, the
+// One warp, before the row's lse is known, given each lane's answers
+// (answer k = lane + 32 j: id, label value and the logit's bf16 bits; the
+// ids also in S.id): the label's validity, the restricted softmax, the
 // targets, CE_res, Brier and the restricted + Brier part of each answer's
 // gradient.  Needs only the K answer logits, so it overlaps the row's
-// stream.
-__device__ __forceinline__ void dec_slot_compute(const DecParams& P, const DecHead& h, int lane, DecSlot& S) {
+// stream; the logits are first used after the label checks, so their loads
+// can still be in flight during them.
+__device__ __forceinline__ void dec_slot_compute(const DecParams& P, const DecHead& h, int lane, DecSlot& S,
+                                                 const int (&id_in)[4], const float (&v)[4],
+                                                 const uint16_t (&zb)[4]) {
     const int K = h.K;
     const int kind = h.kind;
     // 3: the slot's row or its answer offsets lie outside the given arrays;
     // 2: a malformed label; 1: an answer id outside the vocabulary
     int bad = h.bad;
-    float z[4], v[4];
     int id[4];
     int n_one = 0, n_other = 0;    // label checks: values equal to 1, and not in {0, 1}
     int bad_id = 0, bad_dist = 0;
     #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int k = lane + 32 * j;
-        id[j] = -1; z[j] = -INFINITY; v[j] = 0.f;
+        id[j] = -1;
         if (!bad && k < K) {
-            id[j] = S.id[k];
-            v[j] = S.v[k];
+            id[j] = id_in[j];
             if (id[j] < 0 || id[j] >= P.vocab) { bad_id = 1; id[j] = -1; }
-            else z[j] = (id[j] & 1) ? bf16hi(S.zw[k]) : bf16lo(S.zw[k]);
             n_one += (v[j] == 1.f);
             n_other += (v[j] != 0.f && v[j] != 1.f);
             bad_dist |= !(v[j] >= 0.f && v[j] < INFINITY);
@@ -333,6 +311,9 @@ __device__ __forceinline__ void dec_slot_compute(const DecParams& P, const DecHe
         else if (kind == DLM_LABEL_DIST && bad_dist) bad = 2;
     }
     if (!bad) {
+        float z[4];
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) z[j] = id[j] >= 0 ? bf16_bits_to_float(zb[j]) : -INFINITY;
         // candidate-restricted softmax (hardware ex2 / lg2: relative error
         // about 2^-22, far below the bf16 gradient and the loss tolerance)
         const float cm = warp_max_f32(fmaxf(fmaxf(z[0], z[1]), fmaxf(z[2], z[3])));
@@ -380,14 +361,29 @@ __device__ __forceinline__ void dec_slot_compute(const DecParams& P, const DecHe
     }
 }
 
-// One warp, all steps in a row with plain loads (rows of any alignment).
+// One warp: the slot's answers and label values, the answers' logits
+// (loads issued before the label checks that do not need them), then
+// dec_slot_compute.
 __device__ __forceinline__ void dec_slot_prepare(const DecParams& P, int slot, const uint16_t* x, bool row_ok,
                                                  int lane, DecSlot& S) {
     const DecHead h = dec_slot_head(P, row_ok, P.cand_off[slot], P.cand_off[slot + 1], P.kind[slot]);
-    dec_fetch_answers(P, h, lane, S);
-    dec_fetch_logits(P, x, h, lane, S);
-    __syncwarp();
-    dec_slot_compute(P, h, lane, S);
+    int id[4];
+    float v[4];
+    uint16_t zb[4];
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int k = lane + 32 * j;
+        id[j] = -1; v[j] = 0.f;
+        if (!h.bad && k < h.K) {
+            id[j] = P.cand_ids[h.o0 + k];
+            v[j] = P.val[h.o0 + k];
+            S.id[k] = id[j];
+        }
+    }
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) zb[j] = (id[j] >= 0 && id[j] < P.vocab) ? x[id[j]] : uint16_t(0);
+    __syncwarp();                      // S.id of every lane, for the repeated-id check
+    dec_slot_compute(P, h, lane, S, id, v, zb);
 }
 
 // One warp, once lse is known: the full-vocabulary CE and its share of each
