@@ -110,6 +110,7 @@ def test_decision_full_workload(label_softmax):
     (300, 2048, 2, 8, 0, 2),      # many slots, one CTA per row
     (3, 16, 16, 16, 0, 3),        # every token of the vocabulary an answer
     (4, 300000, 2, 26, 0, 4),     # long rows: clusters of 8 CTAs of 37,500 columns
+    (6, 8192, 33, 128, 0, 5),     # the cluster path with more than one group of 32 answers
 ])
 def test_decision_elementwise(n, V, kmin, kmax, ld_pad, seed):
     off, ids, kind, val = _batch(seed, n, V, kmax, kmin=kmin)
@@ -185,6 +186,38 @@ def test_decision_invalid_slots_are_flagged_and_skipped():
     # a call after the failing one starts from a clean status word
     out2 = dlm.decision_loss_fwd_bwd(logits, V, *_dev(off, ids, kind, val), out=out)
     assert out2.device_status() == 0
+
+
+def test_decision_repeated_ids_across_answer_groups():
+    """Repeated answer ids found wherever they sit among K = 70 answers
+    (the label warp holds answers k, k + 32, k + 64 per lane): across two
+    groups of 32, inside the second group and inside the third.  Those
+    slots are refused (DEV_BAD_LABEL, zero share and gradient), the valid
+    one matches the oracle -- on both kernel paths."""
+    n, V, K = 4, 4096, 70
+    rng = np.random.default_rng(11)
+    off = np.arange(0, (n + 1) * K, K, dtype=np.int32)
+    ids = np.concatenate([rng.choice(V, size=K, replace=False) for _ in range(n)]).astype(np.int32)
+    kind = np.full(n, oracle.DIST, np.int32)
+    val = np.concatenate([rng.dirichlet(np.ones(K)) for _ in range(n)]).astype(np.float32)
+    ids[off[1] + 40] = ids[off[1] + 3]          # across groups 0 and 1
+    ids[off[2] + 50] = ids[off[2] + 33]         # inside group 1
+    ids[off[3] + 69] = ids[off[3] + 64]         # inside group 2
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(11)
+    for ld_pad in (0, 3):
+        base = (torch.randn((n, V + ld_pad), generator=gen, device="cuda") * 2).to(torch.bfloat16)
+        logits = base[:, :V] if ld_pad else base
+        out = dlm.decision_loss_fwd_bwd(logits, V, *_dev(off, ids, kind, val))
+        torch.cuda.synchronize()
+        assert out.device_status() == dlm.DEV_BAD_LABEL
+        g = out.dlogits.float().cpu()
+        sl = out.slot_loss.cpu().numpy()[:n]
+        for s_ in (1, 2, 3):
+            assert sl[s_] == 0.0 and bool((g[s_] == 0).all())
+        ref = oracle.decision_loss(di.bf16_bits(logits), V, np.array([0]), off[:2], ids[:K], kind[:1], val[:K])
+        assert_loss_close(float(out.loss.item()), ref["loss"] / n)
+        np.testing.assert_allclose(sl[0], ref["slot_loss"][0] / n, rtol=1e-5)
 
 
 def test_decision_no_slots_and_reproducible():
