@@ -191,12 +191,7 @@ __global__ void __launch_bounds__(kDecThreads) k_dec_partial(DecParams P) {
         cv = c0 + nv * 8;
     }
     for (int c = cv + tid; c < c1; c += kDecThreads) acc_value(bf16_bits_to_float(x[c]), m, s);
-    #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-        const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-        lse_merge(m, s, m2, s2);
-    }
+    warp_lse(m, s);
     if ((tid & 31) == 0) { sm_m[tid >> 5] = m; sm_s[tid >> 5] = s; }
     __syncthreads();
     if (tid == 0) {
