@@ -230,7 +230,7 @@ struct DecSlot {
     uint32_t bad;                         // status bits the slot raises (0 when valid)
 };
 
-// A slot's answer range and label kind, and the first verdict on them:
+// A slot's answer range and label kind, and the first check of them:
 // bad = 3 when the slot's row or its answer offsets lie outside the given
 // arrays, 2 when K is outside 1..128 or the label kind is unknown, else 0.
 struct DecHead {
