@@ -145,6 +145,51 @@ def test_linear_uniform_rejections(L):
     assert L.dlm_linear_loss_uniform_workspace_size(ctypes.byref(half), ctypes.byref(half), 64, 1024) == 0
 
 
+def test_decision_and_scale_rejections(L):
+    """dlm_decision_loss_fwd_bwd and dlm_scale_bf16 refuse bad arguments
+    before any device query or launch."""
+    n, V = 4, 1024
+    ws = L.dlm_decision_workspace_size(n, V)
+    assert ws > 0
+    assert L.dlm_decision_workspace_size(dlm.DECISION_MAX_SLOTS, V) > 0
+    assert L.dlm_decision_workspace_size(dlm.DECISION_MAX_SLOTS + 1, V) == 0
+    assert L.dlm_decision_workspace_size(-1, V) == 0
+    assert L.dlm_decision_workspace_size(n, 0) == 0
+    # n_slots, logits, n_rows, ld, vocab, slot_rows, cand_off, n_cands, cand_ids, kind, val,
+    # label_softmax, brier, smoothing, grad_scale, loss, slot_loss, dlogits, ld_out, ws, ws_bytes, stream
+    args = [n, 4096, n, V, V, None, 256, 8, 512, 768, 1024, dlm.LABEL_SOFTMAX_BOTH, 0.1, 0.0, 1.0, 1280,
+            None, 8192, V, 1 << 20, ws, None]
+
+    def rc(**kw):
+        a = list(args)
+        for k, v in kw.items():
+            a[int(k[1:])] = v
+        return L.dlm_decision_loss_fwd_bwd(*a)
+
+    assert rc(a0=dlm.DECISION_MAX_SLOTS + 1) == 1         # too many slots
+    assert rc(a0=-1) == 1
+    assert rc(a4=0) == 1                                  # vocab
+    assert rc(a3=V - 1) == 1                              # ld < vocab
+    assert rc(a18=V - 1) == 1                             # ld_out < vocab
+    assert rc(a2=0) == 1                                  # no rows
+    assert rc(a2=n - 1) == 1                              # fewer rows than slots, no slot_rows
+    assert rc(a7=-1) == 1                                 # n_cands
+    assert rc(a11=0) == 1 and rc(a11=4) == 1              # label_softmax
+    assert rc(a12=-0.5) == 1 and rc(a12=float("inf")) == 1   # brier weight
+    assert rc(a13=1.5) == 1 and rc(a13=-0.1) == 1         # smoothing
+    assert rc(a14=float("nan")) == 1                      # grad_scale
+    assert rc(a15=None) == 1 and rc(a19=None) == 1        # loss, workspace
+    assert rc(a1=None) == 1 and rc(a6=None) == 1 and rc(a17=None) == 1
+    assert rc(a19=(1 << 20) + 4) == 1                     # misaligned workspace
+    assert rc(a20=ws - 1) == 3                            # workspace too small
+    # scale: rows, cols, ld, scale
+    assert L.dlm_scale_bf16(4096, -1, 64, 64, 256, None) == 1
+    assert L.dlm_scale_bf16(4096, 4, 64, 63, 256, None) == 1
+    assert L.dlm_scale_bf16(4096, 4, 64, 64, None, None) == 1
+    assert L.dlm_scale_bf16(None, 4, 64, 64, 256, None) == 1
+    assert L.dlm_scale_bf16(None, 0, 64, 64, 256, None) == 0   # empty: nothing to do
+
+
 def test_workspace_size_grows_with_rows(L):
     a = dlm.Layout(1, 4096, 4096, None, None)
     b = dlm.Layout(1, 8192, 8192, None, None)

@@ -220,6 +220,28 @@ def test_decision_repeated_ids_across_answer_groups():
         np.testing.assert_allclose(sl[0], ref["slot_loss"][0] / n, rtol=1e-5)
 
 
+def test_decision_most_slots_one_call():
+    """DLM_DECISION_MAX_SLOTS label slots in one call (the cluster grid's
+    y extent at its limit; one CTA per slot of V = 64), with one- to
+    four-answer questions, against the oracle element by element; one slot
+    more is refused before anything runs."""
+    n, V = dlm.DECISION_MAX_SLOTS, 64
+    off, ids, kind, val = _batch(12, n, V, 4, kmin=1)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(12)
+    logits = (torch.randn((n + 1, V), generator=gen, device="cuda") * 2).to(torch.bfloat16)
+    out = dlm.decision_loss_fwd_bwd(logits[:n], V, *_dev(off, ids, kind, val))
+    torch.cuda.synchronize()
+    assert out.device_status() == 0
+    ref = oracle.decision_loss(di.bf16_bits(logits[:n]), V, None, off, ids, kind, val)
+    _check(out, ref, off, ids, None, 1.0, 0.1, n, V, oracle.LABEL_BOTH)
+    off2 = np.concatenate([off, [off[-1] + 1]]).astype(np.int32)
+    ids2 = np.concatenate([ids, [0]]).astype(np.int32)
+    with pytest.raises(dlm.DlmError):
+        dlm.decision_loss_fwd_bwd(logits, V, *_dev(off2, ids2, np.concatenate([kind, [oracle.HARD]]).astype(np.int32),
+                                                   np.concatenate([val, [1.0]]).astype(np.float32)))
+
+
 def test_decision_no_slots_and_reproducible():
     V = 1024
     z = torch.zeros((0, V), dtype=torch.bfloat16, device="cuda")

@@ -81,6 +81,15 @@ def test_every_entry_point_reports_its_cuda_failure(L):
         _fails_at(L, L.dlm_linear_loss_uniform_fwd_bwd(lp, 4096, ctypes.byref(enc), 8192, 512, 16384, 64,
                                                        1024, 256, 0, 1.0, 1.0, 1024, 1280, 32768, 65536,
                                                        None, WS, ws_u, None), "k_plan")
+        ws_d = L.dlm_decision_workspace_size(4, 1024)
+        dec = [4, 4096, 4, 1024, 1024, None, 256, 8, 512, 768, 1024, 3, 0.1, 0.0, 1.0, 1280, None, 8192, 1024,
+               WS, ws_d, None]
+        _fails_at(L, L.dlm_decision_loss_fwd_bwd(*dec), "k_dec_cluster launch")          # 16-byte rows
+        dec_g = list(dec); dec_g[3] = 1025
+        _fails_at(L, L.dlm_decision_loss_fwd_bwd(*dec_g), "k_dec_partial launch")      # any row stride
+        dec_0 = list(dec); dec_0[0] = 0
+        _fails_at(L, L.dlm_decision_loss_fwd_bwd(*dec_0), "status reset")              # no slots
+        _fails_at(L, L.dlm_scale_bf16(4096, 4, 64, 64, 256, None), "k_scale_bf16 launch")
         _fails_at(L, L.dlm_selftest_bounded_wait(1000, 256, None), "k_selftest_wait launch")
         _fails_at(L, L.dlm_get_device_status(WS, ctypes.byref(ctypes.c_uint32()), None),
                   "dlm_get_device_status")
