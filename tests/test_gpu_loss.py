@@ -135,10 +135,12 @@ def test_dream_like_shifted_full_size():
 
 
 @pytest.mark.parametrize("V,ld", [(1003, 1003), (1000, 1010), (5000, 5000), (8192, 8200),
-                                  (40000, 40000), (262144, 262144)])
+                                  (40000, 40000), (262144, 262144), (1048576, 1048576), (1000003, 1000003)])
 def test_vocab_and_stride_variants(V, ld):
     """Ragged vocabularies (general kernel), padded row strides (columns past
-    V untouched), and the largest cluster split."""
+    V untouched), the largest cluster split, and rows of about a million
+    columns (2 MB each: the rows in flight no longer fit in L2) on both
+    kernels."""
     spec = di.WORKLOADS["abs_b2_l64_v1024"].scaled(vocab=V, mask_id=V - 1, ids_high=V - 2,
                                                    n_units=2, seq_len=24, std=3.0)
     case = di.make_case(spec.scaled(vocab=ld), "cuda")      # draw [rows, ld], use the first V
