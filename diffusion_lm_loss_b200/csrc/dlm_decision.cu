@@ -604,32 +604,35 @@ constexpr int kDecRedThreads = 256;
 
 // The mean over slots (fixed order, double) and, after the cluster path,
 // the status word: the or of every CTA's error word (written on every call,
-// so nothing needs zeroing between calls).
+// so nothing needs zeroing between calls).  Warp butterflies and one CTA
+// barrier: the kernel sits at the end of the call, so its latency counts.
 __global__ void __launch_bounds__(kDecRedThreads) k_dec_reduce(const float* __restrict__ slot_loss, int n,
                                                                float* __restrict__ loss,
                                                                const uint32_t* __restrict__ err, int n_err,
                                                                uint32_t* __restrict__ status) {
-    __shared__ double red[kDecRedThreads];
-    __shared__ uint32_t bits;
-    const int tid = threadIdx.x;
+    constexpr int kWarps = kDecRedThreads / 32;
+    __shared__ double red[kWarps];
+    __shared__ uint32_t bits[kWarps];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_wait();                        // slot losses of the gradient kernel
-    if (tid == 0) bits = 0u;
-    __syncthreads();
-    if (err) {
-        uint32_t b = 0u;
+    uint32_t b = 0u;
+    if (err)
         for (int i = tid; i < n_err; i += kDecRedThreads) b |= err[i];
-        if (b) atomicOr(&bits, b);
-    }
     double acc = 0.0;
     for (int i = tid; i < n; i += kDecRedThreads) acc += double(slot_loss[i]);
-    red[tid] = acc;
+    #pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    b = __reduce_or_sync(0xffffffffu, b);
+    if (lane == 0) { red[warp] = acc; bits[warp] = b; }
     __syncthreads();
-    if (err && tid == 0) *status = bits;
-    for (int o = kDecRedThreads / 2; o > 0; o >>= 1) {
-        if (tid < o) red[tid] += red[tid + o];
-        __syncthreads();
+    if (tid == 0) {
+        double t = 0.0;
+        uint32_t bb = 0u;
+        #pragma unroll
+        for (int w = 0; w < kWarps; ++w) { t += red[w]; bb |= bits[w]; }
+        *loss = float(t);
+        if (err) *status = bb;
     }
-    if (tid == 0) *loss = float(red[0]);
 }
 
 struct DecPlan {
