@@ -641,14 +641,28 @@ struct DecPlan {
 };
 
 // The cluster path: n_split in {1, 2, 4, 8} (a portable cluster size), the
-// smallest that gives about 512 CTAs in all (3.5 per SM, every cluster
-// resident at once) without cutting splits under 2,048 columns.  Needs
-// vocab % 8 == 0 (16-byte vectors).
-inline bool dec_cluster_plan(int n_slots, int vocab, int& n_split, int& chunk) {
+// smallest that both gives about 512 CTAs in all (3.5 per SM, every cluster
+// of a small call resident at once) and keeps the rows in flight -- the
+// resident CTAs' rows, each read twice -- within an L2 budget, without
+// cutting splits under 2,048 columns.  The second read must find its row in
+// L2: on 2,048 slots of V = 126,464, one CTA per row (150 MB in flight) ran
+// at 0.66 of HBM, two (75 MB) at 0.78, four (37 MB) at 0.80, eight at 0.60
+// (per-CTA overheads).  Needs vocab % 8 == 0 (16-byte vectors).
+constexpr int kDecCtasPerSm = 4;             // k_dec_cluster's launch bound
+#ifndef DLM_DEC_L2_BUDGET
+#define DLM_DEC_L2_BUDGET 40e6
+#endif
+constexpr double kDecL2RowBudget = DLM_DEC_L2_BUDGET;   // bytes of rows in flight between the two reads
+inline bool dec_cluster_plan(int n_slots, int vocab, int sms, int& n_split, int& chunk) {
     if (n_slots <= 0 || vocab % 8 != 0) return false;
     const int64_t want = (512 + n_slots - 1) / n_slots;   // CTAs wanted per slot
+    const int64_t resident = int64_t(sms > 0 ? sms : 148) * kDecCtasPerSm;
+    auto fits = [&](int ns) {
+        const int64_t rows = resident / ns < n_slots ? resident / ns : n_slots;
+        return double(rows) * 2.0 * double(vocab) <= kDecL2RowBudget;
+    };
     int ns = 1;
-    while (ns < 8 && ns < want && int64_t(vocab) / (2 * ns) >= 2048) ns *= 2;
+    while (ns < 8 && (ns < want || !fits(ns)) && int64_t(vocab) / (2 * ns) >= 2048) ns *= 2;
     n_split = ns;
     chunk = int((int64_t(vocab) / 8 + ns - 1) / ns * 8);
     return true;
@@ -738,7 +752,10 @@ extern "C" dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_
     P.status = reinterpret_cast<uint32_t*>(ws);
     P.vec = (ld % 8 == 0) && (ld_out % 8 == 0) && aligned16(logits) && aligned16(dlogits);
     int cl_split = 0, cl_chunk = 0;
-    if (n_slots > 0 && P.vec && dec_cluster_plan(n_slots, vocab, cl_split, cl_chunk)) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (n_slots > 0 && P.vec && dec_cluster_plan(n_slots, vocab, sms, cl_split, cl_chunk)) {
         // one cluster per slot: lse partials through distributed shared memory
         P.err = reinterpret_cast<uint32_t*>(ws + plan.partial_off);   // n_slots x cl_split words fit
         DecParams C = P;

@@ -111,6 +111,7 @@ def test_decision_full_workload(label_softmax):
     (3, 16, 16, 16, 0, 3),        # every token of the vocabulary an answer
     (4, 300000, 2, 26, 0, 4),     # long rows: clusters of 8 CTAs of 37,500 columns
     (6, 8192, 33, 128, 0, 5),     # the cluster path with more than one group of 32 answers
+    (1024, 65536, 2, 26, 0, 8),   # clusters of 2 (rows in flight kept within L2), several waves
 ])
 def test_decision_elementwise(n, V, kmin, kmax, ld_pad, seed):
     off, ids, kind, val = _batch(seed, n, V, kmax, kmin=kmin)
