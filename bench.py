@@ -272,6 +272,12 @@ def run_ours(args):
     recs = []
     for i, key in enumerate(keys):
         spec = di.WORKLOADS[key]
+        if args.slots and spec.kind == "decision":
+            # the same recipe on another number of label slots
+            spec = spec.scaled(key=key.replace(f"_s{spec.n_units}_", f"_s{args.slots}_"), n_units=args.slots,
+                               description=spec.description.replace(
+                                   f"{spec.n_units} label slots (16 canvases x 8 questions)",
+                                   f"{args.slots} label slots"))
         run = {"linear": run_linear, "decision": run_decision}.get(spec.kind, run_logits)
         if i == 0 or world > 1:
             recs.append(run(args, spec, dev, rank, world, headline=(i == 0)))
@@ -720,7 +726,8 @@ def run_decision(args, spec, dev, rank, world, headline=True):
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": spec.key, "description": spec.description, "label_slots": n, "vocab": V,
                        "parallelism": f"replicas{world}", "label_softmax": "both", "brier_weight": 0.1,
-                       "l2": "eight input sets used in turn (8 x 32 MB of logits, larger than L2)",
+                       "l2": f"eight input sets used in turn (8 x {n * V * 2 / 1e6:.0f} MB of logits, "
+                             f"{'larger' if 8 * n * V * 2 > 126e6 else 'smaller'} than L2)",
                        "timing": "steps run from one CUDA graph of all timed calls (no host gap between calls); "
                                  "steps rounded up to a multiple of eight",
                        "unit_note": "scored tokens = label slots"},
@@ -1045,7 +1052,11 @@ def main():
                     help="fused-head workloads: targets aligned (row i scores token i) or shifted (token i+1)")
     ap.add_argument("--objective", choices=["plain", "rhine"], default="plain",
                     help="uniform-noise workloads: plain canvas mean, or the Rhine objective options")
+    ap.add_argument("--slots", type=int, default=0,
+                    help="typed-decision workloads: label slots per call (default: the workload's 128)")
     args = ap.parse_args()
+    if args.slots < 0 or args.slots > 65535:
+        raise SystemExit("--slots must be in 0..65535")
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
