@@ -509,8 +509,13 @@ __device__ __forceinline__ uint4 ldg_v4_hint(const void* p, uint64_t pol) {
 // no CTA waits for a second wave (holding each split in shared memory
 // instead measured slower: the call's rows do not fit on chip at once).
 // The final cluster barrier keeps every CTA's partials alive until all
-// peers have read them.
-__global__ void __launch_bounds__(kDecThreads, 4) k_dec_cluster(DecParams P) {
+// peers have read them.  MINB = CTAs resident per SM (the launch bound): 4
+// (58 registers) when the call's CTAs fit on the chip at once, 5 (48) when
+// they come in waves -- more CTAs streaming while others sit in their
+// barriers and tails (1,024 and 2,048 slots: 0.76 -> 0.80, 0.78 -> 0.83 of
+// HBM; on 128 slots 5 was 1% slower).
+template <int MINB>
+__global__ void __launch_bounds__(kDecThreads, MINB) k_dec_cluster(DecParams P) {
     constexpr int kU = DLM_DEC_CU;     // 16-byte loads in flight per thread, first read
     constexpr int kU2 = DLM_DEC_CU2;   // the same, second read
     __shared__ __align__(8) float2 s_part[kDecThreads / 32];   // (max, sum exp) per warp
@@ -645,18 +650,20 @@ struct DecPlan {
 // of a small call resident at once) and keeps the rows in flight -- the
 // resident CTAs' rows, each read twice -- within an L2 budget, without
 // cutting splits under 2,048 columns.  The second read must find its row in
-// L2: on 2,048 slots of V = 126,464, one CTA per row (150 MB in flight) ran
-// at 0.66 of HBM, two (75 MB) at 0.78, four (37 MB) at 0.80, eight at 0.60
-// (per-CTA overheads).  Needs vocab % 8 == 0 (16-byte vectors).
-constexpr int kDecCtasPerSm = 4;             // k_dec_cluster's launch bound
+// L2: on 2,048 slots of V = 126,464 at four CTAs per SM, one CTA per row
+// (150 MB in flight) ran at 0.66 of HBM, two (75 MB) at 0.78, four (37 MB)
+// at 0.80, eight at 0.60 (per-CTA overheads); 50 MB keeps four per row at
+// five CTAs per SM too (47 MB).  Needs vocab % 8 == 0 (16-byte vectors).
+constexpr int kDecOneWaveCtasPerSm = 4;      // k_dec_cluster<4>: calls whose CTAs fit at once
+constexpr int kDecWaveCtasPerSm = 5;         // k_dec_cluster<5>: calls that come in waves
 #ifndef DLM_DEC_L2_BUDGET
-#define DLM_DEC_L2_BUDGET 40e6
+#define DLM_DEC_L2_BUDGET 50e6
 #endif
 constexpr double kDecL2RowBudget = DLM_DEC_L2_BUDGET;   // bytes of rows in flight between the two reads
 inline bool dec_cluster_plan(int n_slots, int vocab, int sms, int& n_split, int& chunk) {
     if (n_slots <= 0 || vocab % 8 != 0) return false;
     const int64_t want = (512 + n_slots - 1) / n_slots;   // CTAs wanted per slot
-    const int64_t resident = int64_t(sms > 0 ? sms : 148) * kDecCtasPerSm;
+    const int64_t resident = int64_t(sms > 0 ? sms : 148) * kDecWaveCtasPerSm;
     auto fits = [&](int ns) {
         const int64_t rows = resident / ns < n_slots ? resident / ns : n_slots;
         return double(rows) * 2.0 * double(vocab) <= kDecL2RowBudget;
@@ -775,7 +782,9 @@ extern "C" dlm_status_t dlm_decision_loss_fwd_bwd(int32_t n_slots, const uint16_
         at[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = at;
         cfg.numAttrs = 2;
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, k_dec_cluster, C);
+        const bool one_wave = int64_t(n_slots) * cl_split <= int64_t(sms) * kDecOneWaveCtasPerSm;
+        const cudaError_t e = one_wave ? cudaLaunchKernelEx(&cfg, k_dec_cluster<kDecOneWaveCtasPerSm>, C)
+                                       : cudaLaunchKernelEx(&cfg, k_dec_cluster<kDecWaveCtasPerSm>, C);
         if (e != cudaSuccess) { cudaGetLastError(); return cuda_status(e, "k_dec_cluster launch"); }
     } else if (n_slots > 0) {
         const dim3 grid(unsigned(plan.n_split), unsigned(n_slots));
