@@ -243,6 +243,34 @@ def test_decision_most_slots_one_call():
                                                    np.concatenate([val, [1.0]]).astype(np.float32)))
 
 
+def test_decision_concurrent_streams():
+    """Calls with their own workspaces on two streams at once (one of them
+    a multi-wave call, the other the one-wave kernel) give the serial
+    results bit for bit."""
+    base = di.WORKLOADS["dec_s128_k26_v126464"]
+    specs = [base, base.scaled(n_units=700)]
+    cases = [di.make_case(sp, "cuda", seed=20 + i) for i, sp in enumerate(specs)]
+
+    def run(i):
+        e = cases[i].extra
+        return dlm.decision_loss_fwd_bwd(cases[i].logits, specs[i].vocab, e["cand_off"], e["cand_ids"], e["kind"],
+                                         e["val"])
+
+    serial = [run(0), run(1)]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    conc = [None, None]
+    for _ in range(3):
+        for i, st in enumerate(streams):
+            with torch.cuda.stream(st):
+                conc[i] = run(i)
+        torch.cuda.synchronize()
+        for a, b in zip(serial, conc):
+            assert torch.equal(a.loss, b.loss)
+            assert torch.equal(a.dlogits.view(torch.int16), b.dlogits.view(torch.int16))
+            assert b.device_status() == 0
+
+
 def test_decision_no_slots_and_reproducible():
     V = 1024
     z = torch.zeros((0, V), dtype=torch.bfloat16, device="cuda")
