@@ -993,6 +993,42 @@ def cpu_baseline(spec, budget_s=15.0, min_steps=3, max_steps=100_000, single_thr
     return res
 
 
+def _decision_reference(args, spec, world):
+    """The reference arm on a typed-decision workload: each step one run of
+    the decision oracle over every label slot of the workload."""
+    import dlm_inputs as di
+    import oracle
+
+    if args.slots:
+        spec = spec.scaled(key=spec.key.replace(f"_s{spec.n_units}_", f"_s{args.slots}_"), n_units=args.slots)
+    case = di.make_case(spec, "cpu")
+    e = {k: v.numpy() for k, v in case.extra.items()}
+    x = di.bf16_bits(case.logits)
+
+    def step():
+        oracle.decision_loss(x, spec.vocab, None, e["cand_off"], e["cand_ids"], e["kind"], e["val"])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    val = spec.n_units * args.steps / dt
+    sample = (f"each step: the whole workload ({spec.n_units} label slots, V = {spec.vocab}; the three terms "
+              f"and the double-precision gradient of every logit)")
+    print(json.dumps({"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+                      "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+                      "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                      "data": "synthetic",
+                      "config": {"workload": spec.key, "description": spec.description,
+                                 "label_slots": spec.n_units, "vocab": spec.vocab, "parallelism": "cpu"},
+                      "cpu_baseline": {"value": val, "unit": UNIT, "cores": _oracle_threads(), "kind": "oracle",
+                                       "sample": sample},
+                      "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+          flush=True)
+
+
 def run_reference(args):
     """The reference arm: the CPU oracle as it stands, on the machine's host
     cores, each step a bounded sample of the workload sized so that the
@@ -1003,6 +1039,9 @@ def run_reference(args):
     import dlm_inputs as di
 
     spec = di.WORKLOADS[SUITE_HEADLINE if args.workload == SUITE else args.workload]
+    if spec.kind == "decision":
+        _decision_reference(args, spec, world)
+        return
     need = oracle_host_bytes(spec, 1024)
     if need > 0.6 * __import__("psutil").virtual_memory().available:
         print(json.dumps({"impl": "reference",

@@ -70,6 +70,19 @@ def test_reference_arm_prints_on_rank0_only():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["n_gpus"] == 2
 
 
+def test_reference_arm_on_typed_decisions():
+    """The reference arm on the typed-decision workload (label slots
+    scaled down): the decision oracle over every slot, one line."""
+    env = dict(os.environ, RANK="0", LOCAL_RANK="0", WORLD_SIZE="1", OMP_NUM_THREADS="2")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "dec_s128_k26_v126464", "--slots", "8", "--steps", "3", "--warmup", "3"],
+                       capture_output=True, text=True, env=env, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["config"]["label_slots"] == 8
+    assert line["config"]["workload"] == "dec_s8_k26_v126464" and line["cpu_baseline"]["kind"] == "oracle"
+
+
 def test_cpu_baseline_all_cores_and_one_thread():
     """The CPU baseline: the oracle on a bounded sample for about its time
     budget, then again on one thread in a child process."""
