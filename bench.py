@@ -58,6 +58,7 @@ DEFAULT_WORKLOAD = SUITE
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 CE_SOURCE = os.path.join(ROOT, "diffusion_lm_loss_b200", "csrc", "dlm_ce.cu")
+DEC_SOURCE = os.path.join(ROOT, "diffusion_lm_loss_b200", "csrc", "dlm_decision.cu")
 ABSORBING, UNIFORM = 0, 1          # noise modes, as numbered in include/dlm.h
 
 
@@ -76,20 +77,25 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def ce_traffic_ratio(workload: str):
-    """DRAM bytes / algorithmic bytes of the CE kernel on `workload` from its
-    committed ncu summary (profiles/ce_stream_<workload>.md), or None when
-    there is none or the kernel source changed since the capture."""
+def profile_traffic_ratio(name: str, source: str):
+    """DRAM bytes / algorithmic bytes of a kernel from its committed ncu
+    summary (profiles/<name>.md), or None when there is none or the kernel's
+    source file changed since the capture."""
     try:
-        txt = open(os.path.join(ROOT, "profiles", f"ce_stream_{workload}.md")).read()
+        txt = open(os.path.join(ROOT, "profiles", f"{name}.md")).read()
     except OSError:
         return None
     m_sha = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
     m_r = re.search(r"traffic_over_algorithmic:\s*([0-9.]+)", txt)
     if not (m_sha and m_r):
         return None
-    sha = hashlib.sha256(open(CE_SOURCE, "rb").read()).hexdigest()
+    sha = hashlib.sha256(open(source, "rb").read()).hexdigest()
     return float(m_r.group(1)) if sha == m_sha.group(1) else None
+
+
+def ce_traffic_ratio(workload: str):
+    """The CE kernel's ratio on `workload` (profiles/ce_stream_<workload>.md)."""
+    return profile_traffic_ratio(f"ce_stream_{workload}", CE_SOURCE)
 
 
 # ---------------------------------------------------------------------------
@@ -713,8 +719,11 @@ def run_decision(args, spec, dev, rank, world, headline=True):
                "d2h_bytes_per_step": 4, "steps": Ke, "ms_per_step": float(e_ms[0]) / Ke}
     hbm, _, peak_kind = peaks()
     alg = 4.0 * n * V + 8.0 * n
+    # DRAM bytes of the cluster kernel per call, from its committed capture
+    # (the gradient it writes is still in L2 when the kernel ends)
+    ratio = profile_traffic_ratio(f"dec_cluster_{spec.key}", DEC_SOURCE)
     roof = {"bound": "hbm", "achieved": alg / (call_ms / 1e3) / 1e9, "peak": hbm, "unit": "GB/s",
-            "frac": alg / (call_ms / 1e3) / 1e9 / hbm, "traffic": None,
+            "frac": alg / (call_ms / 1e3) / 1e9 / hbm, "traffic": ratio * alg if ratio else None,
             "kernel": "k_dec_cluster + k_dec_reduce (timed as the whole dlm_decision_loss_fwd_bwd call)",
             "algorithmic_bytes_per_launch": alg, "launch_ms": call_ms,
             "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)"}
