@@ -453,9 +453,11 @@ DLM_API dlm_status_t dlm_selftest_bounded_wait(uint64_t limit_ns, uint32_t *dev_
  *       256-byte aligned; its status word is read by dlm_get_device_status.
  * Errors: n_slots outside 0..DLM_DECISION_MAX_SLOTS, vocab <= 0, a bad
  * label_softmax, a negative or non-finite brier_weight, smoothing outside
- * [0, 1], a null pointer, ld / ld_out < vocab, n_rows < 1 (or < n_slots
- * without slot_rows) or n_cands < 0 return DLM_ERR_INVALID_ARGUMENT before
- * anything is enqueued.  On the device, a slot whose row is outside
+ * [0, 1], a non-finite grad_scale, a null pointer, ld / ld_out < vocab,
+ * n_rows < 1 (or < n_slots without slot_rows), n_cands < 0 or a workspace
+ * that is not 256-byte aligned return DLM_ERR_INVALID_ARGUMENT, and a
+ * workspace smaller than dlm_decision_workspace_size() returns
+ * DLM_ERR_WORKSPACE_TOO_SMALL, before anything is enqueued.  On the device, a slot whose row is outside
  * [0, n_rows) or whose answer offsets leave 0..n_cands sets
  * DLM_DEV_BAD_LAYOUT; an answer id outside [0, vocab) sets
  * DLM_DEV_BAD_TOKEN_ID; K outside 1..128, repeated answer ids, an unknown
